@@ -1,0 +1,409 @@
+"""Benchmark of attention over a cross-layer shared KV cache on B200.
+
+Default workload (one step = one decode step over all 22 layers of the
+1.1B-shaped CLA2 model: 32 q / 4 kv heads, d 64, bf16, batch 32, context
+2048). Secondary lines time the DepthGraft pair-mix decode (24 layers, 16/4
+heads, d 128, batch 16, context 8192).
+
+Timing: W untimed warm-up steps, then K timed steps between a barrier +
+synchronize on both sides. Every layer launch is bracketed by CUDA events on
+the launching stream; L2 (126 MB) is flushed by writing a 2x-L2 buffer before
+every layer, outside the events, so shared-source layers re-read HBM as a real
+model would after its MLP. Step time = sum of per-layer event times; max over
+ranks. `e2e` times the host-buffer entry point (q H2D, decode, out D2H).
+
+--impl reference times the fp64 CPU oracle (the reference arm) on a bounded
+sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from synth.configs import BY_NAME  # noqa: E402
+
+METRIC = "decode tok/s and KV GB/s (% of HBM peak); prefill TFLOP/s, 1×B200"
+
+# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel,
+# for the kernel as currently built (None until captured for this build)
+NCU_TRAFFIC_BYTES = {"cla2_1p1b": None}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def decode_read_bytes(cfg, l):
+    """Algorithmic bytes one decode layer reads: its source(s)' K and V."""
+    kind = cfg.layer_map[l][0]
+    nsrc = 2 if kind == 1 else 1
+    es = 4 if cfg.dtype == "f32" else 2
+    return nsrc * 2 * cfg.batch * cfg.kv_heads * cfg.context * cfg.head_dim * es
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(r[1]) for r in self.rows if len(r) > 8 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) > 8 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.rows)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+class DecodeRunner:
+    def __init__(self, cfg, K, torch, sgpu):
+        self.cfg, self.K, self.torch = cfg, K, torch
+        self.dev = {n: sgpu.make_device(cfg, n) for n in cfg.recipe()}
+        self.w = cfg.make("w")
+        _, self.h = K.kvshare_create(cfg.layers, cfg.q_heads, cfg.kv_heads, cfg.head_dim,
+                                     K.KVS_F32 if cfg.dtype == "f32" else K.KVS_BF16, cfg.batch, cfg.context)
+        K.kvshare_set_map(self.h, cfg.layer_map, self.w)
+        self.out = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim, device="cuda")
+        self.lse = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, device="cuda")
+        self.cache = K.Cache(batch=cfg.batch, context=cfg.context, k=self.dev["k"], v=self.dev["v"], slots=cfg.slots)
+        self.stream = torch.cuda.current_stream()
+        l2 = torch.cuda.get_device_properties(0).L2_cache_size
+        self.flush_buf = torch.empty(2 * l2, dtype=torch.int8, device="cuda")
+
+    def flush(self):
+        self.flush_buf.fill_(1)
+
+    def layer(self, l):
+        self.K.kvshare_decode(self.h, self.cache, self.dev["q"], self.out, self.lse, l, l + 1, self.stream)
+
+    def step_flushed(self, events=None):
+        torch = self.torch
+        for l in range(self.cfg.layers):
+            self.flush()
+            if events is not None:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(self.stream)
+                self.layer(l)
+                e1.record(self.stream)
+                events.append((l, e0, e1))
+            else:
+                self.layer(l)
+
+    def close(self):
+        self.K.kvshare_destroy(self.h)
+
+
+def gpu_arm(args, cfg_name, secondary=False):
+    import torch
+    import synth.gpu as sgpu
+    from cross_layer_kv_shared_b200 import kvshare as K
+
+    cfg = BY_NAME[cfg_name]
+    r = DecodeRunner(cfg, K, torch, sgpu)
+    for _ in range(args.warmup):
+        r.step_flushed()
+    torch.cuda.synchronize()
+    if dist_on():
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = K.kvshare_launch_count(r.h)
+    events = []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_wall = time.perf_counter()
+        for _ in range(args.steps):
+            r.step_flushed(events)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if dist_on():
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches = K.kvshare_launch_count(r.h) - n0
+    st = K.kvshare_sync_status(r.h)
+    assert st == K.KVS_OK, K.kvshare_status_string(st)
+    per_layer = np.zeros(cfg.layers)
+    for l, e0, e1 in events:
+        per_layer[l] += e0.elapsed_time(e1)
+    per_layer /= args.steps                       # ms per layer launch
+    step_ms = float(per_layer.sum())
+    step_ms = max_over_ranks(step_ms)
+
+    # no-flush, back-to-back step (one call for all layers): L2 may serve shared sources
+    torch.cuda.synchronize()
+    nf = []
+    for _ in range(max(3, args.steps // 2)):
+        r.flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(r.stream)
+        K.kvshare_decode(r.h, r.cache, r.dev["q"], r.out, r.lse, 0, cfg.layers, r.stream)
+        e1.record(r.stream)
+        nf.append((e0, e1))
+    torch.cuda.synchronize()
+    nf_ms = statistics.median([a.elapsed_time(b) for a, b in nf])
+
+    # e2e through the host-buffer entry point: q H2D + decode + out/lse D2H
+    q_host = r.dev["q"].cpu().pin_memory()
+    out_host = torch.empty(r.out.shape, dtype=torch.float32).pin_memory()
+    lse_host = torch.empty(r.lse.shape, dtype=torch.float32).pin_memory()
+    e2e = []
+    for i in range(args.warmup + args.steps):
+        r.flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(r.stream)
+        K.kvshare_decode_host(r.h, r.cache, q_host, out_host, lse_host, 0, cfg.layers, r.stream)
+        e1.record(r.stream)
+        if i >= args.warmup:
+            e2e.append((e0, e1))
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in e2e]))
+
+    read_bytes = sum(decode_read_bytes(cfg, l) for l in range(cfg.layers))
+    res = {
+        "cfg": cfg, "step_ms": step_ms, "per_layer_ms": per_layer, "launches": launches,
+        "kv_gbs": read_bytes / (step_ms * 1e-3) / 1e9, "tok_s": cfg.batch / (step_ms * 1e-3),
+        "no_flush_ms": nf_ms, "e2e_ms": e2e_ms, "wall_s": t_wall, "clocks": clk.summary(),
+        "h2d": q_host.numel() * q_host.element_size(),
+        "d2h": out_host.numel() * 4 + lse_host.numel() * 4,
+        "read_bytes": read_bytes,
+    }
+    r.close()
+    del r
+    torch.cuda.empty_cache()
+    return res
+
+
+def dist_on():
+    return int(os.environ.get("WORLD_SIZE", "1")) > 1
+
+
+def max_over_ranks(x: float) -> float:
+    if not dist_on():
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arm
+def oracle_sample(cfg, seconds: float, rng_seed: int = 0, distinct: int = 4):
+    """Time the fp64 oracle on (layer, batch) units of the workload for about ``seconds``.
+
+    ``distinct`` units are drawn outside the timed region and evaluated in turn
+    until the budget is spent. Returns (seconds per unit, units, threads).
+    """
+    from oracle import kvshare_ref as ref
+    w = cfg.make("w")
+    rng = np.random.default_rng(rng_seed)
+    pool = []
+    for _ in range(distinct):
+        l = int(rng.integers(cfg.layers))
+        b = int(rng.integers(cfg.batch))
+        kind, s0, s1 = cfg.layer_map[l]
+        store = {}
+        for s in [s0] + ([s1] if kind == 1 else []):
+            store[("k", s)] = cfg.make("k", (s, b))
+            store[("v", s)] = cfg.make("v", (s, b))
+        pool.append((l, b, store, cfg.make("q", (l, b))))
+    timed = 0.0
+    units = 0
+    g = cfg.group
+    while timed < seconds and units < 100000:
+        l, b, store, qlb = pool[units % distinct]
+
+        def get(name, index, store=store):
+            return ref.to_f64(store[(name, index[0])][index[2]], cfg.dtype)
+        t0 = time.perf_counter()
+        for j in range(cfg.kv_heads):
+            ref.decode_head_group(cfg.layer_map, l, b, j, ref.to_f64(qlb[j * g:(j + 1) * g], cfg.dtype), get, w=w)
+        timed += time.perf_counter() - t0
+        units += 1
+    return timed / units, units, blas_threads()
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, seconds=12.0):
+    per_unit, units, threads = oracle_sample(cfg, seconds)
+    step_s = per_unit * cfg.layers * cfg.batch
+    return {"value": cfg.batch / step_s, "unit": "tok/s", "cores": threads, "kind": "oracle",
+            "sample": f"{units} (layer, batch) units of {cfg.name}, fp64 numpy, extrapolated to "
+                      f"{cfg.layers} layers x {cfg.batch} batch"}
+
+
+def reference_arm(args):
+    cfg = BY_NAME[args.config]
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(cfg, 0.2, rng_seed=1, distinct=1)
+    times = []
+    units_total = 0
+    threads = 1
+    for s in range(args.steps):
+        per_unit, units, threads = oracle_sample(cfg, 2.0, rng_seed=100 + s, distinct=2)
+        times.append(per_unit * cfg.layers * cfg.batch)
+        units_total += units
+    step_s = statistics.median(times)
+    val = cfg.batch / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tok/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox, N(0,1))",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "context": cfg.context, "layers": cfg.layers,
+                   "q_heads": cfg.q_heads, "kv_heads": cfg.kv_heads, "head_dim": cfg.head_dim},
+        "cpu_baseline": {"value": val, "unit": "tok/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{units_total} (layer, batch) units over {args.steps} steps, extrapolated"},
+        "e2e": {"value": val, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvshare", choices=["kvshare", "reference"])
+    ap.add_argument("--config", default="cla2_1p1b")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    hbm_peak, bf16_peak, bf16_sust, peak_src = load_peaks()
+    main_res = gpu_arm(args, args.config)
+    cfg = main_res["cfg"]
+    sec = {}
+    if not args.no_secondary:
+        for name in ("depthgraft_decode",):
+            if name == args.config:
+                continue
+            r2 = gpu_arm(argparse.Namespace(steps=max(5, args.steps // 2), warmup=3), name)
+            sec[name] = {"tok_s": r2["tok_s"] * world, "kv_gbs": r2["kv_gbs"],
+                         "hbm_frac": r2["kv_gbs"] / hbm_peak, "ms_per_step": r2["step_ms"],
+                         "no_flush_ms_per_step": r2["no_flush_ms"], "gpu_launches": r2["launches"]}
+    avg_launch_ms = float(np.mean(main_res["per_layer_ms"]))
+    per_launch_bytes = decode_read_bytes(cfg, 0)
+    achieved = per_launch_bytes / (avg_launch_ms * 1e-3) / 1e9
+    traffic = NCU_TRAFFIC_BYTES.get(cfg.name)
+    line = {
+        "metric": METRIC,
+        "value": main_res["tok_s"] * world,
+        "unit": "tok/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": main_res["step_ms"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded Philox, N(0,1)/8 q/k/v)",
+        "config": {"workload": cfg.name, "layers": cfg.layers, "batch_per_gpu": cfg.batch, "context": cfg.context,
+                   "q_heads": cfg.q_heads, "kv_heads": cfg.kv_heads, "head_dim": cfg.head_dim,
+                   "layer_map": "CLA2: layer l reads slot l//2", "parallelism": f"replicas x{world}",
+                   "l2": "flushed (2x L2 write) before every layer, outside the timed events"},
+        "kv_gbs": main_res["kv_gbs"],
+        "hbm_frac": main_res["kv_gbs"] / hbm_peak,
+        "no_flush_ms_per_step": main_res["no_flush_ms"],
+        "gpu_launches": main_res["launches"],
+        "clocks": main_res["clocks"],
+        "e2e": {"value": cfg.batch * world / (main_res["e2e_ms"] * 1e-3), "unit": "tok/s",
+                "h2d_bytes_per_step": main_res["h2d"], "d2h_bytes_per_step": main_res["d2h"],
+                "ms_per_step": main_res["e2e_ms"]},
+        "roofline": {"kernel": "decode_bf16_kernel<64,single>", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": per_launch_bytes,
+                     "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"},
+        "secondary": sec,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

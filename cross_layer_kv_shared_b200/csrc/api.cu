@@ -1,0 +1,497 @@
+// Host side of libkvshare: argument validation, layer-table resolution,
+// split heuristic, TMA descriptors and kernel launches. See include/kvshare.h.
+#include "kvshare.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "kvs_internal.h"
+
+using namespace kvs;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+struct MapKey {
+    const void* ptr;
+    uint64_t d0, d1, d2;
+    uint32_t box0, box1;
+    int dtype;
+    bool operator==(const MapKey& o) const {
+        return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && box0 == o.box0 && box1 == o.box1 &&
+               dtype == o.dtype;
+    }
+};
+
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_device_ptr(const void* p) {
+    if (p == nullptr) return false;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+bool dev_ok(const void* p) { return p != nullptr && aligned16(p) && is_device_ptr(p); }
+
+}  // namespace
+
+struct kvshare_ctx {
+    kvshare_config cfg{};
+    int device = 0;
+    int sms = 148;
+    float scale = 0.f;
+    std::vector<kvshare_layer> map;
+    bool map_set = false;
+    float* w_dev = nullptr;          // [L][Hkv]
+    std::vector<float> w_host;
+    float* ws = nullptr;             // split partials
+    size_t ws_floats = 0;
+    unsigned* counters = nullptr;    // [max_batch * Hkv]
+    unsigned* err = nullptr;         // status word
+    int splits_override = 0;
+    int stall_next = 0;
+    long long wait_limit = 4000000000LL;     // ~2 s of SM clock
+    long long stall_limit = 20000000LL;      // ~10 ms
+    uint64_t launches = 0;
+    std::vector<MapEntry> maps;
+    // staging for kvshare_decode_host
+    void* q_stage = nullptr;
+    float* out_stage = nullptr;
+    float* lse_stage = nullptr;
+};
+
+namespace {
+
+size_t elem_size(kvshare_dtype t) { return t == KVS_F32 ? 4 : 2; }
+
+kvshare_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVS_OK : KVS_ECUDA; }
+
+// 3-D tiled map over a store [rows][T][D] with a box of {64, tt, 1}, 128-B swizzle.
+bool get_store_map(kvshare_ctx* c, const void* base, int D, int T, int rows, int tt, CUtensorMap* out) {
+    MapKey key{base, (uint64_t)D, (uint64_t)T, (uint64_t)rows, 64u, (uint32_t)tt, 0};
+    for (auto& e : c->maps)
+        if (e.key == key) {
+            *out = e.map;
+            return true;
+        }
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    CUtensorMap m;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)tt, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    if (c->maps.size() >= 64) c->maps.erase(c->maps.begin());
+    c->maps.push_back({key, m});
+    *out = m;
+    return true;
+}
+
+int choose_splits(const kvshare_ctx* c, int units, int tiles, int ctas_per_sm, int g, int D) {
+    int s;
+    if (c->splits_override > 0) {
+        s = c->splits_override;
+    } else {
+        const int resident = c->sms * ctas_per_sm;
+        s = resident / units;
+        if (s < 1) s = 1;
+    }
+    if (s > tiles) s = tiles;
+    if (s > MAX_SPLITS) s = MAX_SPLITS;
+    // workspace capacity: units * splits * g * (D + 2) floats
+    const size_t per_split = static_cast<size_t>(units) * g * (D + 2);
+    while (s > 1 && per_split * s > c->ws_floats) --s;
+    if (s < 1) s = 1;
+    return s;
+}
+
+kvshare_status validate_cache_common(const kvshare_ctx* c, const kvshare_cache* k) {
+    if (k == nullptr) return KVS_EINVAL;
+    if (k->batch < 1 || k->batch > c->cfg.max_batch) return KVS_EINVAL;
+    if (k->context < 1 || k->context > c->cfg.max_context) return KVS_EINVAL;
+    return KVS_OK;
+}
+
+kvshare_status check_layer_sources(const kvshare_ctx* c, const kvshare_cache* k, int l, bool* need_kv,
+                                   bool* need_lr) {
+    const kvshare_layer& e = c->map[l];
+    if (e.kind == KVS_SRC_SINGLE || e.kind == KVS_SRC_MIX) {
+        if (e.src0 < 0 || e.src0 >= k->slots) return KVS_EINVAL;
+        if (e.kind == KVS_SRC_MIX && (e.src1 < 0 || e.src1 >= k->slots)) return KVS_EINVAL;
+        *need_kv = true;
+    } else if (e.kind == KVS_SRC_LOWRANK) {
+        if (e.src0 < 0 || e.src0 >= k->pairs) return KVS_EINVAL;
+        *need_lr = true;
+    } else {
+        return KVS_EINVAL;
+    }
+    return KVS_OK;
+}
+
+kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void* q, float* out, float* lse,
+                             int l0, int l1, cudaStream_t st) {
+    const kvshare_config& cf = c->cfg;
+    const int D = cf.head_dim;
+    const int B = k->batch;
+    const int T = k->context;
+    const int Hq = cf.num_q_heads;
+    const int Hkv = cf.num_kv_heads;
+    const int g = Hq / Hkv;
+    const size_t es = elem_size(cf.dtype);
+    if (cudaSetDevice(c->device) != cudaSuccess) return KVS_ECUDA;
+
+    for (int l = l0; l < l1; ++l) {
+        const kvshare_layer& e = c->map[l];
+        DecodeArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.q = static_cast<const char*>(q) + static_cast<size_t>(l) * B * Hq * D * es;
+        a.out = out + static_cast<size_t>(l) * B * Hq * D;
+        a.lse = lse ? lse + static_cast<size_t>(l) * B * Hq : nullptr;
+        a.k = k->k;
+        a.v = k->v;
+        a.src0 = e.src0;
+        a.src1 = e.src1;
+        a.w = c->w_dev + static_cast<size_t>(l) * Hkv;
+        a.B = B;
+        a.Hq = Hq;
+        a.Hkv = Hkv;
+        a.T = T;
+        a.g = g;
+        a.scale_log2 = c->scale * 1.4426950408889634f;
+        a.ws = c->ws;
+        a.counters = c->counters;
+        a.err = c->err;
+        a.wait_limit = c->wait_limit;
+        a.stall = c->stall_next;
+        a.stall_limit = c->stall_limit;
+        c->stall_next = 0;
+        cudaError_t err;
+        if (cf.dtype == KVS_F32) {
+            if (e.kind == KVS_SRC_LOWRANK) return KVS_EUNSUPPORTED;
+            const int tt = decode_f32_tile();
+            const int tiles = (T + tt - 1) / tt;
+            int s = choose_splits(c, B * Hkv, tiles, 4, g, D);
+            a.tiles_per_split = (tiles + s - 1) / s;
+            a.splits = (tiles + a.tiles_per_split - 1) / a.tiles_per_split;
+            err = launch_decode_f32(e.kind == KVS_SRC_MIX, D, a, st);
+        } else if (e.kind == KVS_SRC_LOWRANK) {
+            return KVS_EUNSUPPORTED;
+        } else {
+            const bool mix = e.kind == KVS_SRC_MIX;
+            const TileShape ts = decode_bf16_shape(D, mix);
+            static int occ[2][2] = {{0, 0}, {0, 0}};
+            int& o = occ[D == 128][mix];
+            if (o == 0) o = decode_bf16_ctas_per_sm(D, mix);
+            const int tiles = (T + ts.tt - 1) / ts.tt;
+            int s = choose_splits(c, B * Hkv, tiles, o, g, D);
+            a.tiles_per_split = (tiles + s - 1) / s;
+            a.splits = (tiles + a.tiles_per_split - 1) / a.tiles_per_split;
+            CUtensorMap tmK, tmV;
+            const int rows = k->slots * B * Hkv;
+            if (!get_store_map(c, k->k, D, T, rows, ts.tt, &tmK) || !get_store_map(c, k->v, D, T, rows, ts.tt, &tmV))
+                return KVS_ECUDA;
+            err = launch_decode_bf16(D, mix, tmK, tmV, a, st);
+        }
+        if (err != cudaSuccess) return KVS_ECUDA;
+        ++c->launches;
+    }
+    return KVS_OK;
+}
+
+kvshare_status validate_decode(kvshare_ctx* c, const kvshare_cache* k, const void* q, const float* out,
+                               const float* lse, int l0, int l1, bool host_io) {
+    if (c == nullptr) return KVS_EINVAL;
+    if (!c->map_set) return KVS_EINVAL;
+    kvshare_status s = validate_cache_common(c, k);
+    if (s != KVS_OK) return s;
+    if (l0 < 0 || l1 > c->cfg.num_layers || l0 > l1) return KVS_EINVAL;
+    if (q == nullptr || out == nullptr) return KVS_EINVAL;
+    if (!aligned16(q) || !aligned16(out) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u))) return KVS_EINVAL;
+    if (!host_io && (!is_device_ptr(q) || !is_device_ptr(out) || (lse != nullptr && !is_device_ptr(lse))))
+        return KVS_EINVAL;
+    bool need_kv = false, need_lr = false;
+    for (int l = l0; l < l1; ++l) {
+        s = check_layer_sources(c, k, l, &need_kv, &need_lr);
+        if (s != KVS_OK) return s;
+        if (c->map[l].kind == KVS_SRC_LOWRANK && c->cfg.dtype != KVS_BF16) return KVS_EUNSUPPORTED;
+    }
+    if (need_kv) {
+        if (k->slots < 1 || !dev_ok(k->k) || !dev_ok(k->v)) return KVS_EINVAL;
+    }
+    if (need_lr) {
+        if (k->pairs < 1) return KVS_EINVAL;
+        const void* ps[] = {k->coef_k, k->coef_v, k->basis_k, k->basis_v, k->u_k, k->u_v,
+                            k->s_k, k->s_v, k->r_k, k->r_v, k->rank};
+        for (const void* p : ps)
+            if (!dev_ok(p)) return KVS_EINVAL;
+    }
+    return KVS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvshare_status kvshare_create(const kvshare_config* cfg, kvshare_t* out) {
+    if (out == nullptr) return KVS_EINVAL;
+    *out = nullptr;
+    if (cfg == nullptr) return KVS_EINVAL;
+    const kvshare_config& c = *cfg;
+    if (c.num_layers < 1 || c.num_q_heads < 1 || c.num_kv_heads < 1 || c.max_batch < 1 || c.max_context < 1)
+        return KVS_EINVAL;
+    if (c.num_q_heads % c.num_kv_heads != 0) return KVS_EINVAL;
+    if (c.dtype != KVS_F32 && c.dtype != KVS_BF16) return KVS_EINVAL;
+    if (!(c.softmax_scale >= 0.f) || std::isinf(c.softmax_scale)) return KVS_EINVAL;
+    if (c.head_dim != 64 && c.head_dim != 128) return KVS_EUNSUPPORTED;
+    if (c.num_q_heads / c.num_kv_heads > MAX_GROUP) return KVS_EUNSUPPORTED;
+    if (c.basis_rank != 0 && c.basis_rank != 32 && c.basis_rank != c.head_dim) return KVS_EUNSUPPORTED;
+    if (c.max_resid_rank != 0 && c.max_resid_rank != 16) return KVS_EUNSUPPORTED;
+
+    kvshare_ctx* ctx = new (std::nothrow) kvshare_ctx();
+    if (ctx == nullptr) return KVS_ENOMEM;
+    ctx->cfg = c;
+    if (ctx->cfg.basis_rank == 0) ctx->cfg.basis_rank = 32;
+    if (ctx->cfg.max_resid_rank == 0) ctx->cfg.max_resid_rank = 16;
+    ctx->scale = c.softmax_scale > 0.f ? c.softmax_scale : 1.0f / std::sqrt(static_cast<float>(c.head_dim));
+    if (cudaGetDevice(&ctx->device) != cudaSuccess) {
+        delete ctx;
+        return KVS_ECUDA;
+    }
+    cudaDeviceGetAttribute(&ctx->sms, cudaDevAttrMultiProcessorCount, ctx->device);
+    const int g = c.num_q_heads / c.num_kv_heads;
+    const size_t units = static_cast<size_t>(c.max_batch) * c.num_kv_heads;
+    const int max_tiles = (c.max_context + 15) / 16;
+    const int ms = max_tiles < MAX_SPLITS ? max_tiles : MAX_SPLITS;
+    ctx->ws_floats = units * ms * g * (c.head_dim + 2);
+    ctx->map.assign(c.num_layers, kvshare_layer{KVS_SRC_SINGLE, 0, 0});
+    ctx->w_host.assign(static_cast<size_t>(c.num_layers) * c.num_kv_heads, 1.0f);
+    if (cudaMalloc(&ctx->ws, ctx->ws_floats * sizeof(float)) != cudaSuccess ||
+        cudaMalloc(&ctx->counters, units * sizeof(unsigned)) != cudaSuccess ||
+        cudaMalloc(&ctx->err, sizeof(unsigned)) != cudaSuccess ||
+        cudaMalloc(&ctx->w_dev, ctx->w_host.size() * sizeof(float)) != cudaSuccess) {
+        cudaGetLastError();
+        kvshare_destroy(ctx);
+        return KVS_ENOMEM;
+    }
+    if (cudaMemset(ctx->counters, 0, units * sizeof(unsigned)) != cudaSuccess ||
+        cudaMemset(ctx->err, 0, sizeof(unsigned)) != cudaSuccess ||
+        cudaMemcpy(ctx->w_dev, ctx->w_host.data(), ctx->w_host.size() * sizeof(float), cudaMemcpyHostToDevice) !=
+            cudaSuccess) {
+        kvshare_destroy(ctx);
+        return KVS_ECUDA;
+    }
+    *out = ctx;
+    return KVS_OK;
+}
+
+kvshare_status kvshare_destroy(kvshare_t ctx) {
+    if (ctx == nullptr) return KVS_OK;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(ctx->device);
+    cudaFree(ctx->ws);
+    cudaFree(ctx->counters);
+    cudaFree(ctx->err);
+    cudaFree(ctx->w_dev);
+    cudaFree(ctx->q_stage);
+    cudaFree(ctx->out_stage);
+    cudaFree(ctx->lse_stage);
+    cudaSetDevice(prev);
+    delete ctx;
+    return KVS_OK;
+}
+
+kvshare_status kvshare_set_map(kvshare_t ctx, const kvshare_layer* map, const float* w) {
+    if (ctx == nullptr || map == nullptr) return KVS_EINVAL;
+    const int L = ctx->cfg.num_layers;
+    const int Hkv = ctx->cfg.num_kv_heads;
+    bool any_mix = false;
+    for (int l = 0; l < L; ++l) {
+        const kvshare_layer& e = map[l];
+        if (e.kind != KVS_SRC_SINGLE && e.kind != KVS_SRC_MIX && e.kind != KVS_SRC_LOWRANK) return KVS_EINVAL;
+        if (e.src0 < 0) return KVS_EINVAL;
+        if (e.kind == KVS_SRC_MIX) {
+            any_mix = true;
+            if (e.src1 < 0 || e.src1 == e.src0) return KVS_EINVAL;
+        }
+        if (e.kind == KVS_SRC_LOWRANK && ctx->cfg.dtype != KVS_BF16) return KVS_EUNSUPPORTED;
+    }
+    if (any_mix) {
+        if (w == nullptr) return KVS_EINVAL;
+        for (int l = 0; l < L; ++l) {
+            if (map[l].kind != KVS_SRC_MIX) continue;
+            for (int j = 0; j < Hkv; ++j) {
+                const float x = w[static_cast<size_t>(l) * Hkv + j];
+                if (!(x >= 0.f && x <= 1.f)) return KVS_EINVAL;
+            }
+        }
+    }
+    for (int l = 0; l < L; ++l) {
+        for (int j = 0; j < Hkv; ++j)
+            ctx->w_host[static_cast<size_t>(l) * Hkv + j] =
+                (map[l].kind == KVS_SRC_MIX) ? w[static_cast<size_t>(l) * Hkv + j] : 1.0f;
+    }
+    if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
+    if (cudaMemcpy(ctx->w_dev, ctx->w_host.data(), ctx->w_host.size() * sizeof(float), cudaMemcpyHostToDevice) !=
+        cudaSuccess)
+        return KVS_ECUDA;
+    ctx->map.assign(map, map + L);
+    ctx->map_set = true;
+    return KVS_OK;
+}
+
+kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const void* q, float* out, float* lse,
+                              int l0, int l1, void* stream) {
+    kvshare_status s = validate_decode(ctx, cache, q, out, lse, l0, l1, false);
+    if (s != KVS_OK) return s;
+    return decode_layers(ctx, cache, q, out, lse, l0, l1, static_cast<cudaStream_t>(stream));
+}
+
+kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, const void* q_host, float* out_host,
+                                   float* lse_host, int l0, int l1, void* stream) {
+    kvshare_status s = validate_decode(ctx, cache, q_host, out_host, lse_host, l0, l1, true);
+    if (s != KVS_OK) return s;
+    const kvshare_config& cf = ctx->cfg;
+    const size_t es = elem_size(cf.dtype);
+    const size_t per_layer = static_cast<size_t>(cf.max_batch) * cf.num_q_heads * cf.head_dim;
+    if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
+    if (ctx->q_stage == nullptr) {
+        if (cudaMalloc(&ctx->q_stage, per_layer * cf.num_layers * es) != cudaSuccess ||
+            cudaMalloc(&ctx->out_stage, per_layer * cf.num_layers * sizeof(float)) != cudaSuccess ||
+            cudaMalloc(&ctx->lse_stage, static_cast<size_t>(cf.max_batch) * cf.num_q_heads * cf.num_layers *
+                                            sizeof(float)) != cudaSuccess) {
+            cudaGetLastError();
+            return KVS_ENOMEM;
+        }
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t lay = static_cast<size_t>(cache->batch) * cf.num_q_heads * cf.head_dim;   // elements per layer
+    const size_t layh = static_cast<size_t>(cache->batch) * cf.num_q_heads;
+    const size_t nl = static_cast<size_t>(l1 - l0);
+    if (nl == 0) return KVS_OK;
+    cudaError_t e = cudaMemcpyAsync(static_cast<char*>(ctx->q_stage) + l0 * lay * es,
+                                    static_cast<const char*>(q_host) + l0 * lay * es, nl * lay * es,
+                                    cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return KVS_ECUDA;
+    s = decode_layers(ctx, cache, ctx->q_stage, ctx->out_stage, lse_host ? ctx->lse_stage : nullptr, l0, l1, st);
+    if (s != KVS_OK) return s;
+    e = cudaMemcpyAsync(out_host + l0 * lay, ctx->out_stage + l0 * lay, nl * lay * sizeof(float),
+                        cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess && lse_host != nullptr)
+        e = cudaMemcpyAsync(lse_host + l0 * layh, ctx->lse_stage + l0 * layh, nl * layh * sizeof(float),
+                            cudaMemcpyDeviceToHost, st);
+    return cuda_status(e);
+}
+
+kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const void* q, void* out, float* lse,
+                               int l0, int l1, int seqlen, void* stream) {
+    (void)cache; (void)q; (void)out; (void)lse; (void)l0; (void)l1; (void)seqlen; (void)stream;
+    if (ctx == nullptr) return KVS_EINVAL;
+    return KVS_EUNSUPPORTED;
+}
+
+kvshare_status kvshare_pack_residual(kvshare_t ctx, const float* score, const float* u_k, const float* u_v,
+                                     uint8_t* rank, int8_t* u_k8, int8_t* u_v8, uint16_t* s_k, uint16_t* s_v,
+                                     int batch, int context, void* stream) {
+    if (ctx == nullptr) return KVS_EINVAL;
+    if (batch < 1 || context < 1) return KVS_EINVAL;
+    if (ctx->cfg.max_resid_rank != 16) return KVS_EUNSUPPORTED;
+    const void* in[] = {score, u_k, u_v};
+    for (const void* p : in)
+        if (p == nullptr || !is_device_ptr(p)) return KVS_EINVAL;
+    if (!aligned16(u_k) || !aligned16(u_v) || (reinterpret_cast<uintptr_t>(score) & 3u)) return KVS_EINVAL;
+    const void* outp[] = {rank, u_k8, u_v8, s_k, s_v};
+    for (const void* p : outp)
+        if (p == nullptr || !is_device_ptr(p)) return KVS_EINVAL;
+    if (!aligned16(u_k8) || !aligned16(u_v8) || (reinterpret_cast<uintptr_t>(s_k) & 1u) ||
+        (reinterpret_cast<uintptr_t>(s_v) & 1u))
+        return KVS_EINVAL;
+    if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
+    PackArgs a;
+    a.score = score; a.u_k = u_k; a.u_v = u_v;
+    a.rank = rank; a.u_k8 = u_k8; a.u_v8 = u_v8; a.s_k = s_k; a.s_v = s_v;
+    a.tokens = static_cast<long long>(ctx->cfg.num_layers) * batch * context;
+    a.Hkv = ctx->cfg.num_kv_heads;
+    a.T = context;
+    a.Rm = 16;
+    cudaError_t e = launch_pack_residual(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return KVS_ECUDA;
+    ++ctx->launches;
+    return KVS_OK;
+}
+
+kvshare_status kvshare_sync_status(kvshare_t ctx, void* stream) {
+    if (ctx == nullptr) return KVS_EINVAL;
+    if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KVS_ECUDA;
+    unsigned word = 0;
+    if (cudaMemcpy(&word, ctx->err, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) return KVS_ECUDA;
+    if (word != 0) {
+        if (cudaMemset(ctx->err, 0, sizeof(unsigned)) != cudaSuccess) return KVS_ECUDA;
+        if (word & ERR_TIMEOUT) return KVS_ETIMEOUT;
+    }
+    return KVS_OK;
+}
+
+kvshare_status kvshare_set_splits(kvshare_t ctx, int splits) {
+    if (ctx == nullptr || splits < 0) return KVS_EINVAL;
+    ctx->splits_override = splits;
+    return KVS_OK;
+}
+
+kvshare_status kvshare_debug_stall_next(kvshare_t ctx, int on) {
+    if (ctx == nullptr) return KVS_EINVAL;
+    ctx->stall_next = on ? 1 : 0;
+    return KVS_OK;
+}
+
+uint64_t kvshare_launch_count(kvshare_t ctx) { return ctx ? ctx->launches : 0; }
+
+const char* kvshare_status_string(kvshare_status s) {
+    switch (s) {
+        case KVS_OK: return "ok";
+        case KVS_EINVAL: return "invalid argument";
+        case KVS_EUNSUPPORTED: return "unsupported configuration";
+        case KVS_ENOMEM: return "out of device memory";
+        case KVS_ECUDA: return "CUDA runtime error";
+        case KVS_ETIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

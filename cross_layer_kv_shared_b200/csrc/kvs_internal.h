@@ -1,0 +1,83 @@
+// Internal declarations shared by the host library and the kernels of libkvshare.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvs {
+
+// bits of the device status word
+constexpr unsigned ERR_TIMEOUT = 1u;
+
+// one split partial: o[d] (un-normalised, relative to m), m (log2 domain), l
+constexpr int MAX_SPLITS = 160;
+constexpr int MAX_GROUP = 16;
+
+// Arguments of one decode launch (one layer). Pointers are already offset to the layer.
+struct DecodeArgs {
+    const void* q;          // [B][Hq][d] config dtype
+    float* out;             // [B][Hq][d]
+    float* lse;             // [B][Hq] or nullptr
+    const void* k;          // store base [slots][B][Hkv][T][d] (used by the fp32 kernel)
+    const void* v;
+    int src0, src1;         // slots (SINGLE/MIX)
+    const float* w;         // [Hkv] mix weights of this layer (device), MIX only
+    int B, Hq, Hkv, T, g;
+    int splits;             // splits per (b, kv head)
+    int tiles_per_split;    // token tiles per split
+    float scale_log2;       // softmax scale * log2(e)
+    float* ws;              // split partials [B*Hkv][splits][g][d+2]
+    unsigned* counters;     // [B*Hkv] arrival counters, zero between launches
+    unsigned* err;          // device status word
+    long long wait_limit;   // clock cycles a bounded wait may spin
+    int stall;              // test hook: one warp waits on a barrier nothing arrives on
+    long long stall_limit;
+    // form (c)
+    int pair;               // basis pair
+    const void* coef_k; const void* coef_v;     // pair's [B][Hkv][T][Rb]
+    const void* basis_k; const void* basis_v;   // pair's [Hkv][Rb][d]
+    const int8_t* u_k; const int8_t* u_v;       // layer's [B][Hkv][T][Rm]
+    const uint16_t* s_k; const uint16_t* s_v;   // layer's [B][Hkv][T]
+    const void* r_k; const void* r_v;           // layer's [Hkv][Rm][d]
+    const uint8_t* rank;                        // layer's [B][T]
+    int Rb, Rm;
+};
+
+struct PackArgs {
+    const float* score; const float* u_k; const float* u_v;
+    uint8_t* rank; int8_t* u_k8; int8_t* u_v8; uint16_t* s_k; uint16_t* s_v;
+    long long tokens;       // L * B * T
+    int Hkv, T, Rm;
+};
+
+struct PrefillArgs {
+    const void* q;          // layer's [B][Hq][S][d] bf16
+    void* out;              // layer's [B][Hq][S][d] bf16
+    float* lse;             // layer's [B][Hq][S] or nullptr
+    int src0, src1, mix;
+    const float* w;         // [Hkv] (device) when mix
+    int B, Hq, Hkv, S, T, g;
+    float scale_log2;
+    unsigned* err;
+    long long wait_limit;
+};
+
+// kernel launchers (return cudaGetLastError() of the launch)
+struct TileShape { int tt; int nsw; int smem; };
+TileShape decode_bf16_shape(int d, bool mix);
+cudaError_t launch_decode_bf16(int d, bool mix, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                               const DecodeArgs& a, cudaStream_t st);
+int decode_bf16_ctas_per_sm(int d, bool mix);
+
+int decode_f32_tile();
+cudaError_t launch_decode_f32(bool mix, int d, const DecodeArgs& a, cudaStream_t st);
+
+TileShape decode_lowrank_shape();
+cudaError_t launch_decode_lowrank(const DecodeArgs& a, const CUtensorMap& tmCK, const CUtensorMap& tmCV,
+                                  cudaStream_t st);
+int decode_lowrank_ctas_per_sm();
+
+cudaError_t launch_pack_residual(const PackArgs& a, cudaStream_t st);
+
+}  // namespace kvs

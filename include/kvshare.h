@@ -1,0 +1,191 @@
+/*
+ * kvshare.h - C ABI of attention over a cross-layer shared KV cache (B200, sm_100a).
+ *
+ * What is computed. For every layer l, batch b and query head h (kv head
+ * j = h / g, g = num_q_heads / num_kv_heads, contiguous GQA groups), softmax
+ * attention of the query over K~, V~ with scale 1/sqrt(d), where K~, V~ are
+ * rebuilt from a shared cache through the layer table:
+ *
+ *   KVS_SRC_SINGLE   K~ = K[src0]                      - a layer reuses another
+ *                    layer's K/V ("Reducing Transformer Key-Value Cache Size with
+ *                    Cross-Layer Attention", Methodology: some layers compute
+ *                    K/V, the others reuse it; sharing factors CLA2/3/4).
+ *   KVS_SRC_MIX      K~ = w[l][j] K[src0] + (1 - w[l][j]) K[src1], same for V -
+ *                    a deep layer rebuilt from a stride-aligned shallow/middle
+ *                    source pair ("DepthGraft: Structural Regularization through
+ *                    Hierarchical Cross-Layer KV Reconstruction", Abstract; the
+ *                    page gives no operator, this convex mix is the reading used).
+ *   KVS_SRC_LOWRANK  K~_t = sum_{i<Rb} C_K[p][b][j][t][i] B_K[p][j][i][:]
+ *                         + s_K[l][b][j][t] sum_{i<r[l][b][t]} U_K[l][b][j][t][i] R_K[l][j][i][:]
+ *                    with p = src0, same for V - a layer pair shares a low-rank
+ *                    basis and each layer adds its own int8 low-rank residual at a
+ *                    per-token rank ("DepthWeave-KV: Smarter KV Cache Compression
+ *                    by Sharing Across Layers and Adapting Per Token", Core
+ *                    Mechanism and Framework Shift).
+ *
+ * Decode: the query attends to all `context` cached tokens. Prefill: query row i
+ * attends to tokens 0..i (causal, no earlier context).
+ *
+ * Conventions for every entry point
+ *   - Tensors are caller-owned DEVICE pointers (any allocator), dense and
+ *     row-major in the layouts given below, 16-byte aligned. The library never
+ *     frees them and keeps no reference after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued on it; no call synchronises except kvshare_sync_status.
+ *   - Every call validates its arguments on the host first and returns a status
+ *     without launching anything if they are invalid. Faults detected on the
+ *     device (a bounded wait that ran out) are recorded in a device word and
+ *     returned by the next kvshare_sync_status.
+ *   - One context per host thread at a time; calls on one context are not
+ *     thread-safe. Kernels of one context that overlap on the GPU (the same
+ *     context used on two streams at once) share its split workspace and race.
+ *   - bf16 and fp16 values travel as their 16-bit patterns (uint16_t or void*).
+ */
+#ifndef KVSHARE_H
+#define KVSHARE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct kvshare_ctx* kvshare_t;
+
+typedef enum {
+    KVS_OK = 0,
+    KVS_EINVAL = 1,        /* bad argument: null/misaligned pointer, shape, map entry, range */
+    KVS_EUNSUPPORTED = 2,  /* valid but not implemented (head_dim, dtype/kind combination)   */
+    KVS_ENOMEM = 3,        /* device allocation failed in kvshare_create                      */
+    KVS_ECUDA = 4,         /* a CUDA runtime call failed                                      */
+    KVS_ETIMEOUT = 5       /* a device-side bounded wait ran out (reported by sync_status)    */
+} kvshare_status;
+
+typedef enum { KVS_F32 = 0, KVS_BF16 = 1 } kvshare_dtype;
+
+typedef enum { KVS_SRC_SINGLE = 0, KVS_SRC_MIX = 1, KVS_SRC_LOWRANK = 2 } kvshare_kind;
+
+typedef struct {
+    int num_layers;        /* L                                                    */
+    int num_q_heads;       /* Hq, a multiple of num_kv_heads, Hq / Hkv <= 16       */
+    int num_kv_heads;      /* Hkv                                                  */
+    int head_dim;          /* d: 64 or 128                                         */
+    kvshare_dtype dtype;   /* storage type of q, k, v (form (c) is bf16 only)      */
+    float softmax_scale;   /* 0 selects 1/sqrt(d)                                  */
+    int basis_rank;        /* Rb of form (c): 32, or head_dim (full-rank basis)    */
+    int max_resid_rank;    /* Rm of form (c): must be 16                           */
+    int max_batch;         /* largest batch any call will use                      */
+    int max_context;       /* largest context any call will use                    */
+} kvshare_config;
+
+typedef struct {
+    kvshare_kind kind;
+    int src0;              /* store slot (SINGLE, MIX) or basis pair (LOWRANK)     */
+    int src1;              /* second store slot (MIX); ignored otherwise           */
+} kvshare_layer;
+
+/* The shared cache. Forms (a)/(b) use k, v, slots. Form (c) uses the rest.
+ * T below is `context`, the token count of every store.                        */
+typedef struct {
+    const void* k;         /* [slots][batch][Hkv][T][d]  dtype of the config     */
+    const void* v;         /* [slots][batch][Hkv][T][d]                          */
+    int slots;
+    const void* coef_k;    /* [pairs][batch][Hkv][T][Rb] bf16                    */
+    const void* coef_v;
+    const void* basis_k;   /* [pairs][Hkv][Rb][d] bf16                           */
+    const void* basis_v;
+    const int8_t* u_k;     /* [L][batch][Hkv][T][Rm] int8 residual codes         */
+    const int8_t* u_v;
+    const uint16_t* s_k;   /* [L][batch][Hkv][T] fp16 per-token residual scale   */
+    const uint16_t* s_v;
+    const void* r_k;       /* [L][Hkv][Rm][d] bf16 residual factor               */
+    const void* r_v;
+    const uint8_t* rank;   /* [L][batch][T] per-token residual rank, <= Rm       */
+    int pairs;
+    int batch;             /* 1 .. max_batch                                     */
+    int context;           /* 1 .. max_context                                   */
+} kvshare_cache;
+
+/* Create a context on the current CUDA device. Allocates the split workspace
+ * (sized by max_batch / max_context) and a device status word. `out` receives
+ * the handle; on failure it is set to NULL. */
+kvshare_status kvshare_create(const kvshare_config* cfg, kvshare_t* out);
+
+/* Free the context and everything it allocated. Safe with NULL. The caller
+ * must make sure no work of the context is still running. */
+kvshare_status kvshare_destroy(kvshare_t ctx);
+
+/* Install the layer table (HOST pointers; both are copied).
+ *   map: [num_layers] entries. SINGLE/MIX sources are store slots, LOWRANK src0
+ *        a basis pair; MIX needs src0 != src1. Slot/pair ranges are checked
+ *        against the cache at each decode/prefill call.
+ *   w:   [num_layers][num_kv_heads] mix weights in [0, 1]; may be NULL when no
+ *        entry is MIX. Rows of non-MIX layers are ignored. */
+kvshare_status kvshare_set_map(kvshare_t ctx, const kvshare_layer* map, const float* w);
+
+/* One decode step for layers [l0, l1), launched in layer order on `stream`.
+ *   q:   [L][batch][Hq][d] in the config dtype (layer l at offset l*batch*Hq*d)
+ *   out: [L][batch][Hq][d] fp32
+ *   lse: [L][batch][Hq] fp32 natural-log sum of exp of the scaled scores, or NULL
+ * Only rows of layers [l0, l1) are written. */
+kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const void* q,
+                              float* out, float* lse, int l0, int l1, void* stream);
+
+/* kvshare_decode with HOST buffers: copies q for layers [l0, l1) from
+ * `q_host` into a device staging buffer the context owns, decodes, and copies
+ * out/lse of those layers back to `out_host`/`lse_host` (same layouts as
+ * kvshare_decode, host memory; pinned memory makes the copies asynchronous).
+ * The cache stays on the device. Results are valid after the stream has
+ * synchronised. The staging buffers are allocated on the first call and reused. */
+kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, const void* q_host,
+                                   float* out_host, float* lse_host, int l0, int l1, void* stream);
+
+/* Causal prefill of `seqlen` tokens for layers [l0, l1) (bf16 only; SINGLE and
+ * MIX layers, LOWRANK gives KVS_EUNSUPPORTED). A MIX layer's K/V operands are
+ * mixed from its two source slots inside the kernel and never written to HBM.
+ *   q:   [L][batch][Hq][seqlen][d] bf16
+ *   out: [L][batch][Hq][seqlen][d] bf16
+ *   lse: [L][batch][Hq][seqlen] fp32 or NULL
+ * K/V rows 0..seqlen-1 of each store are used (seqlen <= context). */
+kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const void* q,
+                               void* out, float* lse, int l0, int l1, int seqlen, void* stream);
+
+/* Write side of form (c) for all L layers: rank routing and int8 quantisation.
+ *   score [L][batch][T] fp32 router score -> rank [L][batch][T]:
+ *         0 if score < 0.7f, 8 if score < 0.9f, else 16
+ *   u_k, u_v [L][batch][Hkv][T][16] fp32 residual rows ->
+ *   u_k8, u_v8 [L][batch][Hkv][T][16] int8 codes and s_k, s_v [L][batch][Hkv][T]
+ *         fp16 scales: amax = max_{i<r}|u_i|, scale = fp16_rne(min(amax/127f, 65504)),
+ *         code_i = clamp(rint(u_i / scale), -127, 127) for i < r, else 0;
+ *         a zero scale gives zero codes. fp32 IEEE arithmetic, bit-exact.
+ * Inputs must be finite. */
+kvshare_status kvshare_pack_residual(kvshare_t ctx, const float* score, const float* u_k,
+                                     const float* u_v, uint8_t* rank, int8_t* u_k8, int8_t* u_v8,
+                                     uint16_t* s_k, uint16_t* s_v, int batch, int context,
+                                     void* stream);
+
+/* Synchronise `stream`, then read and clear the device status word.
+ * Returns KVS_OK, KVS_ETIMEOUT (a bounded device wait ran out) or KVS_ECUDA. */
+kvshare_status kvshare_sync_status(kvshare_t ctx, void* stream);
+
+/* Split-KV override for decode: 0 = automatic (default), n > 0 = n splits per
+ * (batch, kv head), clamped to the number of token tiles and the workspace. */
+kvshare_status kvshare_set_splits(kvshare_t ctx, int splits);
+
+/* Test hook for the bounded waits: when `on` is non-zero, the next decode
+ * launch makes one warp wait on a barrier nothing arrives on, with a limit of
+ * about 10 ms; the wait gives up, records KVS_ETIMEOUT and the kernel still
+ * completes. The hook clears itself after one launch. */
+kvshare_status kvshare_debug_stall_next(kvshare_t ctx, int on);
+
+/* Number of kernels this context has launched since it was created. */
+uint64_t kvshare_launch_count(kvshare_t ctx);
+
+/* Static text for a status code. */
+const char* kvshare_status_string(kvshare_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVSHARE_H */

@@ -158,10 +158,32 @@ def normal_f64(n: int, offset: int, seed: int, stream: int) -> np.ndarray:
 
 
 def normal_f64_at(idx: np.ndarray, seed: int, stream: int) -> np.ndarray:
-    _, w0, w1, lane = _words_for(np.asarray(idx, dtype=np.uint64), seed, stream)
+    idx = np.asarray(idx, dtype=np.uint64)
+    if idx.size == 0:
+        return np.zeros(0)
+    blk = idx >> np.uint64(2)
+    b0, b1 = int(blk.min()), int(blk.max())
+    if 4 * (b1 - b0 + 1) <= 2 * idx.size + 64:
+        # dense request: one Philox call and one Box-Muller pair per block/pair
+        z = _normal_blocks(b0, b1 - b0 + 1, seed, stream)          # [nblk, 4]
+        return z[(blk - np.uint64(b0)).astype(np.int64), (idx & np.uint64(3)).astype(np.int64)]
+    _, w0, w1, lane = _words_for(idx, seed, stream)
     r = np.sqrt(-2.0 * series_log_u32(w0))
     cos_t, sin_t = series_sincos_u32(w1)
     return np.where((lane & 1) == 0, r * cos_t, r * sin_t)
+
+
+def _normal_blocks(first_blk: int, nblk: int, seed: int, stream: int) -> np.ndarray:
+    """Normals of all 4 elements of blocks [first_blk, first_blk + nblk): array [nblk, 4]."""
+    blk = np.arange(first_blk, first_blk + nblk, dtype=np.uint64)
+    w = philox4x32_10(blk & _MASK32, blk >> np.uint64(32), np.zeros_like(blk), np.zeros_like(blk), seed, stream)
+    out = np.empty((nblk, 4))
+    for p in range(2):
+        r = np.sqrt(-2.0 * series_log_u32(w[2 * p]))
+        cos_t, sin_t = series_sincos_u32(w[2 * p + 1])
+        out[:, 2 * p] = r * cos_t
+        out[:, 2 * p + 1] = r * sin_t
+    return out
 
 
 def f32_bits_to_bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -1,0 +1,65 @@
+"""Helpers shared by the GPU tests: upload seeded inputs, run the C ABI, run the oracle."""
+import numpy as np
+
+import oracle.kvshare_ref as ref
+
+
+def torch_mod():
+    import torch
+    return torch
+
+
+def to_dev(a, dtype_tag):
+    """numpy storage array -> CUDA tensor with the same bytes (bf16 patterns as int16)."""
+    torch = torch_mod()
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).cuda()
+
+
+def kv_dtype(cfg, K):
+    return K.KVS_F32 if cfg.dtype == "f32" else K.KVS_BF16
+
+
+def make_ctx(K, cfg, splits=0, max_batch=None, max_context=None):
+    _, h = K.kvshare_create(cfg.layers, cfg.q_heads, cfg.kv_heads, cfg.head_dim, kv_dtype(cfg, K),
+                            max_batch or cfg.batch, max_context or cfg.context,
+                            basis_rank=cfg.basis_rank, max_resid_rank=cfg.max_resid_rank)
+    if splits:
+        K.kvshare_set_splits(h, splits)
+    return h
+
+
+def decode_gpu(K, cfg, inp, splits=0, layers=None, dev_inputs=None, keep_ctx=False):
+    """Run kvshare_decode over all layers (or [l0, l1)) and return (out, lse) as numpy."""
+    torch = torch_mod()
+    d = dev_inputs if dev_inputs is not None else {n: to_dev(a, cfg.dtype) for n, a in inp.items()}
+    h = make_ctx(K, cfg, splits)
+    try:
+        K.kvshare_set_map(h, cfg.layer_map, inp.get("w") if inp is not None else None)
+        out = torch.full((cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim), float("nan"), device="cuda")
+        lse = torch.full((cfg.layers, cfg.batch, cfg.q_heads), float("nan"), device="cuda")
+        cache = K.Cache(batch=cfg.batch, context=cfg.context, k=d.get("k"), v=d.get("v"), slots=cfg.slots)
+        l0, l1 = layers if layers is not None else (0, cfg.layers)
+        K.kvshare_decode(h, cache, d["q"], out, lse, l0, l1)
+        st = K.kvshare_sync_status(h)
+        assert st == K.KVS_OK, K.kvshare_status_string(st)
+        launches = K.kvshare_launch_count(h)
+    finally:
+        K.kvshare_destroy(h)
+    return out.cpu().numpy(), lse.cpu().numpy(), launches
+
+
+def oracle_decode(cfg, inp, layers=None, batches=None):
+    get = lambda name, index: ref.to_f64(inp[name][index], cfg.dtype)  # noqa: E731
+    return ref.decode(cfg.layer_map, ref.to_f64(inp["q"], cfg.dtype), get, w=inp.get("w"),
+                      layers=layers, batches=batches)
+
+
+def assert_close(got, want, tol, what=""):
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = float(np.max(np.abs(got - want)))
+    rms = float(np.sqrt(np.mean(want ** 2))) or 1.0
+    assert err <= tol, f"{what}: max|d|={err:.3e} > {tol:.1e} (rel to rms {err / rms:.3e})"
+    return err, err / rms

@@ -1,0 +1,204 @@
+"""GPU parity of kvshare_decode (forms SINGLE and MIX) with the fp64 oracle, through the C ABI.
+
+Tolerances: max|d| <= 1e-4 for fp32 caches, <= 2e-2 for bf16 caches (the stated
+bars). Every test also reports the error relative to the output rms.
+"""
+import numpy as np
+import pytest
+
+from synth.configs import CLA2_1P1B, DEPTHGRAFT_DECODE, MIX, SINGLE, TINY_CLA2, Config
+import synth.gpu as sgpu
+
+from gpu_helpers import assert_close, decode_gpu, oracle_decode, to_dev, make_ctx
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+@pytest.fixture(scope="module")
+def K():
+    import torch
+    assert torch.cuda.is_available()
+    from cross_layer_kv_shared_b200 import kvshare
+    return kvshare
+
+
+def small(name, dtype, L, layer_map, slots, Hq, Hkv, d, B, T, scale=1.0, seed=7):
+    return Config(name, "decode", layers=L, q_heads=Hq, kv_heads=Hkv, head_dim=d, batch=B, context=T, dtype=dtype,
+                  layer_map=tuple(layer_map), slots=slots, qkv_scale=scale, seed=seed)
+
+
+CLA_SMALL = small("cla2_small", "bf16", 4, [(SINGLE, l // 2, 0) for l in range(4)], 2, 32, 4, 64, 3, 333, 0.125)
+DG_SMALL = small("depthgraft_small", "bf16", 6,
+                 [(SINGLE, 0, 0), (SINGLE, 1, 0), (SINGLE, 2, 0), (SINGLE, 3, 0), (MIX, 0, 2), (MIX, 1, 3)],
+                 4, 16, 4, 128, 2, 517)
+
+
+def test_tiny_cla2_f32_every_output(K):
+    inp = TINY_CLA2.make_all()
+    out, lse, launches = decode_gpu(K, TINY_CLA2, inp)
+    want, want_lse = oracle_decode(TINY_CLA2, inp)
+    assert_close(out, want, TOL_F32, "out")
+    assert_close(lse, want_lse, TOL_F32, "lse")
+    assert launches == TINY_CLA2.layers
+
+
+@pytest.mark.parametrize("cfg", [CLA_SMALL, DG_SMALL], ids=lambda c: c.name)
+def test_reduced_bf16_every_output(K, cfg):
+    inp = cfg.make_all()
+    out, lse, _ = decode_gpu(K, cfg, inp)
+    want, want_lse = oracle_decode(cfg, inp)
+    _, rel = assert_close(out, want, TOL_BF16, "out")
+    assert rel < 2e-2
+    assert_close(lse, want_lse, TOL_BF16, "lse")
+
+
+@pytest.mark.parametrize("dtype,d,g,T,mix", [
+    ("bf16", 64, 1, 1, False), ("bf16", 64, 16, 15, False), ("bf16", 128, 4, 16, False),
+    ("bf16", 128, 8, 1000, True), ("bf16", 64, 2, 4096, True), ("bf16", 128, 16, 33, True),
+    ("bf16", 64, 8, 31, True), ("f32", 128, 4, 77, True), ("f32", 64, 3, 1, False), ("f32", 128, 1, 300, False),
+])
+def test_edge_shapes(K, dtype, d, g, T, mix):
+    Hkv = 2
+    lmap = [(SINGLE, 0, 0), (MIX, 0, 1) if mix else (SINGLE, 1, 0)]
+    cfg = small(f"edge_{dtype}_{d}_{g}_{T}", dtype, 2, lmap, 2, g * Hkv, Hkv, d, 2, T, seed=11)
+    inp = cfg.make_all()
+    out, lse, _ = decode_gpu(K, cfg, inp)
+    want, want_lse = oracle_decode(cfg, inp)
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    assert_close(out, want, tol, "out")
+    assert_close(lse, want_lse, tol, "lse")
+
+
+@pytest.mark.parametrize("cfg", [CLA_SMALL, DG_SMALL, TINY_CLA2], ids=lambda c: c.name)
+def test_split_count_does_not_change_the_result(K, cfg):
+    inp = cfg.make_all()
+    ref_out, ref_lse, _ = decode_gpu(K, cfg, inp, splits=1)
+    for s in (2, 5, 0):
+        out, lse, _ = decode_gpu(K, cfg, inp, splits=s)
+        assert np.max(np.abs(out - ref_out)) <= 1e-5 * max(1.0, np.max(np.abs(ref_out)))
+        assert np.max(np.abs(lse - ref_lse)) <= 1e-5
+
+
+def test_cla_layers_sharing_a_slot_match_bitwise(K):
+    cfg = CLA_SMALL
+    inp = cfg.make_all()
+    inp["q"] = inp["q"].copy()
+    inp["q"][1] = inp["q"][0]              # layer 1 reuses layer 0's slot; same query
+    out, lse, _ = decode_gpu(K, cfg, inp)
+    assert np.array_equal(out[0], out[1]) and np.array_equal(lse[0], lse[1])
+
+
+@pytest.mark.parametrize("cfg", [CLA_SMALL, DG_SMALL, TINY_CLA2], ids=lambda c: c.name)
+def test_constant_values_give_constant_output(K, cfg):
+    inp = cfg.make_all()
+    one = np.float32(1.0)
+    inp["v"] = (np.full(inp["v"].shape, 0x3F80, np.uint16) if cfg.dtype == "bf16"
+                else np.full(inp["v"].shape, one, np.float32))
+    out, _, _ = decode_gpu(K, cfg, inp)
+    assert np.max(np.abs(out - 1.0)) < 1e-5
+
+
+def test_mix_weight_endpoints_match_single_source(K):
+    base = DG_SMALL
+    inp = base.make_all()
+    w = inp["w"].copy()
+    w[4] = 1.0
+    w[5] = 0.0
+    inp["w"] = w
+    out, _, _ = decode_gpu(K, base, inp)
+    single = base.replace(layer_map=base.layer_map[:4] + ((SINGLE, 0, 0), (SINGLE, 3, 0)))
+    out_s, _, _ = decode_gpu(K, single, inp)
+    assert np.max(np.abs(out[4:] - out_s[4:])) < 1e-5
+
+
+def test_layer_range_writes_only_its_rows(K):
+    cfg = CLA_SMALL
+    inp = cfg.make_all()
+    out, lse, launches = decode_gpu(K, cfg, inp, layers=(1, 3))
+    assert launches == 2
+    assert np.all(np.isnan(out[0])) and np.all(np.isnan(out[3]))
+    want, _ = oracle_decode(cfg, inp, layers=[1, 2])
+    assert_close(out[1:3], want[1:3], TOL_BF16)
+
+
+def test_decode_host_matches_device_call(K):
+    import torch
+    cfg = DG_SMALL
+    inp = cfg.make_all()
+    out, lse, _ = decode_gpu(K, cfg, inp)
+    d = {n: to_dev(a, cfg.dtype) for n, a in inp.items()}
+    h = make_ctx(K, cfg)
+    try:
+        K.kvshare_set_map(h, cfg.layer_map, inp["w"])
+        qh = torch.from_numpy(np.ascontiguousarray(inp["q"]).view(np.int16)).pin_memory()
+        oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        lh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        cache = K.Cache(batch=cfg.batch, context=cfg.context, k=d["k"], v=d["v"], slots=cfg.slots)
+        K.kvshare_decode_host(h, cache, qh, oh, lh)
+        assert K.kvshare_sync_status(h) == K.KVS_OK
+    finally:
+        K.kvshare_destroy(h)
+    assert np.array_equal(oh.numpy(), out) and np.array_equal(lh.numpy(), lse)
+
+
+# ----------------------------------------------------------------------------- full sizes, sampled
+def _device_inputs(cfg):
+    return {n: sgpu.make_device(cfg, n) for n in cfg.recipe()}
+
+
+def _sampled_oracle(cfg, q_host, w, layers, batches):
+    """Oracle outputs at (layer, batch) pairs, drawing only the needed cache slices on the host."""
+    cache = {}
+
+    def get(name, index):
+        key = (name, index)
+        if key not in cache:
+            cache[key] = cfg.make(name, index)
+        from oracle import kvshare_ref as ref
+        return ref.to_f64(cache[key], cfg.dtype)
+    from oracle import kvshare_ref as ref
+    res = {}
+    for l in layers:
+        for b in batches:
+            for j in range(cfg.kv_heads):
+                g = cfg.group
+                o, s = ref.decode_head_group(cfg.layer_map, l, b, j, ref.to_f64(q_host[l, b, j * g:(j + 1) * g], cfg.dtype),
+                                             get, w=w)
+                res[(l, b, j)] = (o, s)
+    return res
+
+
+@pytest.mark.parametrize("cfg,layers,batches", [
+    (CLA2_1P1B, list(range(22)), [0, 17]),
+    (DEPTHGRAFT_DECODE, [0, 3, 8, 11, 16, 19, 23], [5]),
+], ids=["cla2_1p1b", "depthgraft_decode"])
+def test_full_size_sampled(K, cfg, layers, batches):
+    import torch
+    d = _device_inputs(cfg)
+    q_host = cfg.make("q")
+    # the device generator reproduces the host bits
+    assert np.array_equal(d["q"].view(torch.int16).cpu().numpy().view(np.uint16), q_host)
+    w = cfg.make("w")
+    h = make_ctx(K, cfg)
+    try:
+        K.kvshare_set_map(h, cfg.layer_map, w)
+        out = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim, device="cuda")
+        lse = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, device="cuda")
+        cache = K.Cache(batch=cfg.batch, context=cfg.context, k=d["k"], v=d["v"], slots=cfg.slots)
+        K.kvshare_decode(h, cache, d["q"], out, lse)
+        assert K.kvshare_sync_status(h) == K.KVS_OK
+    finally:
+        K.kvshare_destroy(h)
+    out = out.cpu().numpy()
+    lse = lse.cpu().numpy()
+    want = _sampled_oracle(cfg, q_host, w, layers, batches)
+    g = cfg.group
+    worst = 0.0
+    for (l, b, j), (o, s) in want.items():
+        got = out[l, b, j * g:(j + 1) * g]
+        worst = max(worst, assert_close(got, o, TOL_BF16, f"l{l} b{b} j{j}")[0])
+        assert_close(lse[l, b, j * g:(j + 1) * g], s, TOL_BF16, f"lse l{l} b{b} j{j}")
+    print(f"{cfg.name}: worst max|d| {worst:.3e}")
