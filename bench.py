@@ -112,16 +112,54 @@ class DecodeRunner:
     def __init__(self, cfg, K, torch, sgpu):
         self.cfg, self.K, self.torch = cfg, K, torch
         self.dev = {n: sgpu.make_device(cfg, n) for n in cfg.recipe()}
-        self.w = cfg.make("w")
         _, self.h = K.kvshare_create(cfg.layers, cfg.q_heads, cfg.kv_heads, cfg.head_dim,
-                                     K.KVS_F32 if cfg.dtype == "f32" else K.KVS_BF16, cfg.batch, cfg.context)
+                                     K.KVS_F32 if cfg.dtype == "f32" else K.KVS_BF16, cfg.batch, cfg.context,
+                                     basis_rank=cfg.basis_rank)
+        self.w = None if cfg.lowrank else cfg.make("w")
         K.kvshare_set_map(self.h, cfg.layer_map, self.w)
         self.out = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim, device="cuda")
         self.lse = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, device="cuda")
-        self.cache = K.Cache(batch=cfg.batch, context=cfg.context, k=self.dev["k"], v=self.dev["v"], slots=cfg.slots)
         self.stream = torch.cuda.current_stream()
         l2 = torch.cuda.get_device_properties(0).L2_cache_size
         self.flush_buf = torch.empty(2 * l2, dtype=torch.int8, device="cuda")
+        self.pack_ms = None
+        if cfg.lowrank:
+            d = self.dev
+            L, B, T, Hkv = cfg.layers, cfg.batch, cfg.context, cfg.kv_heads
+            self.rank = torch.empty((L, B, T), dtype=torch.uint8, device="cuda")
+            self.ck = torch.empty((L, B, Hkv, T, 16), dtype=torch.int8, device="cuda")
+            self.cv = torch.empty_like(self.ck)
+            self.sk = torch.empty((L, B, Hkv, T), dtype=torch.int16, device="cuda")
+            self.sv = torch.empty_like(self.sk)
+            times = []
+            for i in range(4):
+                self.flush()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(self.stream)
+                K.kvshare_pack_residual(self.h, d["score"], d["u_k"], d["u_v"], self.rank, self.ck, self.cv,
+                                        self.sk, self.sv, B, T, self.stream)
+                e1.record(self.stream)
+                times.append((e0, e1))
+            torch.cuda.synchronize()
+            self.pack_ms = statistics.median([a.elapsed_time(b) for a, b in times[1:]])
+            self.pack_bytes = (d["u_k"].numel() * 4 * 2 + d["score"].numel() * 4 + self.rank.numel()
+                               + self.ck.numel() * 2 + self.sk.numel() * 2 * 2)
+            del d["u_k"], d["u_v"]
+            self.cache = K.Cache(batch=B, context=T, coef_k=d["coef_k"], coef_v=d["coef_v"], basis_k=d["basis_k"],
+                                 basis_v=d["basis_v"], u_k=self.ck, u_v=self.cv, s_k=self.sk, s_v=self.sv,
+                                 r_k=d["r_k"], r_v=d["r_v"], rank=self.rank, pairs=cfg.pairs)
+            # algorithmic bytes per layer: coefficients, codes at each token's rank, scales of
+            # tokens with rank > 0, the rank byte, bases and residual factors
+            r = self.rank.to(torch.int64)
+            per_layer_codes = (2 * Hkv * r.sum(dim=(1, 2))).cpu().numpy()
+            per_layer_scales = (2 * 2 * Hkv * (r > 0).sum(dim=(1, 2))).cpu().numpy()
+            fixed = (2 * B * Hkv * T * cfg.basis_rank * 2 + B * T + 2 * Hkv * cfg.basis_rank * cfg.head_dim * 2
+                     + 2 * Hkv * 16 * cfg.head_dim * 2)
+            self.layer_bytes = [int(fixed + per_layer_codes[l] + per_layer_scales[l]) for l in range(L)]
+        else:
+            self.cache = K.Cache(batch=cfg.batch, context=cfg.context, k=self.dev["k"], v=self.dev["v"],
+                                 slots=cfg.slots)
+            self.layer_bytes = [decode_read_bytes(cfg, l) for l in range(cfg.layers)]
 
     def flush(self):
         self.flush_buf.fill_(1)
@@ -211,19 +249,75 @@ def gpu_arm(args, cfg_name, secondary=False):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in e2e]))
 
-    read_bytes = sum(decode_read_bytes(cfg, l) for l in range(cfg.layers))
+    read_bytes = sum(r.layer_bytes)
     res = {
         "cfg": cfg, "step_ms": step_ms, "per_layer_ms": per_layer, "launches": launches,
         "kv_gbs": read_bytes / (step_ms * 1e-3) / 1e9, "tok_s": cfg.batch / (step_ms * 1e-3),
         "no_flush_ms": nf_ms, "e2e_ms": e2e_ms, "wall_s": t_wall, "clocks": clk.summary(),
         "h2d": q_host.numel() * q_host.element_size(),
         "d2h": out_host.numel() * 4 + lse_host.numel() * 4,
-        "read_bytes": read_bytes,
+        "read_bytes": read_bytes, "pack_ms": r.pack_ms,
+        "pack_bytes": getattr(r, "pack_bytes", None),
     }
     r.close()
     del r
     torch.cuda.empty_cache()
     return res
+
+
+def prefill_flops(cfg):
+    """Causal prefill FLOPs credited per step: 2 * B * Hq * d * S^2 per layer (QK^T + PV, causal half)."""
+    return 2.0 * cfg.batch * cfg.q_heads * cfg.head_dim * cfg.context ** 2 * cfg.layers
+
+
+def prefill_arm(args, cfg_name="depthgraft_prefill"):
+    """Times kvshare_prefill over all layers; per-layer CUDA events, no L2 flush (tensor-bound)."""
+    import torch
+    import synth.gpu as sgpu
+    from cross_layer_kv_shared_b200 import kvshare as K
+
+    cfg = BY_NAME[cfg_name]
+    dev = {n: sgpu.make_device(cfg, n) for n in cfg.recipe()}
+    _, h = K.kvshare_create(cfg.layers, cfg.q_heads, cfg.kv_heads, cfg.head_dim, K.KVS_BF16, cfg.batch, cfg.context)
+    K.kvshare_set_map(h, cfg.layer_map, cfg.make("w"))
+    S = cfg.context
+    out = torch.empty((cfg.layers, cfg.batch, cfg.q_heads, S, cfg.head_dim), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((cfg.layers, cfg.batch, cfg.q_heads, S), device="cuda")
+    cache = K.Cache(batch=cfg.batch, context=S, k=dev["k"], v=dev["v"], slots=cfg.slots)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        K.kvshare_prefill(h, cache, dev["q"], out, lse, stream=stream)
+    torch.cuda.synchronize()
+    n0 = K.kvshare_launch_count(h)
+    ev = []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(args.steps):
+            for l in range(cfg.layers):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                K.kvshare_prefill(h, cache, dev["q"], out, lse, l, l + 1, stream=stream)
+                e1.record(stream)
+                ev.append((l, e0, e1))
+        torch.cuda.synchronize()
+    st = K.kvshare_sync_status(h)
+    assert st == K.KVS_OK, K.kvshare_status_string(st)
+    launches = K.kvshare_launch_count(h) - n0
+    per_layer = np.zeros(cfg.layers)
+    for l, e0, e1 in ev:
+        per_layer[l] += e0.elapsed_time(e1)
+    per_layer /= args.steps
+    step_ms = max_over_ranks(float(per_layer.sum()))
+    single = [l for l in range(cfg.layers) if cfg.layer_map[l][0] == 0]
+    mixed = [l for l in range(cfg.layers) if cfg.layer_map[l][0] == 1]
+    K.kvshare_destroy(h)
+    del dev, out, lse
+    torch.cuda.empty_cache()
+    fl = prefill_flops(cfg)
+    per_layer_fl = fl / cfg.layers
+    return {"cfg": cfg, "step_ms": step_ms, "tflops": fl / (step_ms * 1e-3) / 1e12,
+            "single_layer_tflops": per_layer_fl / (float(np.mean(per_layer[single])) * 1e-3) / 1e12,
+            "mix_layer_tflops": (per_layer_fl / (float(np.mean(per_layer[mixed])) * 1e-3) / 1e12) if mixed else None,
+            "launches": launches, "clocks": clk.summary(), "tokens": cfg.batch * S}
 
 
 def dist_on():
@@ -331,6 +425,7 @@ def main():
     ap.add_argument("--config", default="cla2_1p1b")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -353,13 +448,25 @@ def main():
     cfg = main_res["cfg"]
     sec = {}
     if not args.no_secondary:
-        for name in ("depthgraft_decode",):
+        for name in ("depthgraft_decode", "depthweave_decode"):
             if name == args.config:
                 continue
             r2 = gpu_arm(argparse.Namespace(steps=max(5, args.steps // 2), warmup=3), name)
             sec[name] = {"tok_s": r2["tok_s"] * world, "kv_gbs": r2["kv_gbs"],
                          "hbm_frac": r2["kv_gbs"] / hbm_peak, "ms_per_step": r2["step_ms"],
-                         "no_flush_ms_per_step": r2["no_flush_ms"], "gpu_launches": r2["launches"]}
+                         "algorithmic_bytes_per_step": r2["read_bytes"],
+                         "no_flush_ms_per_step": r2["no_flush_ms"], "gpu_launches": r2["launches"],
+                         "e2e_tok_s": r2["cfg"].batch * world / (r2["e2e_ms"] * 1e-3)}
+            if r2["pack_ms"] is not None:
+                sec[name]["pack_residual_ms"] = r2["pack_ms"]
+                sec[name]["pack_residual_gbs"] = r2["pack_bytes"] / (r2["pack_ms"] * 1e-3) / 1e9
+    if not args.no_secondary and not args.no_prefill:
+        pr = prefill_arm(argparse.Namespace(steps=max(3, args.steps // 3), warmup=3))
+        sec["depthgraft_prefill"] = {
+            "tflops": pr["tflops"], "ms_per_step": pr["step_ms"], "tok_s": pr["tokens"] * world / (pr["step_ms"] * 1e-3),
+            "tensor_frac_of_burst": pr["tflops"] / bf16_peak, "tensor_frac_of_sustained": pr["tflops"] / bf16_sust,
+            "single_source_layer_tflops": pr["single_layer_tflops"], "mix_layer_tflops": pr["mix_layer_tflops"],
+            "flops_per_step": prefill_flops(pr["cfg"]), "gpu_launches": pr["launches"], "clocks": pr["clocks"]}
     avg_launch_ms = float(np.mean(main_res["per_layer_ms"]))
     per_launch_bytes = decode_read_bytes(cfg, 0)
     achieved = per_launch_bytes / (avg_launch_ms * 1e-3) / 1e9

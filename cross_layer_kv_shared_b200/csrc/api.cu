@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "kvs_internal.h"
@@ -38,16 +39,20 @@ struct MapKey {
     const void* ptr;
     uint64_t d0, d1, d2;
     uint32_t box0, box1;
-    int dtype;
+    int dtype, swizzle;
     bool operator==(const MapKey& o) const {
         return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && box0 == o.box0 && box1 == o.box1 &&
-               dtype == o.dtype;
+               dtype == o.dtype && swizzle == o.swizzle;
     }
 };
 
-struct MapEntry {
-    MapKey key;
-    CUtensorMap map;
+struct MapKeyHash {
+    size_t operator()(const MapKey& k) const {
+        size_t h = reinterpret_cast<uintptr_t>(k.ptr);
+        for (uint64_t v : {k.d0, k.d1, k.d2, (uint64_t)k.box0, (uint64_t)k.box1, (uint64_t)k.dtype, (uint64_t)k.swizzle})
+            h = h * 1000003u ^ std::hash<uint64_t>()(v);
+        return h;
+    }
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -84,7 +89,7 @@ struct kvshare_ctx {
     long long wait_limit = 4000000000LL;     // ~2 s of SM clock
     long long stall_limit = 20000000LL;      // ~10 ms
     uint64_t launches = 0;
-    std::vector<MapEntry> maps;
+    std::unordered_map<MapKey, CUtensorMap, MapKeyHash> maps;
     // staging for kvshare_decode_host
     void* q_stage = nullptr;
     float* out_stage = nullptr;
@@ -97,29 +102,34 @@ size_t elem_size(kvshare_dtype t) { return t == KVS_F32 ? 4 : 2; }
 
 kvshare_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVS_OK : KVS_ECUDA; }
 
-// 3-D tiled map over a store [rows][T][D] with a box of {64, tt, 1}, 128-B swizzle.
-bool get_store_map(kvshare_ctx* c, const void* base, int D, int T, int rows, int tt, CUtensorMap* out) {
-    MapKey key{base, (uint64_t)D, (uint64_t)T, (uint64_t)rows, 64u, (uint32_t)tt, 0};
-    for (auto& e : c->maps)
-        if (e.key == key) {
-            *out = e.map;
-            return true;
-        }
+// 3-D tiled map over [rows][T][inner] elements, box {box0, tt, 1}.
+bool get_map(kvshare_ctx* c, const void* base, CUtensorMapDataType dt, int esize, int inner, int T, int rows,
+             int box0, int tt, CUtensorMapSwizzle sw, CUtensorMap* out) {
+    MapKey key{base, (uint64_t)inner, (uint64_t)T, (uint64_t)rows, (uint32_t)box0, (uint32_t)tt, (int)dt, (int)sw};
+    auto it = c->maps.find(key);
+    if (it != c->maps.end()) {
+        *out = it->second;
+        return true;
+    }
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     CUtensorMap m;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
-    cuuint32_t box[3] = {64u, (cuuint32_t)tt, 1u};
+    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)T, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)inner * esize, (cuuint64_t)T * inner * esize};
+    cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)tt, 1u};
     cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(&m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
-    if (c->maps.size() >= 64) c->maps.erase(c->maps.begin());
-    c->maps.push_back({key, m});
+    if (c->maps.size() >= 4096) c->maps.clear();
+    c->maps.emplace(key, m);
     *out = m;
     return true;
+}
+
+// K or V store [rows][T][D] bf16, box {64, tt}, 128-B swizzle
+bool get_store_map(kvshare_ctx* c, const void* base, int D, int T, int rows, int tt, CUtensorMap* out) {
+    return get_map(c, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, rows, 64, tt, CU_TENSOR_MAP_SWIZZLE_128B, out);
 }
 
 int choose_splits(const kvshare_ctx* c, int units, int tiles, int ctas_per_sm, int g, int D) {
@@ -210,7 +220,42 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
             a.splits = (tiles + a.tiles_per_split - 1) / a.tiles_per_split;
             err = launch_decode_f32(e.kind == KVS_SRC_MIX, D, a, st);
         } else if (e.kind == KVS_SRC_LOWRANK) {
-            return KVS_EUNSUPPORTED;
+            const int Rb = cf.basis_rank;
+            const int tt = decode_lowrank_tile(Rb);
+            static int occ_lr[2][3] = {{0, 0, 0}, {0, 0, 0}};
+            int& o = occ_lr[D == 128][Rb == 32 ? 0 : (Rb == 64 ? 1 : 2)];
+            if (o == 0) o = decode_lowrank_occupancy(D, Rb);
+            const int tiles = (T + tt - 1) / tt;
+            int s = choose_splits(c, B * Hkv, tiles, o, g, D);
+            a.tiles_per_split = (tiles + s - 1) / s;
+            a.splits = (tiles + a.tiles_per_split - 1) / a.tiles_per_split;
+            const size_t BHT = static_cast<size_t>(B) * Hkv * T;
+            a.pair = e.src0;
+            a.Rb = Rb;
+            a.Rm = 16;
+            a.coef_k = k->coef_k;
+            a.coef_v = k->coef_v;
+            a.basis_k = static_cast<const uint16_t*>(k->basis_k) + static_cast<size_t>(e.src0) * Hkv * Rb * D;
+            a.basis_v = static_cast<const uint16_t*>(k->basis_v) + static_cast<size_t>(e.src0) * Hkv * Rb * D;
+            a.u_k = k->u_k + static_cast<size_t>(l) * BHT * 16;
+            a.u_v = k->u_v + static_cast<size_t>(l) * BHT * 16;
+            a.s_k = k->s_k + static_cast<size_t>(l) * BHT;
+            a.s_v = k->s_v + static_cast<size_t>(l) * BHT;
+            a.r_k = static_cast<const uint16_t*>(k->r_k) + static_cast<size_t>(l) * Hkv * 16 * D;
+            a.r_v = static_cast<const uint16_t*>(k->r_v) + static_cast<size_t>(l) * Hkv * 16 * D;
+            a.rank = k->rank + static_cast<size_t>(l) * B * T;
+            CUtensorMap maps[4];
+            const int crows = k->pairs * B * Hkv;
+            const int box0 = Rb < 64 ? Rb : 64;
+            const CUtensorMapSwizzle sw = Rb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+            if (!get_map(c, k->coef_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Rb, T, crows, box0, tt, sw, &maps[0]) ||
+                !get_map(c, k->coef_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Rb, T, crows, box0, tt, sw, &maps[1]) ||
+                !get_map(c, a.u_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, T, B * Hkv, 16, tt,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, &maps[2]) ||
+                !get_map(c, a.u_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, T, B * Hkv, 16, tt,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, &maps[3]))
+                return KVS_ECUDA;
+            err = launch_decode_lowrank(D, Rb, a, maps, st);
         } else {
             const bool mix = e.kind == KVS_SRC_MIX;
             const TileShape ts = decode_bf16_shape(D, mix);
@@ -420,9 +465,60 @@ kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, co
 
 kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const void* q, void* out, float* lse,
                                int l0, int l1, int seqlen, void* stream) {
-    (void)cache; (void)q; (void)out; (void)lse; (void)l0; (void)l1; (void)seqlen; (void)stream;
-    if (ctx == nullptr) return KVS_EINVAL;
-    return KVS_EUNSUPPORTED;
+    if (ctx == nullptr || !ctx->map_set) return KVS_EINVAL;
+    kvshare_status s = validate_cache_common(ctx, cache);
+    if (s != KVS_OK) return s;
+    const kvshare_config& cf = ctx->cfg;
+    if (l0 < 0 || l1 > cf.num_layers || l0 > l1) return KVS_EINVAL;
+    if (seqlen < 1 || seqlen > cache->context) return KVS_EINVAL;
+    if (!dev_ok(q) || !dev_ok(out) || (lse != nullptr && (!is_device_ptr(lse) || (reinterpret_cast<uintptr_t>(lse) & 3u))))
+        return KVS_EINVAL;
+    bool need_kv = false, need_lr = false;
+    for (int l = l0; l < l1; ++l) {
+        s = check_layer_sources(ctx, cache, l, &need_kv, &need_lr);
+        if (s != KVS_OK) return s;
+    }
+    if (need_lr || cf.dtype != KVS_BF16) return KVS_EUNSUPPORTED;
+    if (need_kv && (cache->slots < 1 || !dev_ok(cache->k) || !dev_ok(cache->v))) return KVS_EINVAL;
+    if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
+    const int D = cf.head_dim, B = cache->batch, Hq = cf.num_q_heads, Hkv = cf.num_kv_heads, T = cache->context;
+    const size_t per_layer = static_cast<size_t>(B) * Hq * seqlen;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int l = l0; l < l1; ++l) {
+        const kvshare_layer& e = ctx->map[l];
+        const bool mix = e.kind == KVS_SRC_MIX;
+        PrefillArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.q = static_cast<const uint16_t*>(q) + static_cast<size_t>(l) * per_layer * D;
+        a.out = static_cast<uint16_t*>(out) + static_cast<size_t>(l) * per_layer * D;
+        a.lse = lse ? lse + static_cast<size_t>(l) * per_layer : nullptr;
+        a.src0 = e.src0;
+        a.src1 = mix ? e.src1 : e.src0;
+        a.mix = mix ? 1 : 0;
+        a.w = ctx->w_dev + static_cast<size_t>(l) * Hkv;
+        a.B = B;
+        a.Hq = Hq;
+        a.Hkv = Hkv;
+        a.S = seqlen;
+        a.T = T;
+        a.g = Hq / Hkv;
+        a.scale_log2 = ctx->scale * 1.4426950408889634f;
+        a.err = ctx->err;
+        a.wait_limit = ctx->wait_limit;
+        const int bn = prefill_kv_tile(D, mix);
+        CUtensorMap tq, tk, tv;
+        const int rows = cache->slots * B * Hkv;
+        if (!get_map(ctx, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, seqlen, B * Hq, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B, &tq) ||
+            !get_map(ctx, cache->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, rows, 64, bn,
+                     CU_TENSOR_MAP_SWIZZLE_128B, &tk) ||
+            !get_map(ctx, cache->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, rows, 64, bn,
+                     CU_TENSOR_MAP_SWIZZLE_128B, &tv))
+            return KVS_ECUDA;
+        if (launch_prefill(D, mix, tq, tk, tv, a, st) != cudaSuccess) return KVS_ECUDA;
+        ++ctx->launches;
+    }
+    return KVS_OK;
 }
 
 kvshare_status kvshare_pack_residual(kvshare_t ctx, const float* score, const float* u_k, const float* u_v,

@@ -73,11 +73,15 @@ int decode_bf16_ctas_per_sm(int d, bool mix);
 int decode_f32_tile();
 cudaError_t launch_decode_f32(bool mix, int d, const DecodeArgs& a, cudaStream_t st);
 
-TileShape decode_lowrank_shape();
-cudaError_t launch_decode_lowrank(const DecodeArgs& a, const CUtensorMap& tmCK, const CUtensorMap& tmCV,
-                                  cudaStream_t st);
-int decode_lowrank_ctas_per_sm();
+int decode_lowrank_tile(int rb);
+int decode_lowrank_occupancy(int d, int rb);
+// maps: coef_k, coef_v (whole [P*B*Hkv][T][Rb]) and u_k, u_v (the layer's [B*Hkv][T][16])
+cudaError_t launch_decode_lowrank(int d, int rb, const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st);
 
 cudaError_t launch_pack_residual(const PackArgs& a, cudaStream_t st);
+
+int prefill_kv_tile(int d, bool mix);
+cudaError_t launch_prefill(int d, bool mix, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const PrefillArgs& a, cudaStream_t st);
 
 }  // namespace kvs

@@ -74,12 +74,17 @@ def test_edge_shapes(K, dtype, d, g, T, mix):
 
 @pytest.mark.parametrize("cfg", [CLA_SMALL, DG_SMALL, TINY_CLA2], ids=lambda c: c.name)
 def test_split_count_does_not_change_the_result(K, cfg):
+    """fp32 caches agree to fp32 rounding. bf16 caches round each weight p to bf16
+    against the split's own running max, so they agree to bf16 precision of the
+    weights (relative 2^-8 of the output scale), well inside the 2e-2 bar."""
     inp = cfg.make_all()
     ref_out, ref_lse, _ = decode_gpu(K, cfg, inp, splits=1)
+    rel = 1e-5 if cfg.dtype == "f32" else 2.0 ** -8
     for s in (2, 5, 0):
         out, lse, _ = decode_gpu(K, cfg, inp, splits=s)
-        assert np.max(np.abs(out - ref_out)) <= 1e-5 * max(1.0, np.max(np.abs(ref_out)))
-        assert np.max(np.abs(lse - ref_lse)) <= 1e-5
+        assert np.max(np.abs(out - ref_out)) <= rel * np.max(np.abs(ref_out))
+        lse_tol = 1e-5 * max(1.0, np.max(np.abs(ref_lse))) if cfg.dtype == "f32" else 2.0 ** -8
+        assert np.max(np.abs(lse - ref_lse)) <= lse_tol
 
 
 def test_cla_layers_sharing_a_slot_match_bitwise(K):
@@ -108,9 +113,9 @@ def test_mix_weight_endpoints_match_single_source(K):
     w[4] = 1.0
     w[5] = 0.0
     inp["w"] = w
-    out, _, _ = decode_gpu(K, base, inp)
+    out, _, _ = decode_gpu(K, base, inp, splits=1)
     single = base.replace(layer_map=base.layer_map[:4] + ((SINGLE, 0, 0), (SINGLE, 3, 0)))
-    out_s, _, _ = decode_gpu(K, single, inp)
+    out_s, _, _ = decode_gpu(K, single, inp, splits=1)
     assert np.max(np.abs(out[4:] - out_s[4:])) < 1e-5
 
 

@@ -1,0 +1,194 @@
+"""GPU parity of the low-rank form: kvshare_pack_residual bit for bit, decode within 2e-2."""
+import numpy as np
+import pytest
+
+import oracle.kvshare_ref as ref
+import oracle.quant_ref as qr
+import synth.gpu as sgpu
+from synth.configs import DEPTHWEAVE_DECODE, LOWRANK, SINGLE, Config, depthweave_map
+
+from gpu_helpers import assert_close, to_dev
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def K():
+    from cross_layer_kv_shared_b200 import kvshare
+    return kvshare
+
+
+def lr_cfg(name, L, Hq, Hkv, d, B, T, Rb=32, seed=21):
+    return Config(name, "decode", layers=L, q_heads=Hq, kv_heads=Hkv, head_dim=d, batch=B, context=T, dtype="bf16",
+                  layer_map=depthweave_map(L), pairs=(L + 1) // 2, basis_rank=Rb, seed=seed)
+
+
+def dev_u16(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def pack_gpu(K, h, cfg, score, uk, uv):
+    import torch
+    L, B, T, Hkv = cfg.layers, cfg.batch, cfg.context, cfg.kv_heads
+    rank = torch.empty((L, B, T), dtype=torch.uint8, device="cuda")
+    ck = torch.empty((L, B, Hkv, T, 16), dtype=torch.int8, device="cuda")
+    cv = torch.empty_like(ck)
+    sk = torch.empty((L, B, Hkv, T), dtype=torch.int16, device="cuda")
+    sv = torch.empty_like(sk)
+    K.kvshare_pack_residual(h, score, uk, uv, rank, ck, cv, sk, sv, B, T)
+    return rank, ck, cv, sk, sv
+
+
+def make_ctx(K, cfg):
+    _, h = K.kvshare_create(cfg.layers, cfg.q_heads, cfg.kv_heads, cfg.head_dim, K.KVS_BF16, cfg.batch,
+                            cfg.context, basis_rank=cfg.basis_rank)
+    return h
+
+
+def run_small(K, cfg, inp=None):
+    import torch
+    inp = inp or cfg.make_all()
+    d = {n: to_dev(a, "bf16") for n, a in inp.items()}
+    h = make_ctx(K, cfg)
+    try:
+        K.kvshare_set_map(h, cfg.layer_map, None)
+        rank, ck, cv, sk, sv = pack_gpu(K, h, cfg, d["score"], d["u_k"], d["u_v"])
+        out = torch.full((cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim), float("nan"), device="cuda")
+        lse = torch.full((cfg.layers, cfg.batch, cfg.q_heads), float("nan"), device="cuda")
+        cache = K.Cache(batch=cfg.batch, context=cfg.context, coef_k=d["coef_k"], coef_v=d["coef_v"],
+                        basis_k=d["basis_k"], basis_v=d["basis_v"], u_k=ck, u_v=cv, s_k=sk, s_v=sv,
+                        r_k=d["r_k"], r_v=d["r_v"], rank=rank, pairs=cfg.pairs)
+        K.kvshare_decode(h, cache, d["q"], out, lse)
+        assert K.kvshare_sync_status(h) == K.KVS_OK
+    finally:
+        K.kvshare_destroy(h)
+    packed = tuple(x.cpu().numpy() for x in (rank, ck, cv, sk, sv))
+    return out.cpu().numpy(), lse.cpu().numpy(), packed, inp
+
+
+def oracle_lowrank(cfg, inp, packed):
+    rank, ck, cv, sk, sv = packed
+    arrs = {"coef_k": ref.bf16_bits_to_f64(inp["coef_k"]), "coef_v": ref.bf16_bits_to_f64(inp["coef_v"]),
+            "basis_k": ref.bf16_bits_to_f64(inp["basis_k"]), "basis_v": ref.bf16_bits_to_f64(inp["basis_v"]),
+            "u_k": ck.astype(np.float64), "u_v": cv.astype(np.float64),
+            "s_k": ref.f16_bits_to_f64(sk.view(np.uint16)), "s_v": ref.f16_bits_to_f64(sv.view(np.uint16)),
+            "r_k": ref.bf16_bits_to_f64(inp["r_k"]), "r_v": ref.bf16_bits_to_f64(inp["r_v"]), "rank": rank}
+    return ref.decode(cfg.layer_map, ref.bf16_bits_to_f64(inp["q"]), lambda n, i: arrs[n][i])
+
+
+SMALL = [lr_cfg("dw_small", 4, 8, 2, 128, 2, 300), lr_cfg("dw_d64_g16", 2, 16, 1, 64, 1, 129),
+         lr_cfg("dw_t1", 2, 4, 4, 128, 3, 1), lr_cfg("dw_t17_g1", 2, 2, 2, 64, 1, 17)]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_pack_is_bit_exact_and_decode_matches(K, cfg):
+    out, lse, packed, inp = run_small(K, cfg)
+    want = qr.pack_residual(inp["score"], inp["u_k"], inp["u_v"])
+    names = ("rank", "codes_k", "codes_v", "scale_k", "scale_v")
+    for n, got, exp in zip(names, packed, want):
+        assert np.array_equal(got.view(exp.dtype), exp), n
+    o, l = oracle_lowrank(cfg, inp, want)
+    _, rel = assert_close(out, o, TOL, "out")
+    assert rel < 2e-2
+    assert_close(lse, l, TOL, "lse")
+
+
+def test_pack_edge_rows(K):
+    """Ties, zero rows, tiny and huge magnitudes and exact thresholds through the GPU packer."""
+    import torch
+    cfg = lr_cfg("pack_edges", 1, 2, 2, 64, 1, 64)
+    g = np.random.default_rng(3)
+    u = (g.standard_normal((1, 1, 2, 64, 16)) * 10.0 ** g.uniform(-8, 5, size=(1, 1, 2, 64, 1))).astype(np.float32)
+    u[0, 0, 0, 0] = np.array([127, 0.5, 1.5, 2.5, -0.5, -1.5, 126.5, -126.5] + [0] * 8, np.float32) * np.float32(2 ** -9)
+    u[0, 0, 0, 1] = 0.0
+    u[0, 0, 1, 2] = np.array([1e30, -1e30] + [1.0] * 14, np.float32)
+    u[0, 0, 1, 3] = np.array([3e-8, 1e-8, -2e-8] + [0] * 13, np.float32)
+    score = g.uniform(size=(1, 1, 64)).astype(np.float32)
+    score[0, 0, :6] = [0.0, np.nextafter(np.float32(0.7), np.float32(0)), 0.7, np.nextafter(np.float32(0.9), np.float32(0)), 0.9, 0.99999994]
+    score[0, 0, 0] = 0.95
+    score[0, 0, 2] = 0.95
+    h = make_ctx(K, cfg)
+    try:
+        packed = pack_gpu(K, h, cfg, torch.from_numpy(score).cuda(), torch.from_numpy(u).cuda(),
+                          torch.from_numpy(u[:, :, ::-1].copy()).cuda())
+        assert K.kvshare_sync_status(h) == K.KVS_OK
+    finally:
+        K.kvshare_destroy(h)
+    want = qr.pack_residual(score, u, u[:, :, ::-1].copy())
+    for got, exp in zip(packed, want):
+        assert np.array_equal(got.cpu().numpy().view(exp.dtype), exp)
+
+
+def test_full_rank_identity_basis_equals_single_source(K):
+    """Basis = I (rank d), coefficients = K/V bits, residual rank 0 -> same attention as reading K/V."""
+    import torch
+    d, T, Hkv, Hq, B = 64, 200, 2, 8, 1
+    cfg = lr_cfg("dw_identity", 2, Hq, Hkv, d, B, T, Rb=d)
+    inp = cfg.make_all()
+    kvcfg = Config("plain", "decode", layers=2, q_heads=Hq, kv_heads=Hkv, head_dim=d, batch=B, context=T,
+                   dtype="bf16", layer_map=((SINGLE, 0, 0), (SINGLE, 0, 0)), slots=1, seed=33)
+    kv = kvcfg.make_all()
+    eye = np.where(np.eye(d, dtype=bool), np.uint16(0x3F80), np.uint16(0))
+    inp["basis_k"] = np.broadcast_to(eye, cfg.basis_shape()).copy()
+    inp["basis_v"] = inp["basis_k"].copy()
+    inp["coef_k"] = kv["k"].copy()                 # [1][B][Hkv][T][d]
+    inp["coef_v"] = kv["v"].copy()
+    inp["score"] = np.zeros(cfg.score_shape(), np.float32)   # rank 0 everywhere
+    inp["q"] = kv["q"]
+    out, lse, packed, _ = run_small(K, cfg, inp)
+    assert np.all(packed[0] == 0)
+    want = ref.decode(kvcfg.layer_map, ref.bf16_bits_to_f64(kv["q"]), lambda n, i: ref.bf16_bits_to_f64(kv[n][i]))[0]
+    assert_close(out, want, TOL, "identity basis")
+
+
+def test_full_size_sampled(K):
+    import torch
+    cfg = DEPTHWEAVE_DECODE
+    dev = {n: sgpu.make_device(cfg, n) for n in cfg.recipe()}
+    h = make_ctx(K, cfg)
+    try:
+        K.kvshare_set_map(h, cfg.layer_map, None)
+        rank, ck, cv, sk, sv = pack_gpu(K, h, cfg, dev["score"], dev["u_k"], dev["u_v"])
+        del dev["u_k"], dev["u_v"]
+        out = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim, device="cuda")
+        lse = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, device="cuda")
+        cache = K.Cache(batch=1, context=cfg.context, coef_k=dev["coef_k"], coef_v=dev["coef_v"],
+                        basis_k=dev["basis_k"], basis_v=dev["basis_v"], u_k=ck, u_v=cv, s_k=sk, s_v=sv,
+                        r_k=dev["r_k"], r_v=dev["r_v"], rank=rank, pairs=cfg.pairs)
+        K.kvshare_decode(h, cache, dev["q"], out, lse)
+        assert K.kvshare_sync_status(h) == K.KVS_OK
+    finally:
+        K.kvshare_destroy(h)
+    out = out.cpu().numpy()
+    lse = lse.cpu().numpy()
+    q = cfg.make("q")
+    g = cfg.group
+    worst = 0.0
+    for l, j in [(0, 0), (1, 5), (14, 3), (31, 7)]:
+        p = l // 2
+        score = cfg.make("score", (l, 0))
+        uk = cfg.make("u_k", (l, 0, j))
+        uv = cfg.make("u_v", (l, 0, j))
+        r = qr.route_rank(score)
+        codes_k, sck = qr.quantize(uk, r)
+        codes_v, scv = qr.quantize(uv, r)
+        # the GPU packer's bits for this slice
+        assert np.array_equal(rank[l, 0].cpu().numpy(), r)
+        assert np.array_equal(ck[l, 0, j].cpu().numpy(), codes_k)
+        assert np.array_equal(sv[l, 0, j].cpu().numpy().view(np.uint16), scv)
+        arrs = {"coef_k": ref.bf16_bits_to_f64(cfg.make("coef_k", (p, 0, j))),
+                "coef_v": ref.bf16_bits_to_f64(cfg.make("coef_v", (p, 0, j))),
+                "basis_k": ref.bf16_bits_to_f64(cfg.make("basis_k", (p, j))),
+                "basis_v": ref.bf16_bits_to_f64(cfg.make("basis_v", (p, j))),
+                "u_k": codes_k.astype(np.float64), "u_v": codes_v.astype(np.float64),
+                "s_k": ref.f16_bits_to_f64(sck), "s_v": ref.f16_bits_to_f64(scv),
+                "r_k": ref.bf16_bits_to_f64(cfg.make("r_k", (l, j))), "r_v": ref.bf16_bits_to_f64(cfg.make("r_v", (l, j))),
+                "rank": r}
+        K_, V_ = (ref.kv_lowrank(arrs["coef_" + s], arrs["basis_" + s], arrs["s_" + s], arrs["u_" + s],
+                                 arrs["r_" + s], r) for s in "kv")
+        o, s_, _ = ref.attend(ref.bf16_bits_to_f64(q[l, 0, j * g:(j + 1) * g]), K_, V_, 1 / np.sqrt(cfg.head_dim))
+        worst = max(worst, assert_close(out[l, 0, j * g:(j + 1) * g], o, TOL, f"l{l} j{j}")[0])
+        assert_close(lse[l, 0, j * g:(j + 1) * g], s_, TOL, f"lse l{l} j{j}")
+    print(f"depthweave_decode: worst max|d| {worst:.3e}")
