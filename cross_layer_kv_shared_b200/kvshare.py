@@ -66,6 +66,7 @@ def _load():
         "kvshare_debug_stall_next": ([P, I], I),
         "kvshare_launch_count": ([P], ctypes.c_uint64),
         "kvshare_status_string": ([I], ctypes.c_char_p),
+        "kvshare_decode_layer_noalloc": ([P, P, P, P, P, P, I, I, I, I, I, I, I, I, V], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -214,3 +215,15 @@ def kvshare_debug_stall_next(h, on: bool = True) -> int:
 
 def kvshare_launch_count(h) -> int:
     return int(_lib.kvshare_launch_count(h))
+
+
+def kvshare_decode_layer_noalloc(q, k, v, w, out, lse, batch: int, num_q_heads: int, num_kv_heads: int,
+                                 head_dim: int, context: int, slots: int, src0: int, src1: int = -1,
+                                 stream=None, check: bool = True) -> int:
+    """One bf16 decode layer whose scratch lives in the library's fixed device array (no allocation)."""
+    st = _lib.kvshare_decode_layer_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(w), _ptr(out), _ptr(lse), int(batch),
+                                           int(num_q_heads), int(num_kv_heads), int(head_dim), int(context),
+                                           int(slots), int(src0), int(src1), _stream(stream))
+    if check:
+        _check(st, "kvshare_decode_layer_noalloc")
+    return st

@@ -182,6 +182,31 @@ kvshare_status kvshare_debug_stall_next(kvshare_t ctx, int on);
 /* Number of kernels this context has launched since it was created. */
 uint64_t kvshare_launch_count(kvshare_t ctx);
 
+/* One bf16 decode layer that allocates no device memory. The paper has no
+ * counterpart; this entry point exists for callers that cannot call cudaMalloc
+ * (code inside a capture or a host framework whose own allocator must own all
+ * device memory, or a process whose footprint must not grow after start-up).
+ * It needs no context: the split partials, arrival counters and status word
+ * live in a fixed 2 MiB device array inside this library, which every GPU that
+ * loads the library holds until the process exits.
+ *   q:   [batch][Hq][d] bf16        out: [batch][Hq][d] fp32
+ *   lse: [batch][Hq] fp32 or NULL   k, v: [slots][batch][Hkv][T][d] bf16 (T = context)
+ *   src1 < 0: single source src0; src1 >= 0: convex mix of src0 and src1 with
+ *   w: [Hkv] fp32 device weights in [0, 1] (ignored for a single source).
+ *   Softmax scale 1/sqrt(d); d is 64 or 128; Hq / Hkv <= 16.
+ * Limits: batch * Hkv <= 4096, else KVS_EINVAL; the split count is lowered
+ * until the partials fit the array. The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) and should come before
+ * any stream capture. Every call shares the array and keeps the previous
+ * call's contents; the call clears the counters and status word on `stream`
+ * first. Calls that overlap on the GPU (two streams, two host threads) race on
+ * the array. Device-side wait timeouts are recorded in the array's status word
+ * and not reported. */
+kvshare_status kvshare_decode_layer_noalloc(const void* q, const void* k, const void* v, const float* w,
+                                            float* out, float* lse, int batch, int num_q_heads,
+                                            int num_kv_heads, int head_dim, int context, int slots,
+                                            int src0, int src1, void* stream);
+
 /* Static text for a status code. */
 const char* kvshare_status_string(kvshare_status s);
 
