@@ -122,6 +122,7 @@ class DecodeRunner:
         self.stream = torch.cuda.current_stream()
         l2 = torch.cuda.get_device_properties(0).L2_cache_size
         self.flush_buf = torch.empty(2 * l2, dtype=torch.int8, device="cuda")
+        self.flush_read = torch.ones(2 * l2 // 4, dtype=torch.float32, device="cuda")
         self.pack_ms = None
         if cfg.lowrank:
             d = self.dev
@@ -162,7 +163,10 @@ class DecodeRunner:
             self.layer_bytes = [decode_read_bytes(cfg, l) for l in range(cfg.layers)]
 
     def flush(self):
+        # evict the cache by writing 2x L2, then read another 2x L2 so the lines left are
+        # clean: the timed kernel neither hits L2 nor pays for the flush's write-backs
         self.flush_buf.fill_(1)
+        self._sink = self.flush_read.sum()
 
     def layer(self, l):
         self.K.kvshare_decode(self.h, self.cache, self.dev["q"], self.out, self.lse, l, l + 1, self.stream)
@@ -325,13 +329,24 @@ def dist_on():
 
 
 def max_over_ranks(x: float) -> float:
-    if not dist_on():
+    """Max of a per-rank time over all ranks (the job is as slow as its slowest rank)."""
+    import torch.distributed as dist
+    if not dist_on() or not dist.is_initialized():
         return x
     import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def arm_config(cfg, world: int) -> dict:
+    """The `config` object of the JSON line, shared by both arms."""
+    return {"workload": cfg.name, "layers": cfg.layers, "batch_per_gpu": cfg.batch, "context": cfg.context,
+            "q_heads": cfg.q_heads, "kv_heads": cfg.kv_heads, "head_dim": cfg.head_dim,
+            "layer_map": "CLA2: layer l reads slot l//2" if cfg.name == "cla2_1p1b" else cfg.name,
+            "parallelism": f"replicas x{world}",
+            "l2": "flushed before every layer outside the timed events: 2x L2 write, then 2x L2 read (clean lines)"}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) arm
@@ -407,8 +422,7 @@ def reference_arm(args):
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tok/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox, N(0,1))",
-        "config": {"workload": cfg.name, "batch": cfg.batch, "context": cfg.context, "layers": cfg.layers,
-                   "q_heads": cfg.q_heads, "kv_heads": cfg.kv_heads, "head_dim": cfg.head_dim},
+        "config": arm_config(cfg, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": val, "unit": "tok/s", "cores": threads, "kind": "oracle",
                          "sample": f"{units_total} (layer, batch) units over {args.steps} steps, extrapolated"},
         "e2e": {"value": val, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -468,8 +482,10 @@ def main():
             "single_source_layer_tflops": pr["single_layer_tflops"], "mix_layer_tflops": pr["mix_layer_tflops"],
             "flops_per_step": prefill_flops(pr["cfg"]), "gpu_launches": pr["launches"], "clocks": pr["clocks"]}
     avg_launch_ms = float(np.mean(main_res["per_layer_ms"]))
-    per_launch_bytes = decode_read_bytes(cfg, 0)
+    per_launch_bytes = main_res["read_bytes"] / cfg.layers
     achieved = per_launch_bytes / (avg_launch_ms * 1e-3) / 1e9
+    kname = ("decode_lowrank_kernel<%d,%d>" % (cfg.head_dim, cfg.basis_rank) if cfg.lowrank else
+             "decode_bf16_kernel<%d,%s>" % (cfg.head_dim, "mix" if cfg.has_mix else "single"))
     traffic = NCU_TRAFFIC_BYTES.get(cfg.name)
     line = {
         "metric": METRIC,
@@ -484,10 +500,7 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded Philox, N(0,1)/8 q/k/v)",
-        "config": {"workload": cfg.name, "layers": cfg.layers, "batch_per_gpu": cfg.batch, "context": cfg.context,
-                   "q_heads": cfg.q_heads, "kv_heads": cfg.kv_heads, "head_dim": cfg.head_dim,
-                   "layer_map": "CLA2: layer l reads slot l//2", "parallelism": f"replicas x{world}",
-                   "l2": "flushed (2x L2 write) before every layer, outside the timed events"},
+        "config": arm_config(cfg, world),
         "kv_gbs": main_res["kv_gbs"],
         "hbm_frac": main_res["kv_gbs"] / hbm_peak,
         "no_flush_ms_per_step": main_res["no_flush_ms"],
@@ -496,7 +509,7 @@ def main():
         "e2e": {"value": cfg.batch * world / (main_res["e2e_ms"] * 1e-3), "unit": "tok/s",
                 "h2d_bytes_per_step": main_res["h2d"], "d2h_bytes_per_step": main_res["d2h"],
                 "ms_per_step": main_res["e2e_ms"]},
-        "roofline": {"kernel": "decode_bf16_kernel<64,single>", "bound": "hbm", "achieved": achieved,
+        "roofline": {"kernel": kname, "bound": "hbm", "achieved": achieved,
                      "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
                      "traffic": traffic, "algorithmic_bytes_per_launch": per_launch_bytes,
                      "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"},

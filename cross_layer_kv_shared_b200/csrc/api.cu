@@ -85,6 +85,7 @@ struct kvshare_ctx {
     unsigned* counters = nullptr;    // [max_batch * Hkv]
     unsigned* err = nullptr;         // status word
     int splits_override = 0;
+    int grid_override = 0;
     int stall_next = 0;
     long long wait_limit = 4000000000LL;     // ~2 s of SM clock
     long long stall_limit = 20000000LL;      // ~10 ms
@@ -143,8 +144,8 @@ int choose_splits(const kvshare_ctx* c, int units, int tiles, int ctas_per_sm, i
     }
     if (s > tiles) s = tiles;
     if (s > MAX_SPLITS) s = MAX_SPLITS;
-    // workspace capacity: units * splits * g * (D + 2) floats
-    const size_t per_split = static_cast<size_t>(units) * g * (D + 2);
+    // workspace capacity: units * splits * g * partial_width(D) floats
+    const size_t per_split = static_cast<size_t>(units) * g * (D + 4);
     while (s > 1 && per_split * s > c->ws_floats) --s;
     if (s < 1) s = 1;
     return s;
@@ -262,10 +263,29 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
             static int occ[2][2] = {{0, 0}, {0, 0}};
             int& o = occ[D == 128][mix];
             if (o == 0) o = decode_bf16_ctas_per_sm(D, mix);
-            const int tiles = (T + ts.tt - 1) / ts.tt;
-            int s = choose_splits(c, B * Hkv, tiles, o, g, D);
-            a.tiles_per_split = (tiles + s - 1) / s;
-            a.splits = (tiles + a.tiles_per_split - 1) / a.tiles_per_split;
+            // balanced grid: the units' token tiles cut into G equal ranges, one CTA each
+            const int units = B * Hkv;
+            const int n_t = (T + ts.tt - 1) / ts.tt;
+            const long long W = static_cast<long long>(units) * n_t;
+            // default: a whole number of CTAs per unit, as many as fit in one wave, so no
+            // CTA straddles two units (a straddling CTA reloads its queries mid-stream and
+            // every unit then pays a merge); ranges that straddle are still handled
+            long long G;
+            if (c->grid_override > 0) {
+                G = c->grid_override;
+            } else if (c->splits_override > 0) {
+                G = static_cast<long long>(c->splits_override) * units;
+            } else {
+                const long long per_unit = (static_cast<long long>(c->sms) * o) / units;
+                G = static_cast<long long>(units) * (per_unit > 1 ? per_unit : 1);
+            }
+            if (G < units) G = units;
+            if (G > W) G = W;
+            const size_t per = static_cast<size_t>(g) * (D + 4);
+            while (G > units && (static_cast<size_t>(units) + G) * per > c->ws_floats) --G;
+            a.units = units;
+            a.n_t = n_t;
+            a.splits = static_cast<int>(G);
             CUtensorMap tmK, tmV;
             const int rows = k->slots * B * Hkv;
             if (!get_store_map(c, k->k, D, T, rows, ts.tt, &tmK) || !get_store_map(c, k->v, D, T, rows, ts.tt, &tmV))
@@ -342,7 +362,7 @@ kvshare_status kvshare_create(const kvshare_config* cfg, kvshare_t* out) {
     const size_t units = static_cast<size_t>(c.max_batch) * c.num_kv_heads;
     const int max_tiles = (c.max_context + 15) / 16;
     const int ms = max_tiles < MAX_SPLITS ? max_tiles : MAX_SPLITS;
-    ctx->ws_floats = units * ms * g * (c.head_dim + 2);
+    ctx->ws_floats = units * ms * g * (c.head_dim + 4);
     ctx->map.assign(c.num_layers, kvshare_layer{KVS_SRC_SINGLE, 0, 0});
     ctx->w_host.assign(static_cast<size_t>(c.num_layers) * c.num_kv_heads, 1.0f);
     if (cudaMalloc(&ctx->ws, ctx->ws_floats * sizeof(float)) != cudaSuccess ||
@@ -506,16 +526,18 @@ kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const 
         a.err = ctx->err;
         a.wait_limit = ctx->wait_limit;
         const int bn = prefill_kv_tile(D, mix);
-        CUtensorMap tq, tk, tv;
+        CUtensorMap tq, tk, tv, to;
         const int rows = cache->slots * B * Hkv;
         if (!get_map(ctx, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, seqlen, B * Hq, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B, &tq) ||
+            !get_map(ctx, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, seqlen, B * Hq, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B, &to) ||
             !get_map(ctx, cache->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, rows, 64, bn,
                      CU_TENSOR_MAP_SWIZZLE_128B, &tk) ||
             !get_map(ctx, cache->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, rows, 64, bn,
                      CU_TENSOR_MAP_SWIZZLE_128B, &tv))
             return KVS_ECUDA;
-        if (launch_prefill(D, mix, tq, tk, tv, a, st) != cudaSuccess) return KVS_ECUDA;
+        if (launch_prefill(D, mix, tq, tk, tv, to, a, st) != cudaSuccess) return KVS_ECUDA;
         ++ctx->launches;
     }
     return KVS_OK;
@@ -567,6 +589,12 @@ kvshare_status kvshare_sync_status(kvshare_t ctx, void* stream) {
 kvshare_status kvshare_set_splits(kvshare_t ctx, int splits) {
     if (ctx == nullptr || splits < 0) return KVS_EINVAL;
     ctx->splits_override = splits;
+    return KVS_OK;
+}
+
+kvshare_status kvshare_debug_set_grid(kvshare_t ctx, int ctas) {
+    if (ctx == nullptr || ctas < 0) return KVS_EINVAL;
+    ctx->grid_override = ctas;
     return KVS_OK;
 }
 

@@ -1,20 +1,24 @@
 // Split-KV GQA decode over a shared cache, bf16 storage, forms SINGLE and MIX.
 //
-// One CTA = one (split, kv head j, batch b). Four warps; each warp owns a
-// private ring of NSW shared-memory stages and streams every 4th token tile of
-// the split into it with TMA (128-byte swizzle), re-issuing a stage as soon as
-// it has consumed it. Per tile and warp:
-//   S   = Q K^T            mma.sync m16n8k16 bf16 -> fp32, the g query heads of
-//                          kv head j are the M rows (padded to 16)
-//   MIX S = w S1 + (1-w) S2, the two sources' scores mixed in fp32, which equals
-//                          the scores against w K1 + (1-w) K2 (the convex mix of
-//                          the DepthGraft source pair) up to fp32 rounding
-//   online softmax in base 2 (quad shuffles for the row max)
-//   O  += P V              P rounded to bf16 as the A operand; for MIX,
-//                          O += bf16(w P) V1 + bf16((1-w) P) V2
+// Balanced split scheduling: the (batch, kv head) units' token tiles form one
+// flat list of units * n_t tiles that is cut into G equal ranges, one per CTA
+// (G = the CTAs resident at once, one per SM), so every SM streams the same
+// number of bytes whatever the batch. A range covers at most two units; each
+// unit's partial results merge in the last CTA to finish it.
+// Inside a CTA, four warps each own a private ring of NSW shared-memory stages
+// and stream every 4th tile of the range into it with TMA (128-byte swizzle),
+// re-issuing a stage as soon as it is consumed. Per tile and warp, with the
+// tokens as the MMA's M rows and the g query heads of the kv head as its N
+// columns (a group of up to 8 heads wastes nothing on padding):
+//   S^T = K Q^T            mma.sync m16n8k16 bf16 -> fp32
+//   MIX S^T = w S1^T + (1-w) S2^T, the two sources' scores mixed in fp32, which
+//                          equals the scores against w K1 + (1-w) K2 (the convex
+//                          mix of the DepthGraft source pair) up to fp32 rounding
+//   online softmax per head in base 2 (max over tokens by shuffles across lanes)
+//   P^T: the S^T accumulator rounded to bf16 and transposed in registers
+//        (movmatrix) into the B operand of
+//   O^T += V^T P^T         for MIX, O^T += V1^T bf16(w P)^T + V2^T bf16((1-w) P)^T
 // The mixed K/V never exist anywhere, in HBM or in shared memory.
-// The four warps' (m, l, O) are merged in shared memory, then finish_split
-// writes the output or the split partial (the last CTA merges the splits).
 #include "kvs_device.cuh"
 
 namespace kvs {
@@ -30,35 +34,41 @@ struct DecodeCfg {
     static constexpr int NSRC = MIX ? 2 : 1;
     static constexpr int STAGE_BYTES = 2 * NSRC * TILE_BYTES;
     static constexpr int RING_BYTES = NW * NSW * STAGE_BYTES;
-    static constexpr int COMBINE_FLOATS = NW * 16 * D + 2 * NW * 16 + 32 + 16 * D + MAX_GROUP * MAX_SPLITS + 64;
+    static constexpr int COMBINE_FLOATS = NW * 16 * D + 2 * NW * 16 + 32 + 16 * D + 2 * MAX_GROUP * MAX_SPLITS + 64;
+    static constexpr int MERGE_STAGE_OFF = ((COMBINE_FLOATS * 4 + 1023) / 1024) * 1024;   // free smem for the merge
     static constexpr int BODY = RING_BYTES > COMBINE_FLOATS * 4 ? RING_BYTES : COMBINE_FLOATS * 4;
-    static constexpr int SMEM = BODY + 1024;                  // slack to align the ring to 1024 B
-    static_assert(TT % 16 == 0, "token tile must hold whole k16 steps");
+    // per-warp state of the first unit when a warp's tiles cross into the second one
+    static constexpr int SAVE_FLOATS = NW * (16 * D + 32);
+    static constexpr int SMEM = BODY + SAVE_FLOATS * 4 + 1024;  // + slack to align the ring to 1024 B
+    static_assert(TT % 16 == 0, "token tile must hold whole m16 tiles");
     static_assert(HALF_BYTES % 1024 == 0, "swizzled halves must stay 1024-B aligned");
 };
 
-template <int D, bool MIX, int TT, int NSW>
-__global__ void __launch_bounds__(NW * 32)
+template <int D, bool MIX, int TT, int NSW, int NH, bool STRADDLE>
+__global__ void __launch_bounds__(NW * 32, 1)
 decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const DecodeArgs a) {
     using C = DecodeCfg<D, MIX, TT, NSW>;
+    constexpr int MT = TT / 16;      // m16 token tiles per tile
+    constexpr int NB = NH / 8;       // n8 head blocks
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    float* save = reinterpret_cast<float*>(smem + C::BODY);    // [NW][16][D] O, then [NW][16] m, [NW][16] l
     __shared__ __align__(8) uint64_t bars[NW * NSW + 1];
+    __shared__ int fin_unit[NW], sav_unit[NW];
 
-    const int split = blockIdx.x;
-    const int j = blockIdx.y;
-    const int b = blockIdx.z;
+    const int cta = blockIdx.x;
+    const int G = gridDim.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int g = a.g;
-
-    const int ntiles = (a.T + TT - 1) / TT;
-    const int tile0 = split * a.tiles_per_split;
-    const int tile1 = min(tile0 + a.tiles_per_split, ntiles);
+    const long long W = static_cast<long long>(a.units) * a.n_t;
+    const long long tb = (static_cast<long long>(cta) * W + G - 1) / G;
+    const long long te = (static_cast<long long>(cta + 1) * W + G - 1) / G;
+    const int span = static_cast<int>(te - tb);
+    const int u_first = static_cast<int>(tb / a.n_t);
+    const int u_last = static_cast<int>((te - 1) / a.n_t);
     const int BH = a.B * a.Hkv;
-    const int row0 = a.src0 * BH + b * a.Hkv + j;
-    const int row1 = MIX ? a.src1 * BH + b * a.Hkv + j : 0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NW * NSW + 1; ++i) mbar_init(&bars[i], 1);
@@ -71,37 +81,88 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         mbar_wait_bounded(&bars[NW * NSW], 0, a.stall_limit, a.err);
     }
 
-    // A fragments of Q (rows = the g query heads, zero rows beyond g)
-    uint32_t qa[D / 16][4];
-    {
-        const uint16_t* qb = reinterpret_cast<const uint16_t*>(a.q) +
+    uint32_t qb[D / 16][NB][2];      // B fragments of Q^T: column n = head nb*8 + lane/4
+    float o[D / 16][NB][4];          // O^T: rows = channels, columns = heads nb*8 + 2(lane%4) (+1)
+    float mrow[NB][2], lrow[NB][2];  // softmax statistics of those two heads
+    float w = 1.f, w1 = 0.f;
+    auto begin_unit = [&](int u) {
+        const int b = u / a.Hkv;
+        const int j = u % a.Hkv;
+        const uint16_t* qg = reinterpret_cast<const uint16_t*>(a.q) +
                              (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g) * D;
-        const int h0 = lane >> 2;
-        const int h1 = h0 + 8;
         const int cq = 2 * (lane & 3);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            qa[kk][0] = h0 < g ? *reinterpret_cast<const uint32_t*>(qb + h0 * D + kk * 16 + cq) : 0u;
-            qa[kk][1] = h1 < g ? *reinterpret_cast<const uint32_t*>(qb + h1 * D + kk * 16 + cq) : 0u;
-            qa[kk][2] = h0 < g ? *reinterpret_cast<const uint32_t*>(qb + h0 * D + kk * 16 + 8 + cq) : 0u;
-            qa[kk][3] = h1 < g ? *reinterpret_cast<const uint32_t*>(qb + h1 * D + kk * 16 + 8 + cq) : 0u;
-        }
-    }
-    const float w = MIX ? a.w[j] : 1.f;
-    const float w1 = 1.f - w;
-
-    float o[D / 8][4];
+        for (int nb = 0; nb < NB; ++nb) {
+            const int h = nb * 8 + (lane >> 2);
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m0 = NEG_INF, m1 = NEG_INF, l0 = 0.f, l1 = 0.f;
+            for (int ks = 0; ks < D / 16; ++ks) {
+                qb[ks][nb][0] = h < g ? *reinterpret_cast<const uint32_t*>(qg + h * D + ks * 16 + cq) : 0u;
+                qb[ks][nb][1] = h < g ? *reinterpret_cast<const uint32_t*>(qg + h * D + ks * 16 + 8 + cq) : 0u;
+            }
+            mrow[nb][0] = mrow[nb][1] = NEG_INF;
+            lrow[nb][0] = lrow[nb][1] = 0.f;
+#pragma unroll
+            for (int i = 0; i < D / 16; ++i) o[i][nb][0] = o[i][nb][1] = o[i][nb][2] = o[i][nb][3] = 0.f;
+        }
+        w = MIX ? a.w[j] : 1.f;
+        w1 = 1.f - w;
+    };
+    // write this warp's statistics and O^T for heads < g: O to dst_o [16][D], m, l to dst_ml [32]
+    auto store_state = [&](float* dst_o, float* dst_ml) {
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                lrow[nb][0] += __shfl_xor_sync(0xffffffffu, lrow[nb][0], off);
+                lrow[nb][1] += __shfl_xor_sync(0xffffffffu, lrow[nb][1], off);
+            }
+        const int e0 = lane >> 2;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            const int h0 = nb * 8 + 2 * (lane & 3);
+#pragma unroll
+            for (int dt = 0; dt < D / 16; ++dt) {
+                if (h0 < g) {
+                    dst_o[h0 * D + dt * 16 + e0] = o[dt][nb][0];
+                    dst_o[h0 * D + dt * 16 + e0 + 8] = o[dt][nb][2];
+                }
+                if (h0 + 1 < g) {
+                    dst_o[(h0 + 1) * D + dt * 16 + e0] = o[dt][nb][1];
+                    dst_o[(h0 + 1) * D + dt * 16 + e0 + 8] = o[dt][nb][3];
+                }
+            }
+            if (lane < 4) {
+                dst_ml[h0] = mrow[nb][0];
+                dst_ml[h0 + 1] = mrow[nb][1];
+                dst_ml[16 + h0] = lrow[nb][0];
+                dst_ml[16 + h0 + 1] = lrow[nb][1];
+            }
+        }
+    };
 
     uint8_t* ring = smem + warp * NSW * C::STAGE_BYTES;
     uint64_t* wb = &bars[warp * NSW];
-    const int span = tile1 - tile0;
     const int my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
+    // (unit, tile) of this warp's first tile; later tiles step by NW without dividing
+    const long long g0 = tb + warp;
+    const int u_w0 = static_cast<int>(g0 / a.n_t);
+    const int t_w0 = static_cast<int>(g0 - static_cast<long long>(u_w0) * a.n_t);
+    auto advance = [&](int& u, int& t) {
+        t += NW;
+        while (t >= a.n_t) {
+            t -= a.n_t;
+            ++u;
+        }
+    };
+    int iu = u_w0, it = t_w0;        // next tile to issue
 
     auto issue = [&](int k) {
-        const int t = tile0 + warp + k * NW;
+        (void)k;
+        const int u = iu;
+        const int t = it;
+        advance(iu, it);
+        const int row0 = a.src0 * BH + u;
+        const int row1 = MIX ? a.src1 * BH + u : 0;
         const int s = k % NSW;
         uint8_t* st = ring + s * C::STAGE_BYTES;
         mbar_arrive_expect_tx(&wb[s], C::STAGE_BYTES);
@@ -120,7 +181,24 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     }
     __syncwarp();
 
-    for (int k = 0; k < my_n; ++k) {
+    int cur_u = -1, saved_u = -1;
+    const int mi = lane >> 3;        // ldmatrix: which 8x8 matrix this lane addresses
+    const int ri = lane & 7;         //           and which row of it
+    int u = u_w0, t = t_w0;          // tile being consumed
+    if (!STRADDLE && my_n > 0) {
+        // the CTA's range lies inside one unit
+        begin_unit(u_first);
+        cur_u = u_first;
+    }
+    for (int k = 0; k < my_n; ++k, advance(u, t)) {
+        if (STRADDLE && u != cur_u) {
+            if (cur_u >= 0) {
+                store_state(save + warp * 16 * D, save + NW * 16 * D + warp * 32);
+                saved_u = cur_u;
+            }
+            begin_unit(u);
+            cur_u = u;
+        }
         const int s = k % NSW;
         const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&wb[s], (k / NSW) & 1, a.wait_limit, a.err));
         if (!ok) {
@@ -129,120 +207,113 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             for (int kk = k + 1; kk < issued; ++kk) mbar_wait_bounded(&wb[kk % NSW], (kk / NSW) & 1, a.wait_limit, a.err);
             break;
         }
-        const int t = tile0 + warp + k * NW;
         const uint32_t kb = smem_u32(ring + s * C::STAGE_BYTES);
         const uint32_t vb = kb + C::TILE_BYTES;
 
-        float sc[TT / 8][4];
-        float sc2[MIX ? TT / 8 : 1][4];
+        float sc[MT][NB][4];
+        float sc2[MIX ? MT : 1][NB][4];
 #pragma unroll
-        for (int nb = 0; nb < TT / 8; ++nb) {
-            sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
-            if (MIX) sc2[nb][0] = sc2[nb][1] = sc2[nb][2] = sc2[nb][3] = 0.f;
-        }
-        // ---- S = Q K^T
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int kk2 = 0; kk2 < D / 32; ++kk2) {
-            const int c = kk2 * 4 + (lane >> 3);
+            for (int nb = 0; nb < NB; ++nb) {
+                sc[mt][nb][0] = sc[mt][nb][1] = sc[mt][nb][2] = sc[mt][nb][3] = 0.f;
+                if (MIX) sc2[mt][nb][0] = sc2[mt][nb][1] = sc2[mt][nb][2] = sc2[mt][nb][3] = 0.f;
+            }
+        // ---- S^T = K Q^T
 #pragma unroll
-            for (int nb = 0; nb < TT / 8; ++nb) {
-                const int row = nb * 8 + (lane & 7);
+        for (int mt = 0; mt < MT; ++mt) {
+            const int row = mt * 16 + (mi & 1) * 8 + ri;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int c = ks * 2 + (mi >> 1);
                 const uint32_t off = (c >> 3) * C::HALF_BYTES + swz128(row, c & 7);
-                uint32_t r0, r1, r2, r3;
-                ldsm_x4(kb + off, r0, r1, r2, r3);
-                mma_bf16(sc[nb], qa[2 * kk2], r0, r1);
-                mma_bf16(sc[nb], qa[2 * kk2 + 1], r2, r3);
+                uint32_t af[4];
+                ldsm_x4(kb + off, af[0], af[1], af[2], af[3]);
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) mma_bf16(sc[mt][nb], af, qb[ks][nb][0], qb[ks][nb][1]);
                 if (MIX) {
-                    ldsm_x4(kb + 2 * C::TILE_BYTES + off, r0, r1, r2, r3);
-                    mma_bf16(sc2[nb], qa[2 * kk2], r0, r1);
-                    mma_bf16(sc2[nb], qa[2 * kk2 + 1], r2, r3);
+                    ldsm_x4(kb + 2 * C::TILE_BYTES + off, af[0], af[1], af[2], af[3]);
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) mma_bf16(sc2[mt][nb], af, qb[ks][nb][0], qb[ks][nb][1]);
                 }
             }
         }
-        // ---- scale, mask the ragged tail, online softmax
-        const int tb = t * TT + 2 * (lane & 3);
-        float mx0 = NEG_INF, mx1 = NEG_INF;
+        // ---- scale, mask the ragged tail, online softmax per head, P^T by movmatrix
+        uint32_t pb[MT][NB][2];
+        uint32_t pb2[MIX ? MT : 1][NB][2];
+        const int tok0 = t * TT + (lane >> 2);
 #pragma unroll
-        for (int nb = 0; nb < TT / 8; ++nb) {
+        for (int nb = 0; nb < NB; ++nb) {
+            float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float v = MIX ? (w * sc[nb][i] + w1 * sc2[nb][i]) : sc[nb][i];
-                v *= a.scale_log2;
-                if (tb + nb * 8 + (i & 1) >= a.T) v = NEG_INF;
-                sc[nb][i] = v;
-                if (i < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
+            for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float v = MIX ? (w * sc[mt][nb][i] + w1 * sc2[mt][nb][i]) : sc[mt][nb][i];
+                    v *= a.scale_log2;
+                    if (tok0 + mt * 16 + (i >> 1) * 8 >= a.T) v = NEG_INF;
+                    sc[mt][nb][i] = v;
+                    if (i & 1) mx1 = fmaxf(mx1, v); else mx0 = fmaxf(mx0, v);
+                }
+            }
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+            }
+            const float mn0 = fmaxf(mrow[nb][0], mx0);
+            const float mn1 = fmaxf(mrow[nb][1], mx1);
+            const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
+            const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
+            const float cr0 = exp2f(mrow[nb][0] - ref0);
+            const float cr1 = exp2f(mrow[nb][1] - ref1);
+            mrow[nb][0] = mn0;
+            mrow[nb][1] = mn1;
+            lrow[nb][0] *= cr0;
+            lrow[nb][1] *= cr1;
+#pragma unroll
+            for (int dt = 0; dt < D / 16; ++dt) {
+                o[dt][nb][0] *= cr0; o[dt][nb][2] *= cr0;
+                o[dt][nb][1] *= cr1; o[dt][nb][3] *= cr1;
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const float p0 = exp2f(sc[mt][nb][0] - ref0), p1 = exp2f(sc[mt][nb][1] - ref1);
+                const float p2 = exp2f(sc[mt][nb][2] - ref0), p3 = exp2f(sc[mt][nb][3] - ref1);
+                if (!MIX) {
+                    const uint32_t lo = pack_bf16(p0, p1), hi = pack_bf16(p2, p3);
+                    lrow[nb][0] += bf16_lo(lo) + bf16_lo(hi);
+                    lrow[nb][1] += bf16_hi(lo) + bf16_hi(hi);
+                    pb[mt][nb][0] = movmatrix_t(lo);
+                    pb[mt][nb][1] = movmatrix_t(hi);
+                } else {
+                    const uint32_t lo = pack_bf16(w * p0, w * p1), hi = pack_bf16(w * p2, w * p3);
+                    const uint32_t lo2 = pack_bf16(w1 * p0, w1 * p1), hi2 = pack_bf16(w1 * p2, w1 * p3);
+                    lrow[nb][0] += (bf16_lo(lo) + bf16_lo(hi)) + (bf16_lo(lo2) + bf16_lo(hi2));
+                    lrow[nb][1] += (bf16_hi(lo) + bf16_hi(hi)) + (bf16_hi(lo2) + bf16_hi(hi2));
+                    pb[mt][nb][0] = movmatrix_t(lo);
+                    pb[mt][nb][1] = movmatrix_t(hi);
+                    pb2[mt][nb][0] = movmatrix_t(lo2);
+                    pb2[mt][nb][1] = movmatrix_t(hi2);
+                }
             }
         }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0);
-        const float mn1 = fmaxf(m1, mx1);
-        const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
-        const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
-        const float cr0 = exp2f(m0 - ref0);
-        const float cr1 = exp2f(m1 - ref1);
-        m0 = mn0;
-        m1 = mn1;
-        l0 *= cr0;
-        l1 *= cr1;
+        // ---- O^T += V^T P^T
 #pragma unroll
-        for (int db = 0; db < D / 8; ++db) {
-            o[db][0] *= cr0; o[db][1] *= cr0;
-            o[db][2] *= cr1; o[db][3] *= cr1;
-        }
-        uint32_t pa[TT / 16][4];
-        uint32_t pb[MIX ? TT / 16 : 1][4];
+        for (int mt = 0; mt < MT; ++mt) {
+            const int row = mt * 16 + (mi >> 1) * 8 + ri;
 #pragma unroll
-        for (int kk = 0; kk < TT / 16; ++kk) {
-            float p[2][4];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                p[u][0] = exp2f(sc[2 * kk + u][0] - ref0);
-                p[u][1] = exp2f(sc[2 * kk + u][1] - ref0);
-                p[u][2] = exp2f(sc[2 * kk + u][2] - ref1);
-                p[u][3] = exp2f(sc[2 * kk + u][3] - ref1);
-            }
-            if (!MIX) {
-                pa[kk][0] = pack_bf16(p[0][0], p[0][1]);
-                pa[kk][1] = pack_bf16(p[0][2], p[0][3]);
-                pa[kk][2] = pack_bf16(p[1][0], p[1][1]);
-                pa[kk][3] = pack_bf16(p[1][2], p[1][3]);
-                l0 += (bf16_lo(pa[kk][0]) + bf16_hi(pa[kk][0])) + (bf16_lo(pa[kk][2]) + bf16_hi(pa[kk][2]));
-                l1 += (bf16_lo(pa[kk][1]) + bf16_hi(pa[kk][1])) + (bf16_lo(pa[kk][3]) + bf16_hi(pa[kk][3]));
-            } else {
-                pa[kk][0] = pack_bf16(w * p[0][0], w * p[0][1]);
-                pa[kk][1] = pack_bf16(w * p[0][2], w * p[0][3]);
-                pa[kk][2] = pack_bf16(w * p[1][0], w * p[1][1]);
-                pa[kk][3] = pack_bf16(w * p[1][2], w * p[1][3]);
-                pb[kk][0] = pack_bf16(w1 * p[0][0], w1 * p[0][1]);
-                pb[kk][1] = pack_bf16(w1 * p[0][2], w1 * p[0][3]);
-                pb[kk][2] = pack_bf16(w1 * p[1][0], w1 * p[1][1]);
-                pb[kk][3] = pack_bf16(w1 * p[1][2], w1 * p[1][3]);
-                l0 += (bf16_lo(pa[kk][0]) + bf16_hi(pa[kk][0])) + (bf16_lo(pa[kk][2]) + bf16_hi(pa[kk][2])) +
-                      (bf16_lo(pb[kk][0]) + bf16_hi(pb[kk][0])) + (bf16_lo(pb[kk][2]) + bf16_hi(pb[kk][2]));
-                l1 += (bf16_lo(pa[kk][1]) + bf16_hi(pa[kk][1])) + (bf16_lo(pa[kk][3]) + bf16_hi(pa[kk][3])) +
-                      (bf16_lo(pb[kk][1]) + bf16_hi(pb[kk][1])) + (bf16_lo(pb[kk][3]) + bf16_hi(pb[kk][3]));
-            }
-        }
-        // ---- O += P V
-#pragma unroll
-        for (int kk = 0; kk < TT / 16; ++kk) {
-            const int mtx = lane >> 3;
-            const int row = (2 * kk + (mtx & 1)) * 8 + (lane & 7);
-#pragma unroll
-            for (int db2 = 0; db2 < D / 16; ++db2) {
-                const int c = 2 * db2 + (mtx >> 1);
+            for (int dt = 0; dt < D / 16; ++dt) {
+                const int c = dt * 2 + (mi & 1);
                 const uint32_t off = (c >> 3) * C::HALF_BYTES + swz128(row, c & 7);
-                uint32_t r0, r1, r2, r3;
-                ldsm_x4_t(vb + off, r0, r1, r2, r3);
-                mma_bf16(o[2 * db2], pa[kk], r0, r1);
-                mma_bf16(o[2 * db2 + 1], pa[kk], r2, r3);
+                uint32_t af[4];
+                ldsm_x4_t(vb + off, af[0], af[1], af[2], af[3]);
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) mma_bf16(o[dt][nb], af, pb[mt][nb][0], pb[mt][nb][1]);
                 if (MIX) {
-                    ldsm_x4_t(vb + 2 * C::TILE_BYTES + off, r0, r1, r2, r3);
-                    mma_bf16(o[2 * db2], pb[kk], r0, r1);
-                    mma_bf16(o[2 * db2 + 1], pb[kk], r2, r3);
+                    ldsm_x4_t(vb + 2 * C::TILE_BYTES + off, af[0], af[1], af[2], af[3]);
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) mma_bf16(o[dt][nb], af, pb2[mt][nb][0], pb2[mt][nb][1]);
                 }
             }
         }
@@ -253,79 +324,100 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         }
         __syncwarp();
     }
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
 
-    // ---- merge the four warps (reusing the ring; every copy issued has been consumed)
+    // ---- merge the four warps per unit (reusing the ring; every copy issued has been consumed)
     __syncthreads();
+    (void)t;
     float* comb_o = reinterpret_cast<float*>(smem);   // [NW][16][D]
-    float* comb_m = comb_o + NW * 16 * D;             // [NW][16]
-    float* comb_l = comb_m + NW * 16;                 // [NW][16]
-    float* fin_m = comb_l + NW * 16;                  // [16]
+    float* comb_ml = comb_o + NW * 16 * D;            // [NW][32]: m[16], l[16]
+    float* fin_m = comb_ml + NW * 32;                 // [16]
     float* fin_l = fin_m + 16;                        // [16]
     float* fin_o = fin_l + 16;                        // [16][D]
     float* scratch = fin_o + 16 * D;                  // merge scratch
-    {
-        const int h0 = lane >> 2;
-        const int e0 = 2 * (lane & 3);
-#pragma unroll
-        for (int db = 0; db < D / 8; ++db) {
-            float* r0p = comb_o + (warp * 16 + h0) * D + db * 8 + e0;
-            float* r1p = comb_o + (warp * 16 + h0 + 8) * D + db * 8 + e0;
-            r0p[0] = o[db][0]; r0p[1] = o[db][1];
-            r1p[0] = o[db][2]; r1p[1] = o[db][3];
+    if (cur_u >= 0) store_state(comb_o + warp * 16 * D, comb_ml + warp * 32);
+    if (lane == 0) {
+        fin_unit[warp] = cur_u;
+        sav_unit[warp] = saved_u;
+    }
+    __syncthreads();
+    const float* save_o = save;
+    const float* save_ml = save + NW * 16 * D;
+    for (int uu = u_first; uu <= u_last && span > 0; ++uu) {
+        const int u = uu;
+        // the warps' contributions to unit u: final states, and states saved at a unit switch
+        if (threadIdx.x < g) {
+            const int h = threadIdx.x;
+            float M = NEG_INF;
+            for (int ww = 0; ww < NW; ++ww) {
+                if (fin_unit[ww] == u) M = fmaxf(M, comb_ml[ww * 32 + h]);
+                if (sav_unit[ww] == u) M = fmaxf(M, save_ml[ww * 32 + h]);
+            }
+            float L = 0.f;
+            for (int ww = 0; ww < NW; ++ww) {
+                if (fin_unit[ww] == u && comb_ml[ww * 32 + h] != NEG_INF)
+                    L += exp2f(comb_ml[ww * 32 + h] - M) * comb_ml[ww * 32 + 16 + h];
+                if (sav_unit[ww] == u && save_ml[ww * 32 + h] != NEG_INF)
+                    L += exp2f(save_ml[ww * 32 + h] - M) * save_ml[ww * 32 + 16 + h];
+            }
+            fin_m[h] = M;
+            fin_l[h] = L;
         }
-        if ((lane & 3) == 0) {
-            comb_m[warp * 16 + h0] = m0;
-            comb_m[warp * 16 + h0 + 8] = m1;
-            comb_l[warp * 16 + h0] = l0;
-            comb_l[warp * 16 + h0 + 8] = l1;
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < g) {
-        const int h = threadIdx.x;
-        float M = NEG_INF;
-        for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, comb_m[ww * 16 + h]);
-        float L = 0.f;
-        for (int ww = 0; ww < NW; ++ww) L += exp2f(comb_m[ww * 16 + h] - M) * comb_l[ww * 16 + h];
-        fin_m[h] = M;
-        fin_l[h] = L;
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < g * D; idx += blockDim.x) {
-        const int h = idx / D;
-        const int e = idx % D;
-        float acc = 0.f;
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < g * D; idx += blockDim.x) {
+            const int h = idx / D;
+            const int e = idx % D;
+            float acc = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww) acc += exp2f(comb_m[ww * 16 + h] - fin_m[h]) * comb_o[(ww * 16 + h) * D + e];
-        fin_o[idx] = acc;
+            for (int ww = 0; ww < NW; ++ww) {
+                if (fin_unit[ww] == u && comb_ml[ww * 32 + h] != NEG_INF)
+                    acc += exp2f(comb_ml[ww * 32 + h] - fin_m[h]) * comb_o[(ww * 16 + h) * D + e];
+                if (sav_unit[ww] == u && save_ml[ww * 32 + h] != NEG_INF)
+                    acc += exp2f(save_ml[ww * 32 + h] - fin_m[h]) * save_o[(ww * 16 + h) * D + e];
+            }
+            fin_o[idx] = acc;
+        }
+        __syncthreads();
+        // partials of unit u: one per CTA whose range meets it, CTAs c_first .. c_last
+        const int c_first = static_cast<int>((static_cast<long long>(u) * G) / a.units);
+        const int c_last = static_cast<int>(((static_cast<long long>(u + 1) * a.n_t - 1) * G) / W);
+        const EmitPlain emit{a, D, static_cast<size_t>(u / a.Hkv) * a.Hq + static_cast<size_t>(u % a.Hkv) * g};
+        finish_unit(a, D, u, cta - c_first, c_last - c_first + 1, static_cast<long long>(u) + c_first, fin_m, fin_l,
+                    fin_o, scratch, smem + C::MERGE_STAGE_OFF,
+                    C::BODY > C::MERGE_STAGE_OFF ? C::BODY - C::MERGE_STAGE_OFF : 0, emit);
+        __syncthreads();
     }
-    __syncthreads();
-    finish_split(a, D, b, j, split, fin_m, fin_l, fin_o, scratch);
 }
 
-template <int D, bool MIX, int TT, int NSW>
-cudaError_t launch_one(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a, cudaStream_t st) {
+template <int D, bool MIX, int TT, int NSW, int NH, bool STRADDLE>
+cudaError_t launch_nh(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a, cudaStream_t st) {
     using C = DecodeCfg<D, MIX, TT, NSW>;
-    auto kern = decode_bf16_kernel<D, MIX, TT, NSW>;
+    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, NH, STRADDLE>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    dim3 grid(a.splits, a.Hkv, a.B);
-    kern<<<grid, NW * 32, C::SMEM, st>>>(tmK, tmV, a);
+    kern<<<a.splits, NW * 32, C::SMEM, st>>>(tmK, tmV, a);
     return cudaGetLastError();
+}
+
+template <int D, bool MIX, int TT, int NSW>
+cudaError_t launch_one(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a, cudaStream_t st) {
+    // with a whole number m of CTAs per unit, CTA u*m starts exactly at unit u's first
+    // tile (ceil(u*m*W/G) = u*n_t), so no range crosses a unit boundary
+    const bool aligned = a.splits % a.units == 0;
+    if (aligned)
+        return a.g <= 8 ? launch_nh<D, MIX, TT, NSW, 8, false>(tmK, tmV, a, st)
+                        : launch_nh<D, MIX, TT, NSW, 16, false>(tmK, tmV, a, st);
+    return a.g <= 8 ? launch_nh<D, MIX, TT, NSW, 8, true>(tmK, tmV, a, st)
+                    : launch_nh<D, MIX, TT, NSW, 16, true>(tmK, tmV, a, st);
 }
 
 template <int D, bool MIX, int TT, int NSW>
 int occupancy() {
     using C = DecodeCfg<D, MIX, TT, NSW>;
-    auto kern = decode_bf16_kernel<D, MIX, TT, NSW>;
+    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, 8, true>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NW * 32, C::SMEM) != cudaSuccess) return 1;
@@ -337,11 +429,35 @@ TileShape shape_of() {
     return {TT, NSW, DecodeCfg<D, MIX, TT, NSW>::SMEM};
 }
 
-// tile shapes: tokens per tile, stages per warp
-#define KVS_SHAPE_64_SINGLE 32, 3
-#define KVS_SHAPE_64_MIX 16, 3
-#define KVS_SHAPE_128_SINGLE 16, 3
-#define KVS_SHAPE_128_MIX 16, 2
+// tile shapes: tokens per tile (TT) and stages per warp (NSW) for each variant
+#ifndef KVS_TT_64S
+#define KVS_TT_64S 64
+#endif
+#ifndef KVS_NSW_64S
+#define KVS_NSW_64S 2
+#endif
+#ifndef KVS_TT_64M
+#define KVS_TT_64M 32
+#endif
+#ifndef KVS_NSW_64M
+#define KVS_NSW_64M 2
+#endif
+#ifndef KVS_TT_128S
+#define KVS_TT_128S 32
+#endif
+#ifndef KVS_NSW_128S
+#define KVS_NSW_128S 2
+#endif
+#ifndef KVS_TT_128M
+#define KVS_TT_128M 16
+#endif
+#ifndef KVS_NSW_128M
+#define KVS_NSW_128M 2
+#endif
+#define KVS_SHAPE_64_SINGLE KVS_TT_64S, KVS_NSW_64S
+#define KVS_SHAPE_64_MIX KVS_TT_64M, KVS_NSW_64M
+#define KVS_SHAPE_128_SINGLE KVS_TT_128S, KVS_NSW_128S
+#define KVS_SHAPE_128_MIX KVS_TT_128M, KVS_NSW_128M
 
 }  // namespace
 

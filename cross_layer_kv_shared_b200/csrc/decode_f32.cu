@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
     __shared__ float ss[MAX_GROUP][CH];
     __shared__ float sm_m[MAX_GROUP], sm_l[MAX_GROUP], scorr[MAX_GROUP];
     __shared__ float fin_o[MAX_GROUP * D];
-    __shared__ float scratch[MAX_GROUP * MAX_SPLITS + 2 * MAX_GROUP];
+    __shared__ float scratch[2 * MAX_GROUP * MAX_SPLITS];
     __shared__ __align__(8) uint64_t never_bar;
 
     const int split = blockIdx.x;
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
         if (idx < g * D) fin_o[idx] = acc[i];
     }
     __syncthreads();
-    finish_split(a, D, b, j, split, sm_m, sm_l, fin_o, scratch);
+    finish_split(a, D, b, j, split, sm_m, sm_l, fin_o, scratch, nullptr, 0);
 }
 
 template <int D, bool MIX>

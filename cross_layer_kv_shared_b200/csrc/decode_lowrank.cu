@@ -15,7 +15,10 @@
 //   - TMA streams coefficient tiles (64/128-B swizzle) and int8 code tiles per warp;
 //   - q~ = B_K q and q^ = R_K q are split into bf16 hi + lo halves so the score
 //     MMAs (mma.sync m16n8k16) keep ~16 bits of the fp32 projection;
-//   - int8 codes convert exactly to bf16 B operands, masked by the token's rank;
+//   - tokens are the MMA's M rows and the g heads its N columns (S^T = C q~^T),
+//     so a group of up to 8 heads wastes nothing on padding; P^T reaches the
+//     PV MMAs through an in-register transpose (movmatrix);
+//   - int8 codes convert exactly to bf16 operands, masked by the token's rank;
 //   - c^ and u^ accumulate in fp32 MMA accumulators; one projection per CTA.
 #include "kvs_device.cuh"
 
@@ -49,29 +52,63 @@ struct LrCfg {
     // per-warp scratch of per-token s_K, s_V (fp32) and rank (int)
     static constexpr int TOK_BYTES = NW * TT * 3 * 4;
     static constexpr int PD = RB + RM;    // coefficient-space partial width
-    static constexpr int COMBINE_FLOATS = NW * 16 * PD + 2 * NW * 16 + 32 + 16 * PD + 16 * D + MAX_GROUP * MAX_SPLITS + 64;
+    static constexpr int COMBINE_FLOATS = NW * 16 * PD + 2 * NW * 16 + 32 + 16 * PD + 16 * D + 2 * MAX_GROUP * MAX_SPLITS + 64;
+    static constexpr int MERGE_STAGE_OFF = ((COMBINE_FLOATS * 4 + 1023) / 1024) * 1024;   // free smem for the merge
     static constexpr int QPROJ_FLOATS = 16 * PD;
+    // staging: basis [RB][D] + residual factor [RM][D] (bf16), then the query rows [<=16][D]
+    static constexpr int STAGE_FACTORS = (RB + RM) * D * 2;
+    static constexpr int STAGE_BYTES_TOTAL = STAGE_FACTORS + 16 * D * 2;
     static constexpr int BODY0 = RING_BYTES > COMBINE_FLOATS * 4 ? RING_BYTES : COMBINE_FLOATS * 4;
-    static constexpr int SMEM = BODY0 + TOK_BYTES + QPROJ_FLOATS * 4 + 1024;
+    static constexpr int SMEM = BODY0 + TOK_BYTES + QPROJ_FLOATS * 4 + STAGE_BYTES_TOTAL + 1024;
     static_assert(TT % 16 == 0 && COEF_BYTES % 1024 == 0, "tile shape");
 };
 
-__device__ __forceinline__ uint32_t pack_i8_bf16(int a, int b) {
-    return pack_bf16(static_cast<float>(a), static_cast<float>(b));
+// Writes out = (c^ B_V + u^ R_V) / l from the merged coefficient-space sums v [g][RB + 16].
+template <int D, int RB>
+struct EmitProject {
+    const DecodeArgs& a;
+    size_t head0;
+    const uint16_t* Bv;     // [RB][D] bf16 in shared memory
+    const uint16_t* Rv;     // [16][D] bf16 in shared memory
+    __device__ void operator()(const float* v, const float* l, const float* m) const {
+        constexpr int PDV = RB + RM;
+        for (int idx = threadIdx.x; idx < a.g * D; idx += blockDim.x) {
+            const int h = idx / D;
+            const int e = idx % D;
+            float acc = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < RB; ++i) acc += v[h * PDV + i] * bf16_lo(Bv[i * D + e]);
+#pragma unroll
+            for (int i = 0; i < RM; ++i) acc += v[h * PDV + RB + i] * bf16_lo(Rv[i * D + e]);
+            a.out[(head0 + h) * D + e] = acc / l[h];
+        }
+        if (a.lse != nullptr && threadIdx.x < a.g) a.lse[head0 + threadIdx.x] = (m[threadIdx.x] + log2f(l[threadIdx.x])) * LN2_F;
+    }
+};
+
+// int8 pair (low byte = first) -> bf16 pair, each byte kept only if its flag is set
+__device__ __forceinline__ uint32_t i8pair_bf16(uint32_t w16, bool keep0, bool keep1) {
+    const int x0 = keep0 ? static_cast<int>(static_cast<int8_t>(w16 & 0xffu)) : 0;
+    const int x1 = keep1 ? static_cast<int>(static_cast<int8_t>((w16 >> 8) & 0xffu)) : 0;
+    return pack_bf16(static_cast<float>(x0), static_cast<float>(x1));
 }
 
-template <int D, int RB, int TT, int NSW>
+template <int D, int RB, int TT, int NSW, int NH>
 __global__ void __launch_bounds__(NW * 32)
 decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_constant__ CUtensorMap tmCV,
                       const __grid_constant__ CUtensorMap tmUK, const __grid_constant__ CUtensorMap tmUV,
                       const DecodeArgs a) {
     using C = LrCfg<D, RB, TT, NSW>;
     using LY = typename C::L;
+    constexpr int MT = TT / 16;
+    constexpr int NB = NH / 8;
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    float* tok = reinterpret_cast<float*>(smem + C::BODY0);                    // [NW][3][TT]
+    float* tok = reinterpret_cast<float*>(smem + C::BODY0);                    // [NW][3][TT]: s_K, s_V, rank
     float* qproj = tok + NW * TT * 3;                                          // [16][RB + RM]
+    uint8_t* stagebuf = reinterpret_cast<uint8_t*>(qproj + C::QPROJ_FLOATS);   // factors, then q rows
     __shared__ __align__(8) uint64_t bars[NW * NSW + 1];
+    __shared__ __align__(8) uint64_t fac_bar[2];    // [0]: B_K, R_K, q   [1]: B_V, R_V
 
     const int split = blockIdx.x;
     const int j = blockIdx.y;
@@ -87,67 +124,97 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     const size_t tokrow = static_cast<size_t>(b * a.Hkv + j) * a.T;   // s_K / s_V row start
     const uint8_t* rank_row = a.rank + static_cast<size_t>(b) * a.T;
 
+    const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(a.q) +
+                           (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g) * D;
     if (threadIdx.x == 0) {
         for (int i = 0; i < NW * NSW + 1; ++i) mbar_init(&bars[i], 1);
+        mbar_init(&fac_bar[0], 1);
+        mbar_init(&fac_bar[1], 1);
         mbar_init_fence();
+        // B_K[j], R_K[j] and the group's query rows, by bulk copy (all contiguous, 16-B aligned)
+        mbar_arrive_expect_tx(&fac_bar[0], C::STAGE_FACTORS + g * D * 2);
+        bulk_load(stagebuf, static_cast<const uint16_t*>(a.basis_k) + static_cast<size_t>(j) * RB * D, RB * D * 2,
+                  &fac_bar[0]);
+        bulk_load(stagebuf + RB * D * 2, static_cast<const uint16_t*>(a.r_k) + static_cast<size_t>(j) * RM * D,
+                  RM * D * 2, &fac_bar[0]);
+        bulk_load(stagebuf + C::STAGE_FACTORS, qsrc, g * D * 2, &fac_bar[0]);
     }
-    // ---- q~ = B_K q and q^ = R_K q for the g heads (fp32, into shared memory)
+    for (int idx = g * C::PD + threadIdx.x; idx < 16 * C::PD; idx += blockDim.x) qproj[idx] = 0.f;
+    __syncthreads();
+    // ---- q~ = B_K q and q^ = R_K q for the g heads: one warp per output, lanes over d
+    mbar_wait_bounded(&fac_bar[0], 0, a.wait_limit, a.err);
     {
-        const uint16_t* qb = reinterpret_cast<const uint16_t*>(a.q) +
-                             (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g) * D;
-        const uint16_t* Bk = reinterpret_cast<const uint16_t*>(a.basis_k) + static_cast<size_t>(j) * RB * D;
-        const uint16_t* Rk = reinterpret_cast<const uint16_t*>(a.r_k) + static_cast<size_t>(j) * RM * D;
-        for (int idx = threadIdx.x; idx < 16 * C::PD; idx += blockDim.x) {
+        const uint16_t* fac = reinterpret_cast<const uint16_t*>(stagebuf);
+        const uint16_t* qs = reinterpret_cast<const uint16_t*>(stagebuf + C::STAGE_FACTORS);
+        for (int idx = warp; idx < g * C::PD; idx += NW) {
             const int h = idx / C::PD;
             const int i = idx % C::PD;
             float acc = 0.f;
-            if (h < g) {
-                const uint16_t* row = i < RB ? Bk + static_cast<size_t>(i) * D : Rk + static_cast<size_t>(i - RB) * D;
-                for (int e = 0; e < D; e += 2) {
+            {
+                const uint16_t* row = fac + static_cast<size_t>(i) * D;     // basis rows, then factor rows
+                for (int e = 2 * lane; e < D; e += 64) {
                     const uint32_t bw = *reinterpret_cast<const uint32_t*>(row + e);
-                    const uint32_t qw = *reinterpret_cast<const uint32_t*>(qb + h * D + e);
-                    acc += bf16_lo(bw) * bf16_lo(qw);
-                    acc += bf16_hi(bw) * bf16_hi(qw);
+                    const uint32_t qw = *reinterpret_cast<const uint32_t*>(qs + h * D + e);
+                    acc += bf16_lo(bw) * bf16_lo(qw) + bf16_hi(bw) * bf16_hi(qw);
                 }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
             }
-            qproj[idx] = acc;
+            if (lane == 0) qproj[idx] = acc;
         }
     }
     __syncthreads();
+    if (threadIdx.x == 0) {
+        // B_V[j], R_V[j] for the final projection, landing while the tiles stream
+        fence_proxy_async();
+        mbar_arrive_expect_tx(&fac_bar[1], C::STAGE_FACTORS);
+        bulk_load(stagebuf, static_cast<const uint16_t*>(a.basis_v) + static_cast<size_t>(j) * RB * D, RB * D * 2,
+                  &fac_bar[1]);
+        bulk_load(stagebuf + RB * D * 2, static_cast<const uint16_t*>(a.r_v) + static_cast<size_t>(j) * RM * D,
+                  RM * D * 2, &fac_bar[1]);
+    }
     if (a.stall && threadIdx.x == 0) mbar_wait_bounded(&bars[NW * NSW], 0, a.stall_limit, a.err);
 
-    // A fragments: rows = heads; q~ (RB wide) and q^ (16 wide), each as bf16 hi + lo
-    uint32_t qc_hi[RB / 16][4], qc_lo[RB / 16][4], qu_hi[4], qu_lo[4];
+    // B fragments of q~^T (RB rows) and q^^T (16 rows): column = head nb*8 + lane/4, as bf16 hi + lo
+    uint32_t qch[RB / 16][NB][2], qcl[RB / 16][NB][2], quh[NB][2], qul[NB][2];
     {
-        const int h0 = lane >> 2;
         const int cq = 2 * (lane & 3);
-        auto frag = [&](int col0, uint32_t (&hi)[4], uint32_t (&lo)[4]) {
-            const int cols[4] = {col0 + cq, col0 + cq, col0 + 8 + cq, col0 + 8 + cq};
-            const int rows[4] = {h0, h0 + 8, h0, h0 + 8};
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const float x0 = qproj[rows[r] * C::PD + cols[r]];
-                const float x1 = qproj[rows[r] * C::PD + cols[r] + 1];
-                hi[r] = pack_bf16(x0, x1);
-                lo[r] = pack_bf16(x0 - bf16_lo(hi[r]), x1 - bf16_hi(hi[r]));
+        for (int nb = 0; nb < NB; ++nb) {
+            const int h = nb * 8 + (lane >> 2);
+            auto frag = [&](int col, uint32_t& hi, uint32_t& lo) {
+                const float x0 = qproj[h * C::PD + col];
+                const float x1 = qproj[h * C::PD + col + 1];
+                hi = pack_bf16(x0, x1);
+                lo = pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
+            };
+#pragma unroll
+            for (int ks = 0; ks < RB / 16; ++ks) {
+                frag(ks * 16 + cq, qch[ks][nb][0], qcl[ks][nb][0]);
+                frag(ks * 16 + 8 + cq, qch[ks][nb][1], qcl[ks][nb][1]);
             }
-        };
-#pragma unroll
-        for (int kk = 0; kk < RB / 16; ++kk) frag(kk * 16, qc_hi[kk], qc_lo[kk]);
-        frag(RB, qu_hi, qu_lo);
+            frag(RB + cq, quh[nb][0], qul[nb][0]);
+            frag(RB + 8 + cq, quh[nb][1], qul[nb][1]);
+        }
     }
 
-    float cacc[RB / 8][4];
-    float uacc[2][4];
+    // accumulators c^^T (RB rows) and u^^T (16 rows), columns = heads
+    float oc[RB / 16][NB][4];
+    float ou[NB][4];
 #pragma unroll
-    for (int i = 0; i < RB / 8; ++i) cacc[i][0] = cacc[i][1] = cacc[i][2] = cacc[i][3] = 0.f;
+    for (int nb = 0; nb < NB; ++nb) {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) uacc[i][0] = uacc[i][1] = uacc[i][2] = uacc[i][3] = 0.f;
-    float m0 = NEG_INF, m1 = NEG_INF, l0 = 0.f, l1 = 0.f;
+        for (int i = 0; i < RB / 16; ++i) oc[i][nb][0] = oc[i][nb][1] = oc[i][nb][2] = oc[i][nb][3] = 0.f;
+        ou[nb][0] = ou[nb][1] = ou[nb][2] = ou[nb][3] = 0.f;
+    }
+    float mrow[NB][2], lrow[NB][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) mrow[nb][0] = mrow[nb][1] = NEG_INF, lrow[nb][0] = lrow[nb][1] = 0.f;
 
     uint8_t* ring = smem + warp * NSW * C::STAGE_BYTES;
     uint64_t* wb = &bars[warp * NSW];
     float* tks = tok + warp * TT * 3;     // [3][TT]: s_K, s_V, rank
+    int* tkr = reinterpret_cast<int*>(tks + 2 * TT);
     const int span = tile1 - tile0;
     const int my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
 
@@ -166,7 +233,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     };
     // per-token scales and ranks of a tile, loaded by the lanes (tokens lane, lane+32, ...)
     constexpr int TPL = TT / 32;
-    float pf_sk[TPL], pf_sv[TPL], pf_r[TPL];
+    float pf_sk[TPL], pf_sv[TPL];
+    int pf_r[TPL];
     auto prefetch = [&](int k) {
         const int t0 = (tile0 + warp + k * NW) * TT;
 #pragma unroll
@@ -175,9 +243,9 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             if (t < a.T) {
                 pf_sk[u] = __half2float(__ushort_as_half(__ldg(a.s_k + tokrow + t)));
                 pf_sv[u] = __half2float(__ushort_as_half(__ldg(a.s_v + tokrow + t)));
-                pf_r[u] = static_cast<float>(__ldg(rank_row + t));
+                pf_r[u] = static_cast<int>(__ldg(rank_row + t));
             } else {
-                pf_sk[u] = 0.f; pf_sv[u] = 0.f; pf_r[u] = 0.f;
+                pf_sk[u] = 0.f; pf_sv[u] = 0.f; pf_r[u] = 0;
             }
         }
     };
@@ -187,6 +255,9 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     if (my_n > 0) prefetch(0);
     __syncwarp();
 
+    const int mi = lane >> 3;
+    const int ri = lane & 7;
+    const int q4 = lane & 3;
     for (int k = 0; k < my_n; ++k) {
         const int s = k % NSW;
         // publish this tile's per-token values, start fetching the next tile's
@@ -195,7 +266,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         for (int u = 0; u < TPL; ++u) {
             tks[lane + 32 * u] = pf_sk[u];
             tks[TT + lane + 32 * u] = pf_sv[u];
-            tks[2 * TT + lane + 32 * u] = pf_r[u];
+            tkr[lane + 32 * u] = pf_r[u];
         }
         if (k + 1 < my_n) prefetch(k + 1);
         __syncwarp();
@@ -211,118 +282,121 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         const uint8_t* ukp = ring + s * C::STAGE_BYTES + 2 * C::COEF_BYTES;
         const uint8_t* uvp = ukp + C::U_BYTES;
 
-        float sc[TT / 8][4];
-        float su[TT / 8][4];
+        float sc[MT][NB][4];
+        float su[MT][NB][4];
 #pragma unroll
-        for (int nb = 0; nb < TT / 8; ++nb) {
-            sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
-            su[nb][0] = su[nb][1] = su[nb][2] = su[nb][3] = 0.f;
-        }
-        // ---- basis part of the scores: C_K q~ (hi and lo)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int kk2 = 0; kk2 < RB / 32; ++kk2) {
-            const int c = kk2 * 4 + (lane >> 3);
+            for (int nb = 0; nb < NB; ++nb) {
+                sc[mt][nb][0] = sc[mt][nb][1] = sc[mt][nb][2] = sc[mt][nb][3] = 0.f;
+                su[mt][nb][0] = su[mt][nb][1] = su[mt][nb][2] = su[mt][nb][3] = 0.f;
+            }
+        // ---- basis part of the scores: C_K q~^T (hi and lo)
 #pragma unroll
-            for (int nb = 0; nb < TT / 8; ++nb) {
-                const int row = nb * 8 + (lane & 7);
-                uint32_t r0, r1, r2, r3;
-                ldsm_x4(ckb + LY::template off<TT>(row, c), r0, r1, r2, r3);
-                mma_bf16(sc[nb], qc_hi[2 * kk2], r0, r1);
-                mma_bf16(sc[nb], qc_lo[2 * kk2], r0, r1);
-                mma_bf16(sc[nb], qc_hi[2 * kk2 + 1], r2, r3);
-                mma_bf16(sc[nb], qc_lo[2 * kk2 + 1], r2, r3);
+        for (int mt = 0; mt < MT; ++mt) {
+            const int row = mt * 16 + (mi & 1) * 8 + ri;
+#pragma unroll
+            for (int ks = 0; ks < RB / 16; ++ks) {
+                uint32_t af[4];
+                ldsm_x4(ckb + LY::template off<TT>(row, ks * 2 + (mi >> 1)), af[0], af[1], af[2], af[3]);
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    mma_bf16(sc[mt][nb], af, qch[ks][nb][0], qch[ks][nb][1]);
+                    mma_bf16(sc[mt][nb], af, qcl[ks][nb][0], qcl[ks][nb][1]);
+                }
             }
         }
-        // ---- residual part: U_K (masked to the token's rank) q^
+        // ---- residual part: U_K (masked to each token's rank) q^^T
 #pragma unroll
-        for (int nb = 0; nb < TT / 8; ++nb) {
-            const int tt = nb * 8 + (lane >> 2);
-            const int r = static_cast<int>(tks[2 * TT + tt]);
-            const int i0 = 2 * (lane & 3);
-            const int8_t* up = reinterpret_cast<const int8_t*>(ukp + tt * RM);
-            const uint32_t b0 = pack_i8_bf16(i0 < r ? up[i0] : 0, i0 + 1 < r ? up[i0 + 1] : 0);
-            const uint32_t b1 = pack_i8_bf16(i0 + 8 < r ? up[i0 + 8] : 0, i0 + 9 < r ? up[i0 + 9] : 0);
-            mma_bf16(su[nb], qu_hi, b0, b1);
-            mma_bf16(su[nb], qu_lo, b0, b1);
-        }
-        // ---- scores, mask, online softmax
-        const int tb = 2 * (lane & 3);
-        float mx0 = NEG_INF, mx1 = NEG_INF;
+        for (int mt = 0; mt < MT; ++mt) {
+            const int ta = mt * 16 + (lane >> 2);
+            const int ra = tkr[ta], rb = tkr[ta + 8];
+            const uint16_t* ua = reinterpret_cast<const uint16_t*>(ukp + ta * RM);
+            const uint16_t* ub = reinterpret_cast<const uint16_t*>(ukp + (ta + 8) * RM);
+            uint32_t af[4];
+            af[0] = i8pair_bf16(ua[q4], 2 * q4 < ra, 2 * q4 + 1 < ra);
+            af[1] = i8pair_bf16(ub[q4], 2 * q4 < rb, 2 * q4 + 1 < rb);
+            af[2] = i8pair_bf16(ua[q4 + 4], 2 * q4 + 8 < ra, 2 * q4 + 9 < ra);
+            af[3] = i8pair_bf16(ub[q4 + 4], 2 * q4 + 8 < rb, 2 * q4 + 9 < rb);
 #pragma unroll
-        for (int nb = 0; nb < TT / 8; ++nb) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int tt = nb * 8 + tb + (i & 1);
-                float v = (sc[nb][i] + tks[tt] * su[nb][i]) * a.scale_log2;
-                if (t * TT + tt >= a.T) v = NEG_INF;
-                sc[nb][i] = v;
-                if (i < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
+            for (int nb = 0; nb < NB; ++nb) {
+                mma_bf16(su[mt][nb], af, quh[nb][0], quh[nb][1]);
+                mma_bf16(su[mt][nb], af, qul[nb][0], qul[nb][1]);
             }
         }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
-        const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
-        const float cr0 = exp2f(m0 - ref0), cr1 = exp2f(m1 - ref1);
-        m0 = mn0;
-        m1 = mn1;
-        l0 *= cr0;
-        l1 *= cr1;
+        // ---- scores, mask, online softmax per head; P^T and (P s_V)^T by movmatrix
+        uint32_t pb[MT][NB][2], pvb[MT][NB][2];
 #pragma unroll
-        for (int i = 0; i < RB / 8; ++i) { cacc[i][0] *= cr0; cacc[i][1] *= cr0; cacc[i][2] *= cr1; cacc[i][3] *= cr1; }
+        for (int nb = 0; nb < NB; ++nb) {
+            float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) { uacc[i][0] *= cr0; uacc[i][1] *= cr0; uacc[i][2] *= cr1; uacc[i][3] *= cr1; }
-
+            for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
-        for (int kk = 0; kk < TT / 16; ++kk) {
-            float p[2][4];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                p[u][0] = exp2f(sc[2 * kk + u][0] - ref0);
-                p[u][1] = exp2f(sc[2 * kk + u][1] - ref0);
-                p[u][2] = exp2f(sc[2 * kk + u][2] - ref1);
-                p[u][3] = exp2f(sc[2 * kk + u][3] - ref1);
+                for (int i = 0; i < 4; ++i) {
+                    const int tt = mt * 16 + (lane >> 2) + (i >> 1) * 8;
+                    float v = (sc[mt][nb][i] + tks[tt] * su[mt][nb][i]) * a.scale_log2;
+                    if (t * TT + tt >= a.T) v = NEG_INF;
+                    sc[mt][nb][i] = v;
+                    if (i & 1) mx1 = fmaxf(mx1, v); else mx0 = fmaxf(mx0, v);
+                }
             }
-            uint32_t pa[4], pv[4];
-            pa[0] = pack_bf16(p[0][0], p[0][1]);
-            pa[1] = pack_bf16(p[0][2], p[0][3]);
-            pa[2] = pack_bf16(p[1][0], p[1][1]);
-            pa[3] = pack_bf16(p[1][2], p[1][3]);
-            l0 += (bf16_lo(pa[0]) + bf16_hi(pa[0])) + (bf16_lo(pa[2]) + bf16_hi(pa[2]));
-            l1 += (bf16_lo(pa[1]) + bf16_hi(pa[1])) + (bf16_lo(pa[3]) + bf16_hi(pa[3]));
-            // p * s_V for the residual accumulation
-            const int ta = kk * 16 + tb;                 // tokens ta, ta+1 and ta+8, ta+9
-            const float sv0 = tks[TT + ta], sv1 = tks[TT + ta + 1];
-            const float sv8 = tks[TT + ta + 8], sv9 = tks[TT + ta + 9];
-            pv[0] = pack_bf16(p[0][0] * sv0, p[0][1] * sv1);
-            pv[1] = pack_bf16(p[0][2] * sv0, p[0][3] * sv1);
-            pv[2] = pack_bf16(p[1][0] * sv8, p[1][1] * sv9);
-            pv[3] = pack_bf16(p[1][2] * sv8, p[1][3] * sv9);
-            // c^ += P C_V
-            const int mtx = lane >> 3;
-            const int row = (2 * kk + (mtx & 1)) * 8 + (lane & 7);
 #pragma unroll
-            for (int cb2 = 0; cb2 < RB / 16; ++cb2) {
-                const int c = 2 * cb2 + (mtx >> 1);
-                uint32_t r0, r1, r2, r3;
-                ldsm_x4_t(cvb + LY::template off<TT>(row, c), r0, r1, r2, r3);
-                mma_bf16(cacc[2 * cb2], pa, r0, r1);
-                mma_bf16(cacc[2 * cb2 + 1], pa, r2, r3);
+            for (int off = 4; off < 32; off <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
             }
-            // u^ += (P s_V) U_V, codes masked to each token's rank
-            const int r0t = static_cast<int>(tks[2 * TT + ta]), r1t = static_cast<int>(tks[2 * TT + ta + 1]);
-            const int r8t = static_cast<int>(tks[2 * TT + ta + 8]), r9t = static_cast<int>(tks[2 * TT + ta + 9]);
+            const float mn0 = fmaxf(mrow[nb][0], mx0), mn1 = fmaxf(mrow[nb][1], mx1);
+            const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
+            const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
+            const float cr0 = exp2f(mrow[nb][0] - ref0), cr1 = exp2f(mrow[nb][1] - ref1);
+            mrow[nb][0] = mn0;
+            mrow[nb][1] = mn1;
+            lrow[nb][0] *= cr0;
+            lrow[nb][1] *= cr1;
+#pragma unroll
+            for (int i = 0; i < RB / 16; ++i) { oc[i][nb][0] *= cr0; oc[i][nb][2] *= cr0; oc[i][nb][1] *= cr1; oc[i][nb][3] *= cr1; }
+            ou[nb][0] *= cr0; ou[nb][2] *= cr0; ou[nb][1] *= cr1; ou[nb][3] *= cr1;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int ta = mt * 16 + (lane >> 2);
+                const float p0 = exp2f(sc[mt][nb][0] - ref0), p1 = exp2f(sc[mt][nb][1] - ref1);
+                const float p2 = exp2f(sc[mt][nb][2] - ref0), p3 = exp2f(sc[mt][nb][3] - ref1);
+                const uint32_t lo = pack_bf16(p0, p1), hi = pack_bf16(p2, p3);
+                lrow[nb][0] += bf16_lo(lo) + bf16_lo(hi);
+                lrow[nb][1] += bf16_hi(lo) + bf16_hi(hi);
+                pb[mt][nb][0] = movmatrix_t(lo);
+                pb[mt][nb][1] = movmatrix_t(hi);
+                const float sva = tks[TT + ta], svb = tks[TT + ta + 8];
+                pvb[mt][nb][0] = movmatrix_t(pack_bf16(p0 * sva, p1 * sva));
+                pvb[mt][nb][1] = movmatrix_t(pack_bf16(p2 * svb, p3 * svb));
+            }
+        }
+        // ---- c^^T += C_V^T P^T
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int row = mt * 16 + (mi >> 1) * 8 + ri;
+#pragma unroll
+            for (int ct = 0; ct < RB / 16; ++ct) {
+                uint32_t af[4];
+                ldsm_x4_t(cvb + LY::template off<TT>(row, ct * 2 + (mi & 1)), af[0], af[1], af[2], af[3]);
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) mma_bf16(oc[ct][nb], af, pb[mt][nb][0], pb[mt][nb][1]);
+            }
+        }
+        // ---- u^^T += U_V^T (P s_V)^T, codes masked to each token's rank
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int t0 = mt * 16 + 2 * q4;                 // tokens t0, t0+1 and t0+8, t0+9
+            const int r0 = tkr[t0], r1 = tkr[t0 + 1], r8 = tkr[t0 + 8], r9 = tkr[t0 + 9];
             const int8_t* uv = reinterpret_cast<const int8_t*>(uvp);
+            const int i = lane >> 2;                         // channel rows i and i + 8
+            uint32_t af[4];
+            af[0] = pack_bf16(i < r0 ? uv[t0 * RM + i] : 0, i < r1 ? uv[(t0 + 1) * RM + i] : 0);
+            af[1] = pack_bf16(i + 8 < r0 ? uv[t0 * RM + i + 8] : 0, i + 8 < r1 ? uv[(t0 + 1) * RM + i + 8] : 0);
+            af[2] = pack_bf16(i < r8 ? uv[(t0 + 8) * RM + i] : 0, i < r9 ? uv[(t0 + 9) * RM + i] : 0);
+            af[3] = pack_bf16(i + 8 < r8 ? uv[(t0 + 8) * RM + i + 8] : 0, i + 8 < r9 ? uv[(t0 + 9) * RM + i + 8] : 0);
 #pragma unroll
-            for (int nbi = 0; nbi < 2; ++nbi) {
-                const int i = nbi * 8 + (lane >> 2);
-                const uint32_t b0 = pack_i8_bf16(i < r0t ? uv[ta * RM + i] : 0, i < r1t ? uv[(ta + 1) * RM + i] : 0);
-                const uint32_t b1 = pack_i8_bf16(i < r8t ? uv[(ta + 8) * RM + i] : 0, i < r9t ? uv[(ta + 9) * RM + i] : 0);
-                mma_bf16(uacc[nbi], pv, b0, b1);
-            }
+            for (int nb = 0; nb < NB; ++nb) mma_bf16(ou[nb], af, pvb[mt][nb][0], pvb[mt][nb][1]);
         }
         __syncwarp();
         if (lane == 0 && k + NSW < my_n) {
@@ -330,10 +404,13 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             issue(k + NSW);
         }
     }
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            lrow[nb][0] += __shfl_xor_sync(0xffffffffu, lrow[nb][0], off);
+            lrow[nb][1] += __shfl_xor_sync(0xffffffffu, lrow[nb][1], off);
+        }
 
     // ---- merge warps in coefficient space, project once, finish the split
     __syncthreads();
@@ -347,27 +424,27 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     float* fin_o = fin_c + 16 * PD;                 // [16][D]
     float* scratch = fin_o + 16 * D;
     {
-        const int h0 = lane >> 2;
-        const int e0 = 2 * (lane & 3);
+        const int e0 = lane >> 2;
 #pragma unroll
-        for (int cb = 0; cb < RB / 8; ++cb) {
-            float* p0 = comb + (warp * 16 + h0) * PD + cb * 8 + e0;
-            float* p1 = comb + (warp * 16 + h0 + 8) * PD + cb * 8 + e0;
-            p0[0] = cacc[cb][0]; p0[1] = cacc[cb][1];
-            p1[0] = cacc[cb][2]; p1[1] = cacc[cb][3];
-        }
+        for (int nb = 0; nb < NB; ++nb) {
+            const int h0 = nb * 8 + 2 * q4;
 #pragma unroll
-        for (int ub = 0; ub < 2; ++ub) {
-            float* p0 = comb + (warp * 16 + h0) * PD + RB + ub * 8 + e0;
-            float* p1 = comb + (warp * 16 + h0 + 8) * PD + RB + ub * 8 + e0;
-            p0[0] = uacc[ub][0]; p0[1] = uacc[ub][1];
-            p1[0] = uacc[ub][2]; p1[1] = uacc[ub][3];
-        }
-        if ((lane & 3) == 0) {
-            comb_m[warp * 16 + h0] = m0;
-            comb_m[warp * 16 + h0 + 8] = m1;
-            comb_l[warp * 16 + h0] = l0;
-            comb_l[warp * 16 + h0 + 8] = l1;
+            for (int ct = 0; ct < RB / 16; ++ct) {
+                comb[(warp * 16 + h0) * PD + ct * 16 + e0] = oc[ct][nb][0];
+                comb[(warp * 16 + h0) * PD + ct * 16 + e0 + 8] = oc[ct][nb][2];
+                comb[(warp * 16 + h0 + 1) * PD + ct * 16 + e0] = oc[ct][nb][1];
+                comb[(warp * 16 + h0 + 1) * PD + ct * 16 + e0 + 8] = oc[ct][nb][3];
+            }
+            comb[(warp * 16 + h0) * PD + RB + e0] = ou[nb][0];
+            comb[(warp * 16 + h0) * PD + RB + e0 + 8] = ou[nb][2];
+            comb[(warp * 16 + h0 + 1) * PD + RB + e0] = ou[nb][1];
+            comb[(warp * 16 + h0 + 1) * PD + RB + e0 + 8] = ou[nb][3];
+            if (lane < 4) {
+                comb_m[warp * 16 + h0] = mrow[nb][0];
+                comb_m[warp * 16 + h0 + 1] = mrow[nb][1];
+                comb_l[warp * 16 + h0] = lrow[nb][0];
+                comb_l[warp * 16 + h0 + 1] = lrow[nb][1];
+            }
         }
     }
     __syncthreads();
@@ -376,7 +453,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         float M = NEG_INF;
         for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, comb_m[ww * 16 + h]);
         float L = 0.f;
-        for (int ww = 0; ww < NW; ++ww) L += exp2f(comb_m[ww * 16 + h] - M) * comb_l[ww * 16 + h];
+        for (int ww = 0; ww < NW; ++ww)
+            if (comb_m[ww * 16 + h] != NEG_INF) L += exp2f(comb_m[ww * 16 + h] - M) * comb_l[ww * 16 + h];
         fin_m[h] = M;
         fin_l[h] = L;
     }
@@ -385,30 +463,26 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         const int h = idx / PD;
         float acc = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww) acc += exp2f(comb_m[ww * 16 + h] - fin_m[h]) * comb[(ww * 16 + h) * PD + (idx % PD)];
+        for (int ww = 0; ww < NW; ++ww)
+            if (comb_m[ww * 16 + h] != NEG_INF)
+                acc += exp2f(comb_m[ww * 16 + h] - fin_m[h]) * comb[(ww * 16 + h) * PD + (idx % PD)];
         fin_c[idx] = acc;
     }
     __syncthreads();
-    {
-        const uint16_t* Bv = reinterpret_cast<const uint16_t*>(a.basis_v) + static_cast<size_t>(j) * RB * D;
-        const uint16_t* Rv = reinterpret_cast<const uint16_t*>(a.r_v) + static_cast<size_t>(j) * RM * D;
-        for (int idx = threadIdx.x; idx < g * D; idx += blockDim.x) {
-            const int h = idx / D;
-            const int e = idx % D;
-            float acc = 0.f;
-            for (int i = 0; i < RB; ++i) acc += fin_c[h * PD + i] * bf16_lo(Bv[static_cast<size_t>(i) * D + e]);
-            for (int i = 0; i < RM; ++i) acc += fin_c[h * PD + RB + i] * bf16_lo(Rv[static_cast<size_t>(i) * D + e]);
-            fin_o[idx] = acc;
-        }
-    }
-    __syncthreads();
-    finish_split(a, D, b, j, split, fin_m, fin_l, fin_o, scratch);
+    // partials stay in coefficient space (RB + 16 values per head); the CTA that
+    // finishes the unit projects once: o = (c^ B_V + u^ R_V) / l
+    mbar_wait_bounded(&fac_bar[1], 0, a.wait_limit, a.err);
+    const uint16_t* Bv = reinterpret_cast<const uint16_t*>(stagebuf);
+    const EmitProject<D, RB> emit{a, static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g, Bv, Bv + RB * D};
+    const int unit = b * a.Hkv + j;
+    finish_unit(a, PD, unit, split, a.splits, static_cast<long long>(unit) * a.splits, fin_m, fin_l, fin_c, scratch,
+                smem + C::MERGE_STAGE_OFF, C::BODY0 > C::MERGE_STAGE_OFF ? C::BODY0 - C::MERGE_STAGE_OFF : 0, emit);
 }
 
-template <int D, int RB, int TT, int NSW>
-cudaError_t launch_one(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
+template <int D, int RB, int TT, int NSW, int NH>
+cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
     using C = LrCfg<D, RB, TT, NSW>;
-    auto kern = decode_lowrank_kernel<D, RB, TT, NSW>;
+    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NH>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -421,9 +495,14 @@ cudaError_t launch_one(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_
 }
 
 template <int D, int RB, int TT, int NSW>
+cudaError_t launch_one(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
+    return a.g <= 8 ? launch_nh<D, RB, TT, NSW, 8>(a, maps, st) : launch_nh<D, RB, TT, NSW, 16>(a, maps, st);
+}
+
+template <int D, int RB, int TT, int NSW>
 int occupancy_of() {
     using C = LrCfg<D, RB, TT, NSW>;
-    auto kern = decode_lowrank_kernel<D, RB, TT, NSW>;
+    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, 8>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NW * 32, C::SMEM) != cudaSuccess) return 1;
@@ -431,10 +510,16 @@ int occupancy_of() {
 }
 
 // token tile and stages per warp by basis rank (the full-rank basis only serves tests)
+#ifndef KVS_LR_TT
+#define KVS_LR_TT 64
+#endif
+#ifndef KVS_LR_NSW
+#define KVS_LR_NSW 2
+#endif
 template <int RB>
 struct LrShape {
-    static constexpr int TT = RB == 128 ? 32 : 64;
-    static constexpr int NSW = RB == 128 ? 1 : 2;
+    static constexpr int TT = RB == 128 ? 32 : KVS_LR_TT;
+    static constexpr int NSW = RB == 128 ? 1 : KVS_LR_NSW;
 };
 
 template <int D, int RB>

@@ -13,7 +13,7 @@
 // GPU which loads this library holds until the process exits. It holds the
 // arrival counters (one per batch x kv-head unit, at most KVS_NOALLOC_MAX_UNITS),
 // a status word, and the split partials. Requests with more units are rejected;
-// the split count is lowered until the partials fit.
+// the CTA count is lowered until the partials fit.
 #include "kvshare.h"
 
 #include <cuda.h>
@@ -126,13 +126,15 @@ extern "C" kvshare_status kvshare_decode_layer_noalloc(const void* q, const void
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const TileShape ts = decode_bf16_shape(head_dim, mix);
-    const int tiles = (context + ts.tt - 1) / ts.tt;
-    int splits = (sms * decode_bf16_ctas_per_sm(head_dim, mix)) / static_cast<int>(units);
-    if (splits < 1) splits = 1;
-    if (splits > tiles) splits = tiles;
-    if (splits > MAX_SPLITS) splits = MAX_SPLITS;
-    const size_t per_split = static_cast<size_t>(units) * g * (head_dim + 2);
-    while (splits > 1 && per_split * splits > PARTIAL_FLOATS) --splits;
+    // balanced grid: the units' token tiles cut into G equal ranges, one CTA each; a
+    // unit spread over several CTAs keeps one partial per CTA in the array
+    const int n_t = (context + ts.tt - 1) / ts.tt;
+    const long long W = units * n_t;
+    const long long per_unit = (static_cast<long long>(sms) * decode_bf16_ctas_per_sm(head_dim, mix)) / units;
+    long long G = units * (per_unit > 1 ? per_unit : 1);
+    if (G > W) G = W;
+    const size_t per = static_cast<size_t>(g) * (head_dim + 4);
+    while (G > units && (static_cast<size_t>(units) + G) * per > PARTIAL_FLOATS) --G;
 
     DecodeArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -149,8 +151,9 @@ extern "C" kvshare_status kvshare_decode_layer_noalloc(const void* q, const void
     a.Hkv = num_kv_heads;
     a.T = context;
     a.g = g;
-    a.tiles_per_split = (tiles + splits - 1) / splits;
-    a.splits = (tiles + a.tiles_per_split - 1) / a.tiles_per_split;
+    a.units = static_cast<int>(units);
+    a.n_t = n_t;
+    a.splits = static_cast<int>(G);
     a.scale_log2 = (1.0f / std::sqrt(static_cast<float>(head_dim))) * 1.4426950408889634f;
     a.ws = partials;
     a.counters = counters;

@@ -78,6 +78,20 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// 3-D tiled bulk tensor store shared -> global (rows outside the tensor are not written).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Plain (untiled) bulk copy global -> shared; both addresses 16-B aligned, bytes % 16 == 0.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
     asm volatile(
@@ -111,6 +125,14 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Transpose an 8x8 matrix of 16-bit values held one pair per thread (thread t owns
+// row t/4, columns 2(t%4), 2(t%4)+1) so that thread t owns row t/4 of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -126,74 +148,176 @@ __device__ __forceinline__ uint32_t swz128(int row, int c) {
 }
 
 // ------------------------------------------------------------------ split merge
+// Partial layout: [unit][split][head][D + 4] floats: o[0..D), m, l, two pad words
+// (rows stay 16-byte aligned so whole partial blocks can move by bulk copy).
+__host__ __device__ constexpr int partial_width(int D) { return D + 4; }
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
 // Every decode CTA ends here with, in shared memory, for its g query heads:
 //   sm_m[h]  running max of the log2-domain scores,
 //   sm_l[h]  sum of 2^(s - m) weights,
-//   sm_o[h][e] un-normalised output sum_t 2^(s_t - m) V_t.
-// With one split the CTA writes out = o / l and lse = (m + log2 l) ln 2.
-// Otherwise it stores its partial and the last CTA of the (b, kv head) to
-// arrive merges all partials: M = max m_s, l = sum 2^(m_s - M) l_s,
-// o = sum 2^(m_s - M) o_s / l. That CTA resets the arrival counter to zero.
-__device__ inline void finish_split(const DecodeArgs& a, int D, int b, int j, int split, const float* sm_m,
-                                    const float* sm_l, const float* sm_o, float* sm_scratch /* >= g*MAX_SPLITS */) {
+//   sm_v[h][e] un-normalised accumulated vector (e < DV): the output
+//            sum_t 2^(s_t - m) V_t, or the low-rank form's coefficient-space sums.
+// With one partial per unit the CTA emits it at once. Otherwise it stores its
+// partial and the last CTA of the unit to arrive merges all partials:
+// M = max m_s, l = sum 2^(m_s - M) l_s, v = sum 2^(m_s - M) v_s, then emits
+// (and resets the unit's arrival counter to zero). The merge is parallel:
+// every thread loads (m, l) pairs, one warp per head reduces them, and the
+// partial blocks are bulk-copied into `stage` (free shared memory of
+// `stage_bytes`, 16-B aligned; 0 means read them directly).
+// `emit(v, l, m)` writes the unit's outputs from v [g][DV] (shared memory),
+// l[g] and m[g]; it is called by all threads of the CTA.
+// sm_scratch holds at least 2 * g * count floats; sm_v is reused for the merge.
+struct EmitPlain {
+    const DecodeArgs& a;
+    int D;
+    size_t head0;
+    __device__ void operator()(const float* v, const float* l, const float* m) const {
+        for (int idx = threadIdx.x; idx < a.g * D; idx += blockDim.x)
+            a.out[(head0 + idx / D) * D + (idx % D)] = v[idx] / l[idx / D];
+        if (a.lse != nullptr && threadIdx.x < a.g) a.lse[head0 + threadIdx.x] = (m[threadIdx.x] + log2f(l[threadIdx.x])) * LN2_F;
+    }
+};
+
+template <typename Emit>
+__device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int index, int count, long long slot0,
+                                   const float* sm_m, const float* sm_l, float* sm_v, float* sm_scratch,
+                                   uint8_t* stage, int stage_bytes, const Emit& emit) {
     const int g = a.g;
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;
-    const size_t head0 = static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g;
-    if (a.splits == 1) {
-        for (int idx = tid; idx < g * D; idx += nthr) {
-            const int h = idx / D;
-            a.out[(head0 + h) * D + (idx % D)] = sm_o[idx] / sm_l[h];
-        }
-        if (a.lse != nullptr && tid < g) a.lse[head0 + tid] = (sm_m[tid] + log2f(sm_l[tid])) * LN2_F;
+    if (count == 1) {
+        emit(sm_v, sm_l, sm_m);
         return;
     }
-    const int PD = D + 2;
-    const size_t unit = static_cast<size_t>(b) * a.Hkv + j;
-    float* part = a.ws + (unit * a.splits + split) * static_cast<size_t>(g * PD);
-    for (int idx = tid; idx < g * D; idx += nthr) part[(idx / D) * PD + (idx % D)] = sm_o[idx];
+    const int PD = partial_width(DV);
+    const int per = g * PD;
+    const size_t unit = static_cast<size_t>(unit_i);
+    float* part = a.ws + static_cast<size_t>(slot0 + index) * per;
+    for (int idx = tid; idx < g * DV; idx += nthr) part[(idx / DV) * PD + (idx % DV)] = sm_v[idx];
     if (tid < g) {
-        part[tid * PD + D] = sm_m[tid];
-        part[tid * PD + D + 1] = sm_l[tid];
+        part[tid * PD + DV] = sm_m[tid];
+        part[tid * PD + DV + 1] = sm_l[tid];
     }
     __threadfence();
     __syncthreads();
     __shared__ unsigned s_is_last;
     if (tid == 0) {
         const unsigned prev = atomicAdd(a.counters + unit, 1u);
-        s_is_last = (prev == static_cast<unsigned>(a.splits - 1)) ? 1u : 0u;
+        s_is_last = (prev == static_cast<unsigned>(count - 1)) ? 1u : 0u;
     }
     __syncthreads();
     if (!s_is_last) return;
     __threadfence();
-    const float* base = a.ws + unit * a.splits * static_cast<size_t>(g * PD);
-    // per-head max over splits, then per-(head, split) factors 2^(m_s - M)
-    float* fac = sm_scratch;                 // [g][splits]
-    float* hm = sm_scratch + g * a.splits;   // [g] max, then [g] l
-    float* hl = hm + g;
-    if (tid < g) {
-        float M = NEG_INF;
-        for (int s = 0; s < a.splits; ++s) M = fmaxf(M, __ldcg(base + (size_t)s * g * PD + tid * PD + D));
-        float L = 0.f;
-        for (int s = 0; s < a.splits; ++s) {
-            const float ms = __ldcg(base + (size_t)s * g * PD + tid * PD + D);
-            const float f = exp2f(ms - M);
-            fac[tid * a.splits + s] = f;
-            L += f * __ldcg(base + (size_t)s * g * PD + tid * PD + D + 1);
-        }
-        hm[tid] = M;
-        hl[tid] = L;
+    const int n = count;
+    const float* base = a.ws + static_cast<size_t>(slot0) * per;
+    float* fm = sm_scratch;            // [n][g]: m, then the factors 2^(m - M)
+    float* fl = sm_scratch + n * g;    // [n][g]: l
+    __shared__ float hm[MAX_GROUP], hl[MAX_GROUP];
+    for (int idx = tid; idx < n * g; idx += nthr) {
+        const int sp = idx / g;
+        const int h = idx % g;
+        fm[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV);
+        fl[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 1);
     }
     __syncthreads();
-    for (int idx = tid; idx < g * D; idx += nthr) {
-        const int h = idx / D;
-        const int e = idx % D;
-        float acc = 0.f;
-        for (int s = 0; s < a.splits; ++s) acc += fac[h * a.splits + s] * __ldcg(base + (size_t)s * g * PD + h * PD + e);
-        a.out[(head0 + h) * D + e] = acc / hl[h];
+    const int warp = tid >> 5, lane = tid & 31, nwarps = nthr >> 5;
+    for (int h = warp; h < g; h += nwarps) {
+        float M = NEG_INF;
+        for (int sp = lane; sp < n; sp += 32) M = fmaxf(M, fm[sp * g + h]);
+        M = warp_max(M);
+        float L = 0.f;
+        for (int sp = lane; sp < n; sp += 32) {
+            const float f = exp2f(fm[sp * g + h] - M);
+            fm[sp * g + h] = f;
+            L += f * fl[sp * g + h];
+        }
+        L = warp_sum(L);
+        if (lane == 0) {
+            hm[h] = M;
+            hl[h] = L;
+        }
     }
-    if (a.lse != nullptr && tid < g) a.lse[head0 + tid] = (hm[tid] + log2f(hl[tid])) * LN2_F;
+    __syncthreads();
+    constexpr int MAXO = (MAX_GROUP * 128 + 127) / 128;   // values per thread at >= 128 threads
+    float acc[MAXO];
+#pragma unroll
+    for (int k = 0; k < MAXO; ++k) acc[k] = 0.f;
+    const int chunk = stage_bytes / (per * 4);
+    if (chunk >= 1) {
+        __shared__ __align__(8) uint64_t mbar;
+        if (tid == 0) {
+            mbar_init(&mbar, 1);
+            mbar_init_fence();
+        }
+        __syncthreads();
+        float* sp_buf = reinterpret_cast<float*>(stage);
+        unsigned phase = 0;
+        for (int s0 = 0; s0 < n; s0 += chunk) {
+            const int cnt = min(chunk, n - s0);
+            if (tid == 0) {
+                asm volatile("fence.proxy.async;" ::: "memory");
+                mbar_arrive_expect_tx(&mbar, static_cast<unsigned>(cnt * per * 4));
+                bulk_load(sp_buf, base + static_cast<size_t>(s0) * per, static_cast<unsigned>(cnt * per * 4), &mbar);
+            }
+            mbar_wait_bounded(&mbar, phase, a.wait_limit, a.err);
+            phase ^= 1u;
+#pragma unroll
+            for (int k = 0; k < MAXO; ++k) {
+                const int idx = tid + k * nthr;
+                if (idx < g * DV) {
+                    const int h = idx / DV;
+                    const int e = idx % DV;
+                    float v = acc[k];
+                    for (int c = 0; c < cnt; ++c) v += fm[(s0 + c) * g + h] * sp_buf[c * per + h * PD + e];
+                    acc[k] = v;
+                }
+            }
+            __syncthreads();   // the buffer is refilled by the next chunk
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < MAXO; ++k) {
+            const int idx = tid + k * nthr;
+            if (idx < g * DV) {
+                const int h = idx / DV;
+                const int e = idx % DV;
+                float v = 0.f;
+#pragma unroll 8
+                for (int sp = 0; sp < n; ++sp) v += fm[sp * g + h] * __ldcg(base + static_cast<size_t>(sp) * per + h * PD + e);
+                acc[k] = v;
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < MAXO; ++k) {
+        const int idx = tid + k * nthr;
+        if (idx < g * DV) sm_v[idx] = acc[k];
+    }
+    __syncthreads();
+    emit(sm_v, hl, hm);
     if (tid == 0) a.counters[unit] = 0u;
+}
+
+// Split-grid kernels: CTA (split, j, b) holds partial `split` of `a.splits` for its unit.
+__device__ inline void finish_split(const DecodeArgs& a, int D, int b, int j, int split, const float* sm_m,
+                                    const float* sm_l, float* sm_o, float* sm_scratch, uint8_t* stage,
+                                    int stage_bytes) {
+    const int unit = b * a.Hkv + j;
+    const EmitPlain emit{a, D, static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * a.g};
+    finish_unit(a, D, unit, split, a.splits, static_cast<long long>(unit) * a.splits, sm_m, sm_l, sm_o, sm_scratch,
+                stage, stage_bytes, emit);
 }
 
 }  // namespace kvs

@@ -24,8 +24,10 @@ struct DecodeArgs {
     int src0, src1;         // slots (SINGLE/MIX)
     const float* w;         // [Hkv] mix weights of this layer (device), MIX only
     int B, Hq, Hkv, T, g;
-    int splits;             // splits per (b, kv head)
-    int tiles_per_split;    // token tiles per split
+    int splits;             // splits per (b, kv head)            (split-grid kernels)
+    int tiles_per_split;    // token tiles per split               (split-grid kernels)
+    int units;              // B * Hkv                             (balanced-grid kernels)
+    int n_t;                // token tiles per unit                (balanced-grid kernels)
     float scale_log2;       // softmax scale * log2(e)
     float* ws;              // split partials [B*Hkv][splits][g][d+2]
     unsigned* counters;     // [B*Hkv] arrival counters, zero between launches
@@ -82,6 +84,6 @@ cudaError_t launch_pack_residual(const PackArgs& a, cudaStream_t st);
 
 int prefill_kv_tile(int d, bool mix);
 cudaError_t launch_prefill(int d, bool mix, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const PrefillArgs& a, cudaStream_t st);
+                           const CUtensorMap& to, const PrefillArgs& a, cudaStream_t st);
 
 }  // namespace kvs

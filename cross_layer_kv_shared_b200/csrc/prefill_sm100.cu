@@ -1,21 +1,26 @@
 // Causal prefill over a shared cache on the 5th-generation tensor cores (tcgen05 + TMEM).
 //
-// One CTA = 128 query rows of one head. Warp roles:
-//   warp 0       TMA producer: Q once, then K/V tiles into a 2-stage ring
-//   warp 1       TMEM owner and MMA issuer (one thread): S = Q K^T into one of two
-//                TMEM S buffers, O += P V into the TMEM O accumulator
-//   warps 4-7    softmax warpgroup, one thread per query row: S from TMEM,
-//                causal mask, online softmax in base 2 with a lazy max (O is
-//                rescaled in TMEM only when the row max grows by more than 2^8),
-//                P as bf16 into shared memory (128-B swizzled, the MMA's A layout),
-//                epilogue O / l -> bf16 and the log-sum-exp
-//   warps 8-11   (two-source layers only) mixers: K~ = w K1 + (1-w) K2 and the
-//                same for V, in fp32, rounded once to bf16, written in place over
-//                the first source's tile, so the MMA reads the mixed operand and
-//                the mixed K/V never reach HBM ("DepthGraft: Structural
-//                Regularization through Hierarchical Cross-Layer KV
-//                Reconstruction", Abstract: deep-layer KV rebuilt from a
-//                shallow/middle source pair; the convex mix is this library's reading).
+// One CTA = two 128-row query tiles of one head (rows q0 .. q0+255), sharing every
+// K/V tile it streams. TMEM holds both tiles' scores S0, S1 and outputs O0, O1.
+// Warp roles:
+//   warp 8        TMA producer: Q0, Q1 once, then K/V tiles into a 2-stage ring
+//   warp 9        TMEM owner and MMA issuer (one thread), in the order
+//                 S0_j, S1_j, PV0_j, S0_{j+1}, PV1_j, S1_{j+1}, ... so that the
+//                 tensor core computes one tile's product while the other tile's
+//                 softmax runs:  S = Q K^T  (A, B from shared memory)
+//                                O += P V  (A = P straight from TMEM, B = V from shared)
+//   warps 0-3     softmax of tile 0, one thread per query row: scores from TMEM,
+//   warps 4-7     softmax of tile 1   causal mask, online softmax in base 2 with a
+//                 lazy max (O rescaled in TMEM only when a row max grows by more
+//                 than 2^8), P as bf16 written back over the row's S columns;
+//                 epilogue O / l -> bf16 through shared memory and a TMA store
+//   warps 10-13   (two-source layers only) mixers: K~ = w K1 + (1-w) K2 and the
+//                 same for V, in fp32, rounded once to bf16, written in place over
+//                 the first source's tile, so the MMA reads the mixed operand and
+//                 the mixed K/V never reach HBM ("DepthGraft: Structural
+//                 Regularization through Hierarchical Cross-Layer KV
+//                 Reconstruction", Abstract: deep-layer KV rebuilt from a
+//                 shallow/middle source pair; the convex mix is this library's reading).
 // Every mbarrier wait is bounded; a wait that runs out records KVS_ETIMEOUT,
 // makes the other waits of the CTA give up, and the CTA still frees its TMEM.
 #include "tc_sm100.cuh"
@@ -23,22 +28,24 @@
 namespace kvs {
 namespace {
 
-constexpr int BM = 128;
-constexpr int NS = 2;
+constexpr int BM = 128;   // rows per query tile
+constexpr int NQ = 2;     // query tiles per CTA
+constexpr int NS = 2;     // K/V stages
 
 template <int D, bool MIX>
 struct PfCfg {
     static constexpr int BN = MIX ? 64 : 128;
     static constexpr int HALVES = D / 64;
     static constexpr int NSRC = MIX ? 2 : 1;
-    static constexpr int Q_BYTES = BM * D * 2;
+    static constexpr int Q_BYTES = BM * D * 2;     // one query tile
     static constexpr int TILE = BN * D * 2;        // one K or V tile
     static constexpr int HALF_T = BN * 128;        // one 64-column half of it
     static constexpr int STAGE = 2 * NSRC * TILE;
-    static constexpr int P_BYTES = BM * BN * 2;
-    static constexpr int SMEM = Q_BYTES + NS * STAGE + P_BYTES + 1024;
-    static constexpr uint32_t TMEM_COLS = (2 * BN + D) <= 256 ? 256u : 512u;
-    static constexpr int THREADS = MIX ? 384 : 256;
+    static constexpr int SMEM = NQ * Q_BYTES + NS * STAGE + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;     // S0 | S1 | O0 | O1
+    static constexpr int THREADS = MIX ? 448 : 320;
+    static constexpr int W_TMA = 8, W_MMA = 9, W_MIX = 10;
+    static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
 };
 
 struct Sync {
@@ -46,10 +53,8 @@ struct Sync {
     uint64_t kv_full[NS];
     uint64_t kv_ready[NS];
     uint64_t kv_empty[NS];
-    uint64_t s_full[2];
-    uint64_t s_free[2];
-    uint64_t p_full;
-    uint64_t p_free;
+    uint64_t s_full[NQ];
+    uint64_t p_full[NQ];
     uint64_t o_full;
     uint32_t tmem_base;
     volatile int abort;
@@ -69,30 +74,37 @@ __device__ __forceinline__ void wait_cta(Sync& sy, uint64_t* bar, unsigned parit
     }
 }
 
+// number of K/V tiles a query tile whose first row is qbase needs
+__device__ __forceinline__ int kv_tiles(int qbase, int S, int BN) {
+    if (qbase >= S) return 0;
+    return (min(qbase + BM, S) - 1) / BN + 1;
+}
+
 template <int D, bool MIX>
 __global__ void __launch_bounds__(PfCfg<D, MIX>::THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               const PrefillArgs a) {
     using C = PfCfg<D, MIX>;
     constexpr int BN = C::BN;
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = smem;
-    uint8_t* sKV = smem + C::Q_BYTES;
-    uint8_t* sP = sKV + NS * C::STAGE;
+    uint8_t* sQ = smem;                                  // [NQ][HALVES][BM][64]
+    uint8_t* sKV = smem + NQ * C::Q_BYTES;               // [NS][K1 | V1 (| K2 | V2)]
     __shared__ __align__(8) Sync sy;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_mt = (a.S + BM - 1) / BM;
-    const int mt = n_mt - 1 - static_cast<int>(blockIdx.z);     // heaviest query tiles first
+    const int n_ct = (a.S + NQ * BM - 1) / (NQ * BM);
+    const int ct = n_ct - 1 - static_cast<int>(blockIdx.z);    // heaviest query tiles first
     const int h = blockIdx.x;
     const int b = blockIdx.y;
     const int jkv = h / a.g;
-    const int q0 = mt * BM;
-    const int q_last = min(q0 + BM, a.S) - 1;
-    const int n_kv = q_last / BN + 1;
-    const int diag0 = q0 / BN;
+    const int q0 = ct * NQ * BM;
+    int nq[NQ];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) nq[i] = kv_tiles(q0 + i * BM, a.S, BN);
+    const int n_kv = nq[NQ - 1] > nq[0] ? nq[NQ - 1] : nq[0];
 
     if (threadIdx.x == 0) {
         mbar_init(&sy.q_full, 1);
@@ -101,17 +113,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             mbar_init(&sy.kv_ready[s], 128);
             mbar_init(&sy.kv_empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NQ; ++i) {
             mbar_init(&sy.s_full[i], 1);
-            mbar_init(&sy.s_free[i], 128);
+            mbar_init(&sy.p_full[i], 128);
         }
-        mbar_init(&sy.p_full, 128);
-        mbar_init(&sy.p_free, 1);
         mbar_init(&sy.o_full, 1);
         sy.abort = 0;
         mbar_init_fence();
     }
-    if (warp == 1) {
+    if (warp == C::W_MMA) {
         tc::alloc(&sy.tmem_base, C::TMEM_COLS);
         tc::relinquish();
     }
@@ -119,15 +129,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = sy.tmem_base;
-    const uint32_t tmem_o = tmem + 2 * BN;
+    // TMEM columns: S_i at i * BN, O_i at 2 * BN + i * D
+    auto tS = [&](int i) { return tmem + static_cast<uint32_t>(i * BN); };
+    auto tO = [&](int i) { return tmem + static_cast<uint32_t>(2 * BN + i * D); };
 
-    if (warp == 0) {
+    if (warp == C::W_TMA) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(&sy.q_full, C::Q_BYTES);
+            mbar_arrive_expect_tx(&sy.q_full, NQ * C::Q_BYTES);
 #pragma unroll
-            for (int hh = 0; hh < C::HALVES; ++hh)
-                tma_load_3d(sQ + hh * BM * 128, &tmQ, hh * 64, q0, b * a.Hq + h, &sy.q_full);
+            for (int i = 0; i < NQ; ++i)
+#pragma unroll
+                for (int hh = 0; hh < C::HALVES; ++hh)
+                    tma_load_3d(sQ + i * C::Q_BYTES + hh * BM * 128, &tmQ, hh * 64, q0 + i * BM, b * a.Hq + h,
+                                &sy.q_full);
             const int BH = a.B * a.Hkv;
             const int r0 = a.src0 * BH + b * a.Hkv + jkv;
             const int r1 = a.src1 * BH + b * a.Hkv + jkv;
@@ -157,83 +172,87 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == C::W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
             constexpr uint32_t idO = tc::idesc_bf16(BM, D, false, true);
             const uint32_t q_addr = smem_u32(sQ);
-            const uint32_t p_addr = smem_u32(sP);
-            auto issue_pv = [&](int jj) {
-                wait_cta(sy, &sy.p_full, jj & 1, a.wait_limit, a.err);
-                tc::fence_after();
-                const int s = jj % NS;
-                const uint32_t v_addr = smem_u32(sKV + s * C::STAGE + C::TILE);
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t ad = tc::smem_desc(p_addr + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024,
-                                                      tc::LAYOUT_SW128);
-                    const uint64_t bd = tc::smem_desc(v_addr + kk * 16 * 128, C::HALF_T, 1024, tc::LAYOUT_SW128);
-                    tc::mma_ss(tmem_o, ad, bd, idO, (jj > 0 || kk > 0) ? 1u : 0u);
-                }
-                tc::commit(&sy.p_free);
-                tc::commit(&sy.kv_empty[s]);
-            };
-            wait_cta(sy, &sy.q_full, 0, a.wait_limit, a.err);
-            for (int j = 0; j < n_kv; ++j) {
-                const int s = j % NS;
-                wait_cta(sy, MIX ? &sy.kv_ready[s] : &sy.kv_full[s], (j / NS) & 1, a.wait_limit, a.err);
-                const int sb = j & 1;
-                if (j >= 2) wait_cta(sy, &sy.s_free[sb], ((j >> 1) - 1) & 1, a.wait_limit, a.err);
-                tc::fence_after();
-                const uint32_t k_addr = smem_u32(sKV + s * C::STAGE);
+            auto issue_s = [&](int i, int j) {          // S_i = Q_i K_j^T
+                const uint32_t k_addr = smem_u32(sKV + (j % NS) * C::STAGE);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk & 3) * 32;      // 16 bf16 along K inside the 128-B row
-                    const uint64_t ad = tc::smem_desc(q_addr + (kk >> 2) * (BM * 128) + off, 16, 1024, tc::LAYOUT_SW128);
+                    const uint32_t off = (kk & 3) * 32;   // 16 bf16 along K inside the 128-B row
+                    const uint64_t ad = tc::smem_desc(q_addr + i * C::Q_BYTES + (kk >> 2) * (BM * 128) + off, 16, 1024,
+                                                      tc::LAYOUT_SW128);
                     const uint64_t bd = tc::smem_desc(k_addr + (kk >> 2) * C::HALF_T + off, 16, 1024, tc::LAYOUT_SW128);
-                    tc::mma_ss(tmem + sb * BN, ad, bd, idS, kk > 0 ? 1u : 0u);
+                    tc::mma_ss(tS(i), ad, bd, idS, kk > 0 ? 1u : 0u);
                 }
-                tc::commit(&sy.s_full[sb]);
-                if (j >= 1) issue_pv(j - 1);
-                if (sy.abort) break;
+                tc::commit(&sy.s_full[i]);
+            };
+            auto issue_pv = [&](int i, int j) {         // O_i += P_i V_j, P_i read from TMEM
+                wait_cta(sy, &sy.p_full[i], j & 1, a.wait_limit, a.err);
+                tc::fence_after();
+                const uint32_t v_addr = smem_u32(sKV + (j % NS) * C::STAGE + C::TILE);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t bd = tc::smem_desc(v_addr + kk * 16 * 128, C::HALF_T, 1024, tc::LAYOUT_SW128);
+                    tc::mma_ts(tO(i), tS(i) + kk * 8, bd, idO, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+            };
+            auto wait_kv = [&](int j) {
+                wait_cta(sy, MIX ? &sy.kv_ready[j % NS] : &sy.kv_full[j % NS], (j / NS) & 1, a.wait_limit, a.err);
+                tc::fence_after();
+            };
+            wait_cta(sy, &sy.q_full, 0, a.wait_limit, a.err);
+            wait_kv(0);
+            if (nq[0] > 0) issue_s(0, 0);
+            if (nq[1] > 0) issue_s(1, 0);
+            for (int j = 0; j < n_kv && !sy.abort; ++j) {
+                const bool next = j + 1 < n_kv;
+                if (j < nq[0]) issue_pv(0, j);
+                if (next) wait_kv(j + 1);
+                if (next && j + 1 < nq[0]) issue_s(0, j + 1);
+                if (j < nq[1]) issue_pv(1, j);
+                tc::commit(&sy.kv_empty[j % NS]);
+                if (next && j + 1 < nq[1]) issue_s(1, j + 1);
             }
-            if (!sy.abort) issue_pv(n_kv - 1);
             tc::commit(&sy.o_full);
         }
-    } else if (warp >= 4 && warp < 8) {
-        // ------------------------------------------------------------ softmax warpgroup
-        const int row = (warp - 4) * 32 + lane;
-        const int qpos = q0 + row;
-        const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    } else if (warp < 4 * NQ) {
+        // ------------------------------------------------------------ softmax, one warpgroup per query tile
+        const int qi = warp >> 2;
+        const int wq = warp & 3;                         // lane quadrant of TMEM this warp may access
+        const int row = wq * 32 + lane;
+        const int qpos = q0 + qi * BM + row;
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t sS = tS(qi) + lane_base;
+        const uint32_t sO = tO(qi) + lane_base;
+        const int n_my = nq[qi];
+        const int diag0 = (q0 + qi * BM) / BN;
         float m_used = NEG_INF;
         float l = 0.f;
-        for (int j = 0; j < n_kv; ++j) {
-            const int sb = j & 1;
-            wait_cta(sy, &sy.s_full[sb], (j >> 1) & 1, a.wait_limit, a.err);
+        for (int j = 0; j < n_my; ++j) {
+            wait_cta(sy, &sy.s_full[qi], j & 1, a.wait_limit, a.err);
             tc::fence_after();
-            float s[BN];
+            const int k0 = j * BN;
+            const bool masked = j >= diag0;
+            // pass 1: row max of the raw (unscaled) scores, masked on diagonal tiles
+            float mraw = NEG_INF;
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
-                tc::ld32(tmem + lane_base + sb * BN + c * 32, r);
+                tc::ld32(sS + c * 32, r);
                 tc::wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 32; ++i) {
+                    const float v = (masked && k0 + c * 32 + i > qpos) ? NEG_INF : __uint_as_float(r[i]);
+                    mraw = fmaxf(mraw, v);
+                }
             }
-            tc::fence_before();
-            mbar_arrive(&sy.s_free[sb]);
-            const int k0 = j * BN;
-            float mt = NEG_INF;
-#pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                float v = s[c] * a.scale_log2;
-                if (j >= diag0 && k0 + c > qpos) v = NEG_INF;
-                s[c] = v;
-                mt = fmaxf(mt, v);
-            }
-            // lazy max: rescale O only when this row's max grew by more than 2^8; the
-            // TMEM load/store is warp-collective, so the warp rescales if any row needs it
+            const float mt = mraw * a.scale_log2;
+            // lazy max: rescale O only when the row max grew by more than 2^8; the TMEM
+            // load/store is warp-collective, so the warp rescales if any row needs it
             float corr = 1.f;
             if (m_used == NEG_INF) {
                 m_used = mt;
@@ -241,48 +260,55 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 corr = tc::ex2(m_used - mt);
                 m_used = mt;
             }
-            const bool rescale = __any_sync(0xffffffffu, corr != 1.f);
-            if (j >= 1) wait_cta(sy, &sy.p_free, (j - 1) & 1, a.wait_limit, a.err);
-            if (rescale) {
+            if (__any_sync(0xffffffffu, corr != 1.f)) {
                 l *= corr;
-                tc::fence_after();
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tc::ld32(tmem_o + lane_base + c * 32, r);
+                    uint32_t o32[32];
+                    tc::ld32(sO + c * 32, o32);
                     tc::wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
-                    tc::st32(tmem_o + lane_base + c * 32, r);
+                    for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * corr);
+                    tc::st32(sO + c * 32, o32);
                 }
-                tc::wait_st();
             }
+            // pass 2: P = 2^(s * scale - m) as bf16, packed two per column over the row's first BN/2 S columns
+            const float nm = -m_used;
 #pragma unroll
-            for (int c8 = 0; c8 < BN / 8; ++c8) {
-                uint32_t pk[4];
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tc::ld32(sS + c * 32, r);
+                tc::wait_ld();
+                uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    pk[i] = pack_bf16(tc::ex2(s[c8 * 8 + 2 * i] - m_used), tc::ex2(s[c8 * 8 + 2 * i + 1] - m_used));
-                    l += bf16_lo(pk[i]) + bf16_hi(pk[i]);
+                for (int i = 0; i < 16; ++i) {
+                    const int t0 = k0 + c * 32 + 2 * i;
+                    float p0 = tc::ex2(fmaf(__uint_as_float(r[2 * i]), a.scale_log2, nm));
+                    float p1 = tc::ex2(fmaf(__uint_as_float(r[2 * i + 1]), a.scale_log2, nm));
+                    if (masked) {
+                        if (t0 > qpos) p0 = 0.f;
+                        if (t0 + 1 > qpos) p1 = 0.f;
+                    }
+                    l += p0 + p1;
+                    pk[i] = pack_bf16(p0, p1);
                 }
-                uint8_t* dst = sP + (c8 >> 3) * (BM * 128) + swz128(row, c8 & 7);
-                *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                tc::st16(sS + c * 16, pk);
             }
-            fence_proxy_async();
+            tc::wait_st();
             tc::fence_before();
-            mbar_arrive(&sy.p_full);
+            mbar_arrive(&sy.p_full[qi]);
         }
-        // ------------------------------------------------------------ epilogue
-        wait_cta(sy, &sy.o_full, 0, a.wait_limit, a.err);
-        tc::fence_after();
-        const float inv = 1.f / l;
-        uint16_t* orow = reinterpret_cast<uint16_t*>(a.out) + (static_cast<size_t>(b * a.Hq + h) * a.S + qpos) * D;
+        // ------------------------------------------------------------ epilogue through shared memory
+        if (n_my > 0) {
+            wait_cta(sy, &sy.o_full, 0, a.wait_limit, a.err);
+            tc::fence_after();
+            const float inv = 1.f / l;
+            uint8_t* so = sQ + qi * C::Q_BYTES;          // this tile's Q buffer is free now
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tc::ld32(tmem_o + lane_base + c * 32, r);
-            tc::wait_ld();
-            if (qpos < a.S) {
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tc::ld32(sO + c * 32, r);
+                tc::wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; i += 8) {
                     uint4 v;
@@ -290,21 +316,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     v.y = pack_bf16(__uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
                     v.z = pack_bf16(__uint_as_float(r[i + 4]) * inv, __uint_as_float(r[i + 5]) * inv);
                     v.w = pack_bf16(__uint_as_float(r[i + 6]) * inv, __uint_as_float(r[i + 7]) * inv);
-                    *reinterpret_cast<uint4*>(orow + c * 32 + i) = v;
+                    const int chunk = (c * 32 + i) >> 3;          // 16-B chunk of the row
+                    *reinterpret_cast<uint4*>(so + (chunk >> 3) * (BM * 128) + swz128(row, chunk & 7)) = v;
                 }
             }
+            if (a.lse != nullptr && qpos < a.S)
+                a.lse[static_cast<size_t>(b * a.Hq + h) * a.S + qpos] = (m_used + log2f(l)) * LN2_F;
+            fence_proxy_async();
+            named_sync(1 + qi, 128);
+            if (row == 0) {
+#pragma unroll
+                for (int hh = 0; hh < C::HALVES; ++hh)
+                    tma_store_3d(&tmO, so + hh * BM * 128, hh * 64, q0 + qi * BM, b * a.Hq + h);
+                bulk_commit();
+                bulk_wait_read0();
+            }
         }
-        if (a.lse != nullptr && qpos < a.S)
-            a.lse[static_cast<size_t>(b * a.Hq + h) * a.S + qpos] = (m_used + log2f(l)) * LN2_F;
-    } else if (MIX && warp >= 8) {
+    } else if (MIX && warp >= C::W_MIX) {
         // ------------------------------------------------------------ mixers (two-source layers)
-        const int t = threadIdx.x - 256;
+        const int t = threadIdx.x - 32 * C::W_MIX;
         const float w = a.w[jkv];
         const float w1 = 1.f - w;
         for (int j = 0; j < n_kv; ++j) {
             const int s = j % NS;
             wait_cta(sy, &sy.kv_full[s], (j / NS) & 1, a.wait_limit, a.err);
-            uint4* dst = reinterpret_cast<uint4*>(sKV + s * C::STAGE);               // K1 | V1
+            uint4* dst = reinterpret_cast<uint4*>(sKV + s * C::STAGE);                          // K1 | V1
             const uint4* src = reinterpret_cast<const uint4*>(sKV + s * C::STAGE + 2 * C::TILE);   // K2 | V2
             for (int idx = t; idx < 2 * C::TILE / 16; idx += 128) {
                 const uint4 x = dst[idx];
@@ -323,15 +359,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     tc::fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == C::W_MMA) {
         tc::fence_after();
         tc::dealloc(tmem, C::TMEM_COLS);
     }
 }
 
 template <int D, bool MIX>
-cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillArgs& a,
-                       cudaStream_t st) {
+cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                       const PrefillArgs& a, cudaStream_t st) {
     using C = PfCfg<D, MIX>;
     auto kern = prefill_kernel<D, MIX>;
     static bool attr_done = false;
@@ -340,8 +376,8 @@ cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    dim3 grid(a.Hq, a.B, (a.S + BM - 1) / BM);
-    kern<<<grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, a);
+    dim3 grid(a.Hq, a.B, (a.S + NQ * BM - 1) / (NQ * BM));
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, to, a);
     return cudaGetLastError();
 }
 
@@ -353,9 +389,9 @@ int prefill_kv_tile(int d, bool mix) {
 }
 
 cudaError_t launch_prefill(int d, bool mix, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const PrefillArgs& a, cudaStream_t st) {
-    if (d == 64) return mix ? launch_one<64, true>(tq, tk, tv, a, st) : launch_one<64, false>(tq, tk, tv, a, st);
-    return mix ? launch_one<128, true>(tq, tk, tv, a, st) : launch_one<128, false>(tq, tk, tv, a, st);
+                           const CUtensorMap& to, const PrefillArgs& a, cudaStream_t st) {
+    if (d == 64) return mix ? launch_one<64, true>(tq, tk, tv, to, a, st) : launch_one<64, false>(tq, tk, tv, to, a, st);
+    return mix ? launch_one<128, true>(tq, tk, tv, to, a, st) : launch_one<128, false>(tq, tk, tv, to, a, st);
 }
 
 }  // namespace kvs

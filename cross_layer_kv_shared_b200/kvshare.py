@@ -64,6 +64,7 @@ def _load():
         "kvshare_sync_status": ([P, V], I),
         "kvshare_set_splits": ([P, I], I),
         "kvshare_debug_stall_next": ([P, I], I),
+        "kvshare_debug_set_grid": ([P, I], I),
         "kvshare_launch_count": ([P], ctypes.c_uint64),
         "kvshare_status_string": ([I], ctypes.c_char_p),
         "kvshare_decode_layer_noalloc": ([P, P, P, P, P, P, I, I, I, I, I, I, I, I, V], I),
@@ -207,6 +208,10 @@ def kvshare_sync_status(h, stream=None) -> int:
 
 def kvshare_set_splits(h, splits: int) -> int:
     return _check(_lib.kvshare_set_splits(h, int(splits)), "kvshare_set_splits")
+
+
+def kvshare_debug_set_grid(h, ctas: int) -> int:
+    return _check(_lib.kvshare_debug_set_grid(h, int(ctas)), "kvshare_debug_set_grid")
 
 
 def kvshare_debug_stall_next(h, on: bool = True) -> int:

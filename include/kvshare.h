@@ -173,6 +173,13 @@ kvshare_status kvshare_sync_status(kvshare_t ctx, void* stream);
  * (batch, kv head), clamped to the number of token tiles and the workspace. */
 kvshare_status kvshare_set_splits(kvshare_t ctx, int splits);
 
+/* Test hook: force the bf16 decode grid to `ctas` CTAs (0 = automatic). The
+ * units' token tiles are cut into that many equal ranges, so a CTA may cover
+ * the end of one (batch, kv head) unit and the start of the next; the units'
+ * partial results merge exactly as with the automatic grid. Values are
+ * clamped to [batch * Hkv, total tiles]. */
+kvshare_status kvshare_debug_set_grid(kvshare_t ctx, int ctas);
+
 /* Test hook for the bounded waits: when `on` is non-zero, the next decode
  * launch makes one warp wait on a barrier nothing arrives on, with a limit of
  * about 10 ms; the wait gives up, records KVS_ETIMEOUT and the kernel still

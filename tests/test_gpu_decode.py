@@ -87,6 +87,17 @@ def test_split_count_does_not_change_the_result(K, cfg):
         assert np.max(np.abs(lse - ref_lse)) <= lse_tol
 
 
+@pytest.mark.parametrize("cfg", [CLA_SMALL, DG_SMALL], ids=lambda c: c.name)
+@pytest.mark.parametrize("grid", [7, 13, 29, 100])
+def test_grids_whose_ranges_straddle_units(K, cfg, grid):
+    """CTA ranges that end inside one (batch, kv head) unit and start the next."""
+    inp = cfg.make_all()
+    out, lse, _ = decode_gpu(K, cfg, inp, grid=grid)
+    want, want_lse = oracle_decode(cfg, inp)
+    assert_close(out, want, TOL_BF16, "out")
+    assert_close(lse, want_lse, TOL_BF16, "lse")
+
+
 def test_cla_layers_sharing_a_slot_match_bitwise(K):
     cfg = CLA_SMALL
     inp = cfg.make_all()
@@ -116,7 +127,9 @@ def test_mix_weight_endpoints_match_single_source(K):
     out, _, _ = decode_gpu(K, base, inp, splits=1)
     single = base.replace(layer_map=base.layer_map[:4] + ((SINGLE, 0, 0), (SINGLE, 3, 0)))
     out_s, _, _ = decode_gpu(K, single, inp, splits=1)
-    assert np.max(np.abs(out[4:] - out_s[4:])) < 1e-5
+    # same values up to the bf16 rounding of the weights p, which the two kernels
+    # (different token tiles) take against different running maxima
+    assert np.max(np.abs(out[4:] - out_s[4:])) <= 2.0 ** -8 * np.max(np.abs(out_s[4:]))
 
 
 def test_layer_range_writes_only_its_rows(K):
