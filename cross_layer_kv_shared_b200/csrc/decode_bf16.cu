@@ -5,8 +5,8 @@
 // (G = the CTAs resident at once, one per SM), so every SM streams the same
 // number of bytes whatever the batch. A range covers at most two units; each
 // unit's partial results merge in the last CTA to finish it.
-// Inside a CTA, four warps each own a private ring of NSW shared-memory stages
-// and stream every 4th tile of the range into it with TMA (128-byte swizzle),
+// Inside a CTA, NW warps each own a private ring of NSW shared-memory stages
+// and stream every NW-th tile of the range into it with TMA (128-byte swizzle),
 // re-issuing a stage as soon as it is consumed. Per tile and warp, with the
 // tokens as the MMA's M rows and the g query heads of the kv head as its N
 // columns (a group of up to 8 heads wastes nothing on padding):
@@ -24,9 +24,7 @@
 namespace kvs {
 namespace {
 
-constexpr int NW = 4;
-
-template <int D, bool MIX, int TT, int NSW>
+template <int D, bool MIX, int TT, int NSW, int NW>
 struct DecodeCfg {
     static constexpr int HALVES = D / 64;
     static constexpr int HALF_BYTES = TT * 128;              // [TT][64] bf16
@@ -40,15 +38,16 @@ struct DecodeCfg {
     // per-warp state of the first unit when a warp's tiles cross into the second one
     static constexpr int SAVE_FLOATS = NW * (16 * D + 32);
     static constexpr int SMEM = BODY + SAVE_FLOATS * 4 + 1024;  // + slack to align the ring to 1024 B
+    static constexpr int SMEM_ALIGNED = BODY + 1024;             // grids whose ranges never straddle
     static_assert(TT % 16 == 0, "token tile must hold whole m16 tiles");
     static_assert(HALF_BYTES % 1024 == 0, "swizzled halves must stay 1024-B aligned");
 };
 
-template <int D, bool MIX, int TT, int NSW, int NH, bool STRADDLE>
+template <int D, bool MIX, int TT, int NSW, int NW, int NH, bool STRADDLE>
 __global__ void __launch_bounds__(NW * 32, 1)
 decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const DecodeArgs a) {
-    using C = DecodeCfg<D, MIX, TT, NSW>;
+    using C = DecodeCfg<D, MIX, TT, NSW, NW>;
     constexpr int MT = TT / 16;      // m16 token tiles per tile
     constexpr int NB = NH / 8;       // n8 head blocks
     extern __shared__ uint8_t smem_dyn[];
@@ -325,7 +324,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         __syncwarp();
     }
 
-    // ---- merge the four warps per unit (reusing the ring; every copy issued has been consumed)
+    // ---- merge the NW warps per unit (reusing the ring; every copy issued has been consumed)
     __syncthreads();
     (void)t;
     float* comb_o = reinterpret_cast<float*>(smem);   // [NW][16][D]
@@ -388,48 +387,50 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     }
 }
 
-template <int D, bool MIX, int TT, int NSW, int NH, bool STRADDLE>
+template <int D, bool MIX, int TT, int NSW, int NW, int NH, bool STRADDLE>
 cudaError_t launch_nh(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a, cudaStream_t st) {
-    using C = DecodeCfg<D, MIX, TT, NSW>;
-    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, NH, STRADDLE>;
+    using C = DecodeCfg<D, MIX, TT, NSW, NW>;
+    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, NW, NH, STRADDLE>;
+    constexpr int smem = STRADDLE ? C::SMEM : C::SMEM_ALIGNED;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    kern<<<a.splits, NW * 32, C::SMEM, st>>>(tmK, tmV, a);
+    kern<<<a.splits, NW * 32, smem, st>>>(tmK, tmV, a);
     return cudaGetLastError();
 }
 
-template <int D, bool MIX, int TT, int NSW>
+template <int D, bool MIX, int TT, int NSW, int NW>
 cudaError_t launch_one(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a, cudaStream_t st) {
     // with a whole number m of CTAs per unit, CTA u*m starts exactly at unit u's first
     // tile (ceil(u*m*W/G) = u*n_t), so no range crosses a unit boundary
     const bool aligned = a.splits % a.units == 0;
     if (aligned)
-        return a.g <= 8 ? launch_nh<D, MIX, TT, NSW, 8, false>(tmK, tmV, a, st)
-                        : launch_nh<D, MIX, TT, NSW, 16, false>(tmK, tmV, a, st);
-    return a.g <= 8 ? launch_nh<D, MIX, TT, NSW, 8, true>(tmK, tmV, a, st)
-                    : launch_nh<D, MIX, TT, NSW, 16, true>(tmK, tmV, a, st);
+        return a.g <= 8 ? launch_nh<D, MIX, TT, NSW, NW, 8, false>(tmK, tmV, a, st)
+                        : launch_nh<D, MIX, TT, NSW, NW, 16, false>(tmK, tmV, a, st);
+    return a.g <= 8 ? launch_nh<D, MIX, TT, NSW, NW, 8, true>(tmK, tmV, a, st)
+                    : launch_nh<D, MIX, TT, NSW, NW, 16, true>(tmK, tmV, a, st);
 }
 
-template <int D, bool MIX, int TT, int NSW>
+template <int D, bool MIX, int TT, int NSW, int NW>
 int occupancy() {
-    using C = DecodeCfg<D, MIX, TT, NSW>;
-    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, 8, true>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    using C = DecodeCfg<D, MIX, TT, NSW, NW>;
+    // the default grid is unit-aligned, so its CTAs carry no straddle save area
+    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, NW, 8, false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALIGNED);
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NW * 32, C::SMEM) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NW * 32, C::SMEM_ALIGNED) != cudaSuccess) return 1;
     return n > 0 ? n : 1;
 }
 
-template <int D, bool MIX, int TT, int NSW>
+template <int D, bool MIX, int TT, int NSW, int NW>
 TileShape shape_of() {
-    return {TT, NSW, DecodeCfg<D, MIX, TT, NSW>::SMEM};
+    return {TT, NSW, DecodeCfg<D, MIX, TT, NSW, NW>::SMEM};
 }
 
-// tile shapes: tokens per tile (TT) and stages per warp (NSW) for each variant
+// tile shapes: tokens per tile (TT), stages per warp (NSW) and warps per CTA (NW) for each variant
 #ifndef KVS_TT_64S
 #define KVS_TT_64S 64
 #endif
@@ -454,10 +455,22 @@ TileShape shape_of() {
 #ifndef KVS_NSW_128M
 #define KVS_NSW_128M 2
 #endif
-#define KVS_SHAPE_64_SINGLE KVS_TT_64S, KVS_NSW_64S
-#define KVS_SHAPE_64_MIX KVS_TT_64M, KVS_NSW_64M
-#define KVS_SHAPE_128_SINGLE KVS_TT_128S, KVS_NSW_128S
-#define KVS_SHAPE_128_MIX KVS_TT_128M, KVS_NSW_128M
+#ifndef KVS_NW_64S
+#define KVS_NW_64S 4
+#endif
+#ifndef KVS_NW_64M
+#define KVS_NW_64M 4
+#endif
+#ifndef KVS_NW_128S
+#define KVS_NW_128S 4
+#endif
+#ifndef KVS_NW_128M
+#define KVS_NW_128M 4
+#endif
+#define KVS_SHAPE_64_SINGLE KVS_TT_64S, KVS_NSW_64S, KVS_NW_64S
+#define KVS_SHAPE_64_MIX KVS_TT_64M, KVS_NSW_64M, KVS_NW_64M
+#define KVS_SHAPE_128_SINGLE KVS_TT_128S, KVS_NSW_128S, KVS_NW_128S
+#define KVS_SHAPE_128_MIX KVS_TT_128M, KVS_NSW_128M, KVS_NW_128M
 
 }  // namespace
 

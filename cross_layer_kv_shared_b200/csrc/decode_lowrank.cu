@@ -25,7 +25,6 @@
 namespace kvs {
 namespace {
 
-constexpr int NW = 4;
 constexpr int RM = 16;
 
 template <int RB>
@@ -42,7 +41,7 @@ struct CoefLayout {
     }
 };
 
-template <int D, int RB, int TT, int NSW>
+template <int D, int RB, int TT, int NSW, int NW>
 struct LrCfg {
     using L = CoefLayout<RB>;
     static constexpr int COEF_BYTES = TT * RB * 2;
@@ -93,12 +92,12 @@ __device__ __forceinline__ uint32_t i8pair_bf16(uint32_t w16, bool keep0, bool k
     return pack_bf16(static_cast<float>(x0), static_cast<float>(x1));
 }
 
-template <int D, int RB, int TT, int NSW, int NH>
+template <int D, int RB, int TT, int NSW, int NW, int NH>
 __global__ void __launch_bounds__(NW * 32)
 decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_constant__ CUtensorMap tmCV,
                       const __grid_constant__ CUtensorMap tmUK, const __grid_constant__ CUtensorMap tmUV,
                       const DecodeArgs a) {
-    using C = LrCfg<D, RB, TT, NSW>;
+    using C = LrCfg<D, RB, TT, NSW, NW>;
     using LY = typename C::L;
     constexpr int MT = TT / 16;
     constexpr int NB = NH / 8;
@@ -479,10 +478,10 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 smem + C::MERGE_STAGE_OFF, C::BODY0 > C::MERGE_STAGE_OFF ? C::BODY0 - C::MERGE_STAGE_OFF : 0, emit);
 }
 
-template <int D, int RB, int TT, int NSW, int NH>
+template <int D, int RB, int TT, int NSW, int NW, int NH>
 cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
-    using C = LrCfg<D, RB, TT, NSW>;
-    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NH>;
+    using C = LrCfg<D, RB, TT, NSW, NW>;
+    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, NH>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -494,40 +493,44 @@ cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t
     return cudaGetLastError();
 }
 
-template <int D, int RB, int TT, int NSW>
+template <int D, int RB, int TT, int NSW, int NW>
 cudaError_t launch_one(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
-    return a.g <= 8 ? launch_nh<D, RB, TT, NSW, 8>(a, maps, st) : launch_nh<D, RB, TT, NSW, 16>(a, maps, st);
+    return a.g <= 8 ? launch_nh<D, RB, TT, NSW, NW, 8>(a, maps, st) : launch_nh<D, RB, TT, NSW, NW, 16>(a, maps, st);
 }
 
-template <int D, int RB, int TT, int NSW>
+template <int D, int RB, int TT, int NSW, int NW>
 int occupancy_of() {
-    using C = LrCfg<D, RB, TT, NSW>;
-    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, 8>;
+    using C = LrCfg<D, RB, TT, NSW, NW>;
+    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, 8>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NW * 32, C::SMEM) != cudaSuccess) return 1;
     return n > 0 ? n : 1;
 }
 
-// token tile and stages per warp by basis rank (the full-rank basis only serves tests)
+// token tile, stages per warp and warps per CTA by basis rank (the full-rank basis only serves tests)
 #ifndef KVS_LR_TT
 #define KVS_LR_TT 64
 #endif
 #ifndef KVS_LR_NSW
 #define KVS_LR_NSW 2
 #endif
+#ifndef KVS_LR_NW
+#define KVS_LR_NW 4
+#endif
 template <int RB>
 struct LrShape {
     static constexpr int TT = RB == 128 ? 32 : KVS_LR_TT;
     static constexpr int NSW = RB == 128 ? 1 : KVS_LR_NSW;
+    static constexpr int NW = RB == 128 ? 4 : KVS_LR_NW;
 };
 
 template <int D, int RB>
-int occ() { return occupancy_of<D, RB, LrShape<RB>::TT, LrShape<RB>::NSW>(); }
+int occ() { return occupancy_of<D, RB, LrShape<RB>::TT, LrShape<RB>::NSW, LrShape<RB>::NW>(); }
 
 template <int D, int RB>
 cudaError_t run(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
-    return launch_one<D, RB, LrShape<RB>::TT, LrShape<RB>::NSW>(a, maps, st);
+    return launch_one<D, RB, LrShape<RB>::TT, LrShape<RB>::NSW, LrShape<RB>::NW>(a, maps, st);
 }
 
 }  // namespace

@@ -23,6 +23,8 @@
 //                 shallow/middle source pair; the convex mix is this library's reading).
 // Every mbarrier wait is bounded; a wait that runs out records KVS_ETIMEOUT,
 // makes the other waits of the CTA give up, and the CTA still frees its TMEM.
+#include <type_traits>
+
 #include "tc_sm100.cuh"
 
 namespace kvs {
@@ -72,6 +74,33 @@ __device__ __forceinline__ void wait_cta(Sync& sy, uint64_t* bar, unsigned parit
             return;
         }
     }
+}
+
+// 2^x on the FMA pipe, for a share of the softmax exponentials so that the MUFU unit
+// (16 results per clock per SM, the same rate as the tensor core's bf16 products need
+// at BN = D = 128) is not the bottleneck. Range reduction: x = j + f with j = rint(x)
+// taken by the 1.5 * 2^23 rounding shift and f in [-1/2, 1/2]; 2^f from a degree-3
+// polynomial whose coefficients are a relative-error minimax fit on that interval
+// (iteratively reweighted least squares; largest relative error 7.6e-5, well below the
+// bf16 rounding of P); 2^j added to the exponent field. x >= -125 keeps the result a
+// normal float; inputs below that return 2^-125 instead of a smaller value.
+// KVS_PF_EMU_PAIRS (pairs of every 16 that take this path) is 0 by default: on the
+// d = 128 causal prefill every share from 3/16 to 9/16 measured slower, the issue
+// slots and FMA/ALU pipes rather than MUFU bounding this kernel's softmax.
+#ifndef KVS_PF_EMU_PAIRS
+#define KVS_PF_EMU_PAIRS 0
+#endif
+constexpr int EMU_PAIRS = KVS_PF_EMU_PAIRS;
+constexpr float EXP2_C0 = 0.9999281764030457f;
+constexpr float EXP2_C1 = 0.6932609677314758f;
+constexpr float EXP2_C2 = 0.24260950088500977f;
+constexpr float EXP2_C3 = 0.05517100542783737f;
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    const float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, EXP2_C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // number of K/V tiles a query tile whose first row is qbase needs
@@ -232,25 +261,27 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int diag0 = (q0 + qi * BM) / BN;
         float m_used = NEG_INF;
         float l = 0.f;
-        for (int j = 0; j < n_my; ++j) {
-            wait_cta(sy, &sy.s_full[qi], j & 1, a.wait_limit, a.err);
-            tc::fence_after();
-            const int k0 = j * BN;
-            const bool masked = j >= diag0;
-            // pass 1: row max of the raw (unscaled) scores, masked on diagonal tiles
-            float mraw = NEG_INF;
+        // one K/V tile of this row; MASKED (diagonal tiles only) zeroes the columns past qpos
+        auto step = [&](auto mask_tag, int j) {
+            constexpr bool MASKED = decltype(mask_tag)::value;
+            const int lim = qpos - j * BN;               // column c is visible iff c <= lim
+            // pass 1: row max of the raw (unscaled) scores, 64 columns per TMEM round trip
+            float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tc::ld32(sS + c * 32, r);
+            for (int c = 0; c < BN / 64; ++c) {
+                uint32_t r0[32], r1[32];
+                tc::ld32(sS + c * 64, r0);
+                tc::ld32(sS + c * 64 + 32, r1);
                 tc::wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float v = (masked && k0 + c * 32 + i > qpos) ? NEG_INF : __uint_as_float(r[i]);
-                    mraw = fmaxf(mraw, v);
+                    float v0 = __uint_as_float(r0[i]), v1 = __uint_as_float(r1[i]);
+                    if (MASKED && c * 64 + i > lim) v0 = NEG_INF;
+                    if (MASKED && c * 64 + 32 + i > lim) v1 = NEG_INF;
+                    mx[i & 3] = fmaxf(mx[i & 3], fmaxf(v0, v1));
                 }
             }
-            const float mt = mraw * a.scale_log2;
+            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.scale_log2;
             // lazy max: rescale O only when the row max grew by more than 2^8; the TMEM
             // load/store is warp-collective, so the warp rescales if any row needs it
             float corr = 1.f;
@@ -272,28 +303,46 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     tc::st32(sO + c * 32, o32);
                 }
             }
-            // pass 2: P = 2^(s * scale - m) as bf16, packed two per column over the row's first BN/2 S columns
+            // pass 2: P = 2^(s * scale - m) as bf16, packed two per column over the row's first
+            // BN/2 S columns; EMU_PAIRS of every 16 pairs take the FMA-pipe exponential
             const float nm = -m_used;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            auto pexp = [&](uint32_t bits, int col, bool emu) {
+                const float x = fmaf(__uint_as_float(bits), a.scale_log2, nm);
+                float p = emu ? exp2_fma(x) : tc::ex2(x);
+                if (MASKED && col > lim) p = 0.f;
+                return p;
+            };
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tc::ld32(sS + c * 32, r);
+            for (int c = 0; c < BN / 64; ++c) {
+                uint32_t r0[32], r1[32];
+                tc::ld32(sS + c * 64, r0);
+                tc::ld32(sS + c * 64 + 32, r1);
                 tc::wait_ld();
-                uint32_t pk[16];
+                uint32_t pk0[16], pk1[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int t0 = k0 + c * 32 + 2 * i;
-                    float p0 = tc::ex2(fmaf(__uint_as_float(r[2 * i]), a.scale_log2, nm));
-                    float p1 = tc::ex2(fmaf(__uint_as_float(r[2 * i + 1]), a.scale_log2, nm));
-                    if (masked) {
-                        if (t0 > qpos) p0 = 0.f;
-                        if (t0 + 1 > qpos) p1 = 0.f;
-                    }
-                    l += p0 + p1;
-                    pk[i] = pack_bf16(p0, p1);
+                    const bool emu = i < EMU_PAIRS;
+                    const int col = c * 64 + 2 * i;
+                    const float p0 = pexp(r0[2 * i], col, emu), p1 = pexp(r0[2 * i + 1], col + 1, emu);
+                    const float p2 = pexp(r1[2 * i], col + 32, emu), p3 = pexp(r1[2 * i + 1], col + 33, emu);
+                    ls[i & 1] += p0 + p1;
+                    ls[2 + (i & 1)] += p2 + p3;
+                    pk0[i] = pack_bf16(p0, p1);
+                    pk1[i] = pack_bf16(p2, p3);
                 }
-                tc::st16(sS + c * 16, pk);
+                tc::st16(sS + c * 32, pk0);
+                tc::st16(sS + c * 32 + 16, pk1);
             }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        };
+        for (int j = 0; j < n_my; ++j) {
+            wait_cta(sy, &sy.s_full[qi], j & 1, a.wait_limit, a.err);
+            tc::fence_after();
+            if (j >= diag0)
+                step(std::true_type{}, j);
+            else
+                step(std::false_type{}, j);
             tc::wait_st();
             tc::fence_before();
             mbar_arrive(&sy.p_full[qi]);
