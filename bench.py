@@ -32,7 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from synth.configs import BY_NAME  # noqa: E402
+from synth.configs import BY_NAME, LOWRANK, MIX  # noqa: E402
 
 METRIC = "decode tok/s and KV GB/s (% of HBM peak); prefill TFLOP/s, 1×B200"
 
@@ -171,6 +171,33 @@ class DecodeRunner:
     def layer(self, l):
         self.K.kvshare_decode(self.h, self.cache, self.dev["q"], self.out, self.lse, l, l + 1, self.stream)
 
+    def all_layers(self):
+        self.K.kvshare_decode(self.h, self.cache, self.dev["q"], self.out, self.lse, 0, self.cfg.layers,
+                              self.stream)
+
+    def capture_step(self):
+        """One decode step (every layer once, in cold_order) captured as a CUDA graph."""
+        torch, K = self.torch, self.K
+        self.order = cold_order(self.cfg)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for l in self.order:      # one eager pass first: attributes and tensor maps are set up
+                K.kvshare_decode(self.h, self.cache, self.dev["q"], self.out, self.lse, l, l + 1, side)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        n0 = K.kvshare_launch_count(self.h)
+        with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
+            cap = torch.cuda.current_stream()
+            for l in self.order:
+                K.kvshare_decode(self.h, self.cache, self.dev["q"], self.out, self.lse, l, l + 1, cap)
+        self.graph_launches = K.kvshare_launch_count(self.h) - n0
+        torch.cuda.synchronize()
+
+    def step_graph(self):
+        self.graph.replay()
+
     def step_flushed(self, events=None):
         torch = self.torch
         for l in range(self.cfg.layers):
@@ -188,6 +215,24 @@ class DecodeRunner:
         self.K.kvshare_destroy(self.h)
 
 
+def cold_order(cfg):
+    """Order of the layers inside a timed step: by how many earlier layers read one of the
+    layer's sources (store slot, or basis pair for the low-rank form), then by index. For
+    adjacent sharing this issues every first reader of a source before any second reader,
+    so the source a layer reads was last read several hundred MB of other reads ago and
+    comes from HBM, not L2, as in a full model where each layer's weights stream through
+    L2 between two layers sharing a source. Each layer's attention depends only on its own
+    q and sources, so the order changes no result."""
+    seen = {}
+    rank = []
+    for kind, s0, s1 in cfg.layer_map:
+        keys = [("pair", s0)] if kind == LOWRANK else [("slot", s0)] + ([("slot", s1)] if kind == MIX else [])
+        rank.append(max(seen.get(k, 0) for k in keys))
+        for k in keys:
+            seen[k] = seen.get(k, 0) + 1
+    return sorted(range(len(cfg.layer_map)), key=lambda l: (rank[l], l))
+
+
 def gpu_arm(args, cfg_name, secondary=False):
     import torch
     import synth.gpu as sgpu
@@ -195,8 +240,25 @@ def gpu_arm(args, cfg_name, secondary=False):
 
     cfg = BY_NAME[cfg_name]
     r = DecodeRunner(cfg, K, torch, sgpu)
+
+    # one decode step = every layer once, back to back (consecutive launches overlap
+    # through programmatic dependent launch), replayed from a CUDA graph; L2 is flushed
+    # before the step outside its events, and the layer order keeps shared sources cold
+    r.capture_step()
+
+    def step(events=None):
+        r.flush()
+        if events is None:
+            r.step_graph()
+            return
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(r.stream)
+        r.step_graph()
+        e1.record(r.stream)
+        events.append((e0, e1))
+
     for _ in range(args.warmup):
-        r.step_flushed()
+        step()
     torch.cuda.synchronize()
     if dist_on():
         import torch.distributed as dist
@@ -207,35 +269,47 @@ def gpu_arm(args, cfg_name, secondary=False):
     with ClockSampler(torch.cuda.current_device()) as clk:
         t_wall = time.perf_counter()
         for _ in range(args.steps):
-            r.step_flushed(events)
+            step(events)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     if dist_on():
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    launches = K.kvshare_launch_count(r.h) - n0
+    launches = r.graph_launches * args.steps + (K.kvshare_launch_count(r.h) - n0)
     st = K.kvshare_sync_status(r.h)
     assert st == K.KVS_OK, K.kvshare_status_string(st)
-    per_layer = np.zeros(cfg.layers)
-    for l, e0, e1 in events:
-        per_layer[l] += e0.elapsed_time(e1)
-    per_layer /= args.steps                       # ms per layer launch
-    step_ms = float(per_layer.sum())
+    step_ms = sum(a.elapsed_time(b) for a, b in events) / len(events)
     step_ms = max_over_ranks(step_ms)
 
-    # no-flush, back-to-back step (one call for all layers): L2 may serve shared sources
-    torch.cuda.synchronize()
-    nf = []
-    for _ in range(max(3, args.steps // 2)):
+    # secondary: the step in model order, one call for all layers; a layer that shares a
+    # source with the layer before it may find that source in L2
+    io = []
+    for i in range(3 + max(3, args.steps // 2)):
         r.flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(r.stream)
-        K.kvshare_decode(r.h, r.cache, r.dev["q"], r.out, r.lse, 0, cfg.layers, r.stream)
+        r.all_layers()
         e1.record(r.stream)
-        nf.append((e0, e1))
+        if i >= 3:
+            io.append((e0, e1))
     torch.cuda.synchronize()
-    nf_ms = statistics.median([a.elapsed_time(b) for a, b in nf])
+    in_order_ms = statistics.median([a.elapsed_time(b) for a, b in io])
+
+    # secondary: every layer alone on a cold L2 (flushed before each layer, one launch
+    # between its own events), so no layer can find a shared source in L2
+    for _ in range(2):
+        r.step_flushed()
+    torch.cuda.synchronize()
+    cold = []
+    for _ in range(max(3, args.steps // 2)):
+        r.step_flushed(cold)
+    torch.cuda.synchronize()
+    per_layer = np.zeros(cfg.layers)
+    for l, e0, e1 in cold:
+        per_layer[l] += e0.elapsed_time(e1)
+    per_layer /= max(3, args.steps // 2)
+    cold_ms = float(per_layer.sum())
 
     # e2e through the host-buffer entry point: q H2D + decode + out/lse D2H
     q_host = r.dev["q"].cpu().pin_memory()
@@ -257,7 +331,7 @@ def gpu_arm(args, cfg_name, secondary=False):
     res = {
         "cfg": cfg, "step_ms": step_ms, "per_layer_ms": per_layer, "launches": launches,
         "kv_gbs": read_bytes / (step_ms * 1e-3) / 1e9, "tok_s": cfg.batch / (step_ms * 1e-3),
-        "no_flush_ms": nf_ms, "e2e_ms": e2e_ms, "wall_s": t_wall, "clocks": clk.summary(),
+        "cold_layer_ms": cold_ms, "in_order_ms": in_order_ms, "e2e_ms": e2e_ms, "wall_s": t_wall, "clocks": clk.summary(),
         "h2d": q_host.numel() * q_host.element_size(),
         "d2h": out_host.numel() * 4 + lse_host.numel() * 4,
         "read_bytes": read_bytes, "pack_ms": r.pack_ms,
@@ -346,7 +420,9 @@ def arm_config(cfg, world: int) -> dict:
             "q_heads": cfg.q_heads, "kv_heads": cfg.kv_heads, "head_dim": cfg.head_dim,
             "layer_map": "CLA2: layer l reads slot l//2" if cfg.name == "cla2_1p1b" else cfg.name,
             "parallelism": f"replicas x{world}",
-            "l2": "flushed before every layer outside the timed events: 2x L2 write, then 2x L2 read (clean lines)"}
+            "l2": ("flushed before every timed step outside its events (2x L2 write, then 2x L2 read, so the "
+                   "lines left are clean); one step reads several times the 126 MB L2. cold_layer_*: flushed "
+                   "before every layer, each layer timed alone")}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) arm
@@ -469,7 +545,8 @@ def main():
             sec[name] = {"tok_s": r2["tok_s"] * world, "kv_gbs": r2["kv_gbs"],
                          "hbm_frac": r2["kv_gbs"] / hbm_peak, "ms_per_step": r2["step_ms"],
                          "algorithmic_bytes_per_step": r2["read_bytes"],
-                         "no_flush_ms_per_step": r2["no_flush_ms"], "gpu_launches": r2["launches"],
+                         "cold_layer_ms_per_step": r2["cold_layer_ms"],
+                         "in_model_order_ms_per_step": r2["in_order_ms"], "gpu_launches": r2["launches"],
                          "e2e_tok_s": r2["cfg"].batch * world / (r2["e2e_ms"] * 1e-3)}
             if r2["pack_ms"] is not None:
                 sec[name]["pack_residual_ms"] = r2["pack_ms"]
@@ -481,7 +558,9 @@ def main():
             "tensor_frac_of_burst": pr["tflops"] / bf16_peak, "tensor_frac_of_sustained": pr["tflops"] / bf16_sust,
             "single_source_layer_tflops": pr["single_layer_tflops"], "mix_layer_tflops": pr["mix_layer_tflops"],
             "flops_per_step": prefill_flops(pr["cfg"]), "gpu_launches": pr["launches"], "clocks": pr["clocks"]}
-    avg_launch_ms = float(np.mean(main_res["per_layer_ms"]))
+    # average launch duration over the timed region: the step's time over its launches
+    # (gaps between launches included)
+    avg_launch_ms = main_res["step_ms"] / cfg.layers
     per_launch_bytes = main_res["read_bytes"] / cfg.layers
     achieved = per_launch_bytes / (avg_launch_ms * 1e-3) / 1e9
     kname = ("decode_lowrank_kernel<%d,%d>" % (cfg.head_dim, cfg.basis_rank) if cfg.lowrank else
@@ -503,7 +582,10 @@ def main():
         "config": arm_config(cfg, world),
         "kv_gbs": main_res["kv_gbs"],
         "hbm_frac": main_res["kv_gbs"] / hbm_peak,
-        "no_flush_ms_per_step": main_res["no_flush_ms"],
+        "layer_order": "cold order (first readers of each source, then second readers)",
+        "cold_layer_ms_per_step": main_res["cold_layer_ms"],
+        "cold_layer_tok_s": cfg.batch * world / (main_res["cold_layer_ms"] * 1e-3),
+        "in_model_order_ms_per_step": main_res["in_order_ms"],
         "gpu_launches": main_res["launches"],
         "clocks": main_res["clocks"],
         "e2e": {"value": cfg.batch * world / (main_res["e2e_ms"] * 1e-3), "unit": "tok/s",

@@ -211,6 +211,8 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
         a.stall = c->stall_next;
         a.stall_limit = c->stall_limit;
         c->stall_next = 0;
+        // consecutive decode layers overlap launch and prologue with the previous tail
+        a.pdl = 1;
         cudaError_t err;
         if (cf.dtype == KVS_F32) {
             if (e.kind == KVS_SRC_LOWRANK) return KVS_EUNSUPPORTED;

@@ -70,10 +70,16 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     const int BH = a.B * a.Hkv;
 
     if (threadIdx.x == 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
         for (int i = 0; i < NW * NSW + 1; ++i) mbar_init(&bars[i], 1);
         mbar_init_fence();
     }
     __syncthreads();
+    // under a dependent launch everything above overlapped the previous kernel's tail;
+    // global memory (inputs, workspace, counters) is touched only from here on
+    grid_dep_wait();
+    if (threadIdx.x == 0) grid_dep_launch();
 
     if (a.stall && threadIdx.x == 0) {
         // test hook: nothing ever arrives on the spare barrier; the bounded wait gives up
@@ -398,8 +404,7 @@ cudaError_t launch_nh(const CUtensorMap& tmK, const CUtensorMap& tmV, const Deco
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    kern<<<a.splits, NW * 32, smem, st>>>(tmK, tmV, a);
-    return cudaGetLastError();
+    return launch_kernel(kern, dim3(a.splits), dim3(NW * 32), smem, st, a.pdl != 0, tmK, tmV, a);
 }
 
 template <int D, bool MIX, int TT, int NSW, int NW>

@@ -19,7 +19,8 @@
 //     so a group of up to 8 heads wastes nothing on padding; P^T reaches the
 //     PV MMAs through an in-register transpose (movmatrix);
 //   - int8 codes convert exactly to bf16 operands, masked by the token's rank;
-//   - c^ and u^ accumulate in fp32 MMA accumulators; one projection per CTA.
+//   - c^ and u^ accumulate in fp32 MMA accumulators; split partials stay in this
+//     coefficient space and the CTA that merges a unit projects it once.
 #include "kvs_device.cuh"
 
 namespace kvs {
@@ -126,10 +127,20 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(a.q) +
                            (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g) * D;
     if (threadIdx.x == 0) {
+        prefetch_tmap(&tmCK);
+        prefetch_tmap(&tmCV);
+        prefetch_tmap(&tmUK);
+        prefetch_tmap(&tmUV);
         for (int i = 0; i < NW * NSW + 1; ++i) mbar_init(&bars[i], 1);
         mbar_init(&fac_bar[0], 1);
         mbar_init(&fac_bar[1], 1);
         mbar_init_fence();
+    }
+    // under a dependent launch everything above overlapped the previous kernel's tail;
+    // global memory (inputs, workspace, counters) is touched only from here on
+    grid_dep_wait();
+    if (threadIdx.x == 0) {
+        grid_dep_launch();
         // B_K[j], R_K[j] and the group's query rows, by bulk copy (all contiguous, 16-B aligned)
         mbar_arrive_expect_tx(&fac_bar[0], C::STAGE_FACTORS + g * D * 2);
         bulk_load(stagebuf, static_cast<const uint16_t*>(a.basis_k) + static_cast<size_t>(j) * RB * D, RB * D * 2,
@@ -489,8 +500,7 @@ cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t
         attr_done = true;
     }
     dim3 grid(a.splits, a.Hkv, a.B);
-    kern<<<grid, NW * 32, C::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], a);
-    return cudaGetLastError();
+    return launch_kernel(kern, grid, dim3(NW * 32), C::SMEM, st, a.pdl != 0, maps[0], maps[1], maps[2], maps[3], a);
 }
 
 template <int D, int RB, int TT, int NSW, int NW>
@@ -509,14 +519,17 @@ int occupancy_of() {
 }
 
 // token tile, stages per warp and warps per CTA by basis rank (the full-rank basis only serves tests)
+// (defaults: the fastest of a measured sweep on the 64K-token, Rb = 32 workload; the
+// kernel is issue-latency bound, so 16 warps with one 32-token stage each beat deeper
+// rings on fewer warps)
 #ifndef KVS_LR_TT
-#define KVS_LR_TT 64
+#define KVS_LR_TT 32
 #endif
 #ifndef KVS_LR_NSW
-#define KVS_LR_NSW 2
+#define KVS_LR_NSW 1
 #endif
 #ifndef KVS_LR_NW
-#define KVS_LR_NW 4
+#define KVS_LR_NW 16
 #endif
 template <int RB>
 struct LrShape {

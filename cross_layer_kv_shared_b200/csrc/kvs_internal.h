@@ -44,7 +44,28 @@ struct DecodeArgs {
     const void* r_k; const void* r_v;           // layer's [Hkv][Rm][d]
     const uint8_t* rank;                        // layer's [B][T]
     int Rb, Rm;
+    // launch with programmatic stream serialization: the kernel may be scheduled while
+    // the previous kernel on the stream drains, and waits (griddepcontrol.wait) before
+    // its first global memory access
+    int pdl;
 };
+
+// cudaLaunchKernelEx with the programmatic-stream-serialization attribute when `pdl`
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 bool pdl, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
 
 struct PackArgs {
     const float* score; const float* u_k; const float* u_v;

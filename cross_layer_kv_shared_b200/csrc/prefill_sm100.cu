@@ -2,19 +2,20 @@
 //
 // One CTA = two 128-row query tiles of one head (rows q0 .. q0+255), sharing every
 // K/V tile it streams. TMEM holds both tiles' scores S0, S1 and outputs O0, O1.
-// Warp roles:
-//   warp 8        TMA producer: Q0, Q1 once, then K/V tiles into a 2-stage ring
-//   warp 9        TMEM owner and MMA issuer (one thread), in the order
-//                 S0_j, S1_j, PV0_j, S0_{j+1}, PV1_j, S1_{j+1}, ... so that the
-//                 tensor core computes one tile's product while the other tile's
-//                 softmax runs:  S = Q K^T  (A, B from shared memory)
-//                                O += P V  (A = P straight from TMEM, B = V from shared)
-//   warps 0-3     softmax of tile 0, one thread per query row: scores from TMEM,
-//   warps 4-7     softmax of tile 1   causal mask, online softmax in base 2 with a
-//                 lazy max (O rescaled in TMEM only when a row max grows by more
-//                 than 2^8), P as bf16 written back over the row's S columns;
-//                 epilogue O / l -> bf16 through shared memory and a TMA store
-//   warps 10-13   (two-source layers only) mixers: K~ = w K1 + (1-w) K2 and the
+// Warp roles, by warpgroup (each moves its register budget with setmaxnreg first):
+//   warpgroups 0, 1  softmax of query tile 0 / 1, one thread per query row: the
+//                 whole S row from TMEM in one round trip, causal mask on diagonal
+//                 tiles only, online softmax in base 2 with a lazy max (O rescaled
+//                 in TMEM only when a row max grows by more than 2^8), P as bf16
+//                 written back over the row's S columns; epilogue O / l -> bf16
+//                 through shared memory and a TMA store
+//   last warpgroup  one warp TMA producer (Q0, Q1 once, then K/V tiles into a
+//                 2-stage ring), one warp TMEM owner and MMA issuer (one thread),
+//                 in the order S0_j, S1_j, PV0_j, S0_{j+1}, PV1_j, S1_{j+1}, ... so
+//                 that the tensor core computes one tile's product while the other
+//                 tile's softmax runs:  S = Q K^T  (A, B from shared memory)
+//                                       O += P V  (A = P straight from TMEM, B = V from shared)
+//   warpgroup 2   (two-source layers only) mixers: K~ = w K1 + (1-w) K2 and the
 //                 same for V, in fp32, rounded once to bf16, written in place over
 //                 the first source's tile, so the MMA reads the mixed operand and
 //                 the mixed K/V never reach HBM ("DepthGraft: Structural
@@ -45,8 +46,18 @@ struct PfCfg {
     static constexpr int STAGE = 2 * NSRC * TILE;
     static constexpr int SMEM = NQ * Q_BYTES + NS * STAGE + 1024;
     static constexpr uint32_t TMEM_COLS = 512;     // S0 | S1 | O0 | O1
-    static constexpr int THREADS = MIX ? 448 : 320;
-    static constexpr int W_TMA = 8, W_MMA = 9, W_MIX = 10;
+    // warpgroups: 0, 1 softmax; MIX: 2 mixers, 3 TMA + MMA (+2 idle); single: 2 TMA + MMA (+2 idle)
+    static constexpr int THREADS = MIX ? 512 : 384;
+    static constexpr int W_MIX = 8;
+    static constexpr int W_TMA = MIX ? 12 : 8, W_MMA = W_TMA + 1;
+    // per-thread registers after the split (setmaxnreg): the softmax threads hold a whole
+    // S row; the sum over the block must not exceed what the block was launched with
+    static constexpr int LAUNCH_REGS = MIX ? 128 : 168;
+    static constexpr int REG_SOFTMAX = MIX ? 192 : 224;
+    static constexpr int REG_MIXER = 64;
+    static constexpr int REG_CTRL = 56;
+    static constexpr int REG_SUM = 2 * 128 * REG_SOFTMAX + (MIX ? 128 * REG_MIXER : 0) + 128 * REG_CTRL;
+    static_assert(REG_SUM <= THREADS * LAUNCH_REGS, "register split exceeds the launch allocation");
     static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
 };
 
@@ -136,6 +147,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int n_kv = nq[NQ - 1] > nq[0] ? nq[NQ - 1] : nq[0];
 
     if (threadIdx.x == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmO);
         mbar_init(&sy.q_full, 1);
         for (int s = 0; s < NS; ++s) {
             mbar_init(&sy.kv_full[s], 1);
@@ -162,93 +177,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     auto tS = [&](int i) { return tmem + static_cast<uint32_t>(i * BN); };
     auto tO = [&](int i) { return tmem + static_cast<uint32_t>(2 * BN + i * D); };
 
-    if (warp == C::W_TMA) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&sy.q_full, NQ * C::Q_BYTES);
-#pragma unroll
-            for (int i = 0; i < NQ; ++i)
-#pragma unroll
-                for (int hh = 0; hh < C::HALVES; ++hh)
-                    tma_load_3d(sQ + i * C::Q_BYTES + hh * BM * 128, &tmQ, hh * 64, q0 + i * BM, b * a.Hq + h,
-                                &sy.q_full);
-            const int BH = a.B * a.Hkv;
-            const int r0 = a.src0 * BH + b * a.Hkv + jkv;
-            const int r1 = a.src1 * BH + b * a.Hkv + jkv;
-            for (int j = 0; j < n_kv; ++j) {
-                const int s = j % NS;
-                if (j >= NS) wait_cta(sy, &sy.kv_empty[s], ((j / NS) - 1) & 1, a.wait_limit, a.err);
-                if (sy.abort) break;
-                uint8_t* st = sKV + s * C::STAGE;
-                mbar_arrive_expect_tx(&sy.kv_full[s], C::STAGE);
-#pragma unroll
-                for (int hh = 0; hh < C::HALVES; ++hh) {
-                    tma_load_3d(st + hh * C::HALF_T, &tmK, hh * 64, j * BN, r0, &sy.kv_full[s]);
-                    tma_load_3d(st + C::TILE + hh * C::HALF_T, &tmV, hh * 64, j * BN, r0, &sy.kv_full[s]);
-                    if (MIX) {
-                        tma_load_3d(st + 2 * C::TILE + hh * C::HALF_T, &tmK, hh * 64, j * BN, r1, &sy.kv_full[s]);
-                        tma_load_3d(st + 3 * C::TILE + hh * C::HALF_T, &tmV, hh * 64, j * BN, r1, &sy.kv_full[s]);
-                    }
-                }
-            }
-            if (sy.abort) {
-                // let copies still in flight land before the CTA's shared memory goes away
-                const int first = n_kv > NS ? n_kv - NS : 0;
-                for (int j = first; j < n_kv; ++j) {
-                    const long long t0 = clock64();
-                    while (!mbar_try_wait(&sy.kv_full[j % NS], (j / NS) & 1) && clock64() - t0 < a.wait_limit) {
-                    }
-                }
-            }
-        }
-    } else if (warp == C::W_MMA) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
-            constexpr uint32_t idO = tc::idesc_bf16(BM, D, false, true);
-            const uint32_t q_addr = smem_u32(sQ);
-            auto issue_s = [&](int i, int j) {          // S_i = Q_i K_j^T
-                const uint32_t k_addr = smem_u32(sKV + (j % NS) * C::STAGE);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk & 3) * 32;   // 16 bf16 along K inside the 128-B row
-                    const uint64_t ad = tc::smem_desc(q_addr + i * C::Q_BYTES + (kk >> 2) * (BM * 128) + off, 16, 1024,
-                                                      tc::LAYOUT_SW128);
-                    const uint64_t bd = tc::smem_desc(k_addr + (kk >> 2) * C::HALF_T + off, 16, 1024, tc::LAYOUT_SW128);
-                    tc::mma_ss(tS(i), ad, bd, idS, kk > 0 ? 1u : 0u);
-                }
-                tc::commit(&sy.s_full[i]);
-            };
-            auto issue_pv = [&](int i, int j) {         // O_i += P_i V_j, P_i read from TMEM
-                wait_cta(sy, &sy.p_full[i], j & 1, a.wait_limit, a.err);
-                tc::fence_after();
-                const uint32_t v_addr = smem_u32(sKV + (j % NS) * C::STAGE + C::TILE);
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bd = tc::smem_desc(v_addr + kk * 16 * 128, C::HALF_T, 1024, tc::LAYOUT_SW128);
-                    tc::mma_ts(tO(i), tS(i) + kk * 8, bd, idO, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-            };
-            auto wait_kv = [&](int j) {
-                wait_cta(sy, MIX ? &sy.kv_ready[j % NS] : &sy.kv_full[j % NS], (j / NS) & 1, a.wait_limit, a.err);
-                tc::fence_after();
-            };
-            wait_cta(sy, &sy.q_full, 0, a.wait_limit, a.err);
-            wait_kv(0);
-            if (nq[0] > 0) issue_s(0, 0);
-            if (nq[1] > 0) issue_s(1, 0);
-            for (int j = 0; j < n_kv && !sy.abort; ++j) {
-                const bool next = j + 1 < n_kv;
-                if (j < nq[0]) issue_pv(0, j);
-                if (next) wait_kv(j + 1);
-                if (next && j + 1 < nq[0]) issue_s(0, j + 1);
-                if (j < nq[1]) issue_pv(1, j);
-                tc::commit(&sy.kv_empty[j % NS]);
-                if (next && j + 1 < nq[1]) issue_s(1, j + 1);
-            }
-            tc::commit(&sy.o_full);
-        }
-    } else if (warp < 4 * NQ) {
+    // Warpgroup roles. Each branch first moves its per-thread register budget
+    // (setmaxnreg, executed by all four warps of the warpgroup), so the softmax threads
+    // can hold a whole S row; the budgets add up to at most the launch allocation.
+    const int wg = warp >> 2;
+    if (wg < NQ) {
+        tc::reg_inc<C::REG_SOFTMAX>();
         // ------------------------------------------------------------ softmax, one warpgroup per query tile
         const int qi = warp >> 2;
         const int wq = warp & 3;                         // lane quadrant of TMEM this warp may access
@@ -265,22 +199,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         auto step = [&](auto mask_tag, int j) {
             constexpr bool MASKED = decltype(mask_tag)::value;
             const int lim = qpos - j * BN;               // column c is visible iff c <= lim
-            // pass 1: row max of the raw (unscaled) scores, 64 columns per TMEM round trip
+            // the whole row of S in one TMEM round trip
+            uint32_t r[BN / 32][32];
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) tc::ld32(sS + c * 32, r[c]);
+            tc::wait_ld();
+            if (MASKED) {
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c * 32 + i > lim) r[c][i] = __float_as_uint(NEG_INF);
+            }
+            // row max of the raw (unscaled) scores over four independent chains
             float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c) {
-                uint32_t r0[32], r1[32];
-                tc::ld32(sS + c * 64, r0);
-                tc::ld32(sS + c * 64 + 32, r1);
-                tc::wait_ld();
+            for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    float v0 = __uint_as_float(r0[i]), v1 = __uint_as_float(r1[i]);
-                    if (MASKED && c * 64 + i > lim) v0 = NEG_INF;
-                    if (MASKED && c * 64 + 32 + i > lim) v1 = NEG_INF;
-                    mx[i & 3] = fmaxf(mx[i & 3], fmaxf(v0, v1));
-                }
-            }
+                for (int i = 0; i < 32; i += 2)
+                    mx[(i >> 1) & 3] = fmaxf(mx[(i >> 1) & 3], fmaxf(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])));
             const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.scale_log2;
             // lazy max: rescale O only when the row max grew by more than 2^8; the TMEM
             // load/store is warp-collective, so the warp rescales if any row needs it
@@ -303,36 +240,32 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     tc::st32(sO + c * 32, o32);
                 }
             }
-            // pass 2: P = 2^(s * scale - m) as bf16, packed two per column over the row's first
-            // BN/2 S columns; EMU_PAIRS of every 16 pairs take the FMA-pipe exponential
+            // P = 2^(s * scale - m) as bf16, packed two per column over the row's first BN/2
+            // S columns (every S value is in registers already); masked columns hold -inf,
+            // whose exponential is 0. EMU_PAIRS of every 16 pairs take the FMA-pipe exponential.
             const float nm = -m_used;
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
-            auto pexp = [&](uint32_t bits, int col, bool emu) {
-                const float x = fmaf(__uint_as_float(bits), a.scale_log2, nm);
-                float p = emu ? exp2_fma(x) : tc::ex2(x);
-                if (MASKED && col > lim) p = 0.f;
-                return p;
-            };
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c) {
-                uint32_t r0[32], r1[32];
-                tc::ld32(sS + c * 64, r0);
-                tc::ld32(sS + c * 64 + 32, r1);
-                tc::wait_ld();
-                uint32_t pk0[16], pk1[16];
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const bool emu = i < EMU_PAIRS;
-                    const int col = c * 64 + 2 * i;
-                    const float p0 = pexp(r0[2 * i], col, emu), p1 = pexp(r0[2 * i + 1], col + 1, emu);
-                    const float p2 = pexp(r1[2 * i], col + 32, emu), p3 = pexp(r1[2 * i + 1], col + 33, emu);
-                    ls[i & 1] += p0 + p1;
-                    ls[2 + (i & 1)] += p2 + p3;
-                    pk0[i] = pack_bf16(p0, p1);
-                    pk1[i] = pack_bf16(p2, p3);
+                    const float x0 = fmaf(__uint_as_float(r[c][2 * i]), a.scale_log2, nm);
+                    const float x1 = fmaf(__uint_as_float(r[c][2 * i + 1]), a.scale_log2, nm);
+                    float p0, p1;
+                    if (i < EMU_PAIRS) {
+                        p0 = exp2_fma(x0);
+                        p1 = exp2_fma(x1);
+                        if (MASKED && c * 32 + 2 * i > lim) p0 = 0.f;
+                        if (MASKED && c * 32 + 2 * i + 1 > lim) p1 = 0.f;
+                    } else {
+                        p0 = tc::ex2(x0);
+                        p1 = tc::ex2(x1);
+                    }
+                    ls[i & 3] += p0 + p1;
+                    pk[i] = pack_bf16(p0, p1);
                 }
-                tc::st16(sS + c * 32, pk0);
-                tc::st16(sS + c * 32 + 16, pk1);
+                tc::st16(sS + c * 16, pk);
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         };
@@ -381,7 +314,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 bulk_wait_read0();
             }
         }
-    } else if (MIX && warp >= C::W_MIX) {
+    } else if (MIX && wg == C::W_MIX / 4) {
+        tc::reg_dec<C::REG_MIXER>();
         // ------------------------------------------------------------ mixers (two-source layers)
         const int t = threadIdx.x - 32 * C::W_MIX;
         const float w = a.w[jkv];
@@ -404,6 +338,95 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             fence_proxy_async();
             mbar_arrive(&sy.kv_ready[s]);
         }
+    } else {
+        tc::reg_dec<C::REG_CTRL>();
+        if (warp == C::W_TMA) {
+            // ------------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sy.q_full, NQ * C::Q_BYTES);
+#pragma unroll
+                for (int i = 0; i < NQ; ++i)
+#pragma unroll
+                    for (int hh = 0; hh < C::HALVES; ++hh)
+                        tma_load_3d(sQ + i * C::Q_BYTES + hh * BM * 128, &tmQ, hh * 64, q0 + i * BM, b * a.Hq + h,
+                                    &sy.q_full);
+                const int BH = a.B * a.Hkv;
+                const int r0 = a.src0 * BH + b * a.Hkv + jkv;
+                const int r1 = a.src1 * BH + b * a.Hkv + jkv;
+                for (int j = 0; j < n_kv; ++j) {
+                    const int s = j % NS;
+                    if (j >= NS) wait_cta(sy, &sy.kv_empty[s], ((j / NS) - 1) & 1, a.wait_limit, a.err);
+                    if (sy.abort) break;
+                    uint8_t* st = sKV + s * C::STAGE;
+                    mbar_arrive_expect_tx(&sy.kv_full[s], C::STAGE);
+#pragma unroll
+                    for (int hh = 0; hh < C::HALVES; ++hh) {
+                        tma_load_3d(st + hh * C::HALF_T, &tmK, hh * 64, j * BN, r0, &sy.kv_full[s]);
+                        tma_load_3d(st + C::TILE + hh * C::HALF_T, &tmV, hh * 64, j * BN, r0, &sy.kv_full[s]);
+                        if (MIX) {
+                            tma_load_3d(st + 2 * C::TILE + hh * C::HALF_T, &tmK, hh * 64, j * BN, r1, &sy.kv_full[s]);
+                            tma_load_3d(st + 3 * C::TILE + hh * C::HALF_T, &tmV, hh * 64, j * BN, r1, &sy.kv_full[s]);
+                        }
+                    }
+                }
+                if (sy.abort) {
+                    // let copies still in flight land before the CTA's shared memory goes away
+                    const int first = n_kv > NS ? n_kv - NS : 0;
+                    for (int j = first; j < n_kv; ++j) {
+                        const long long t0 = clock64();
+                        while (!mbar_try_wait(&sy.kv_full[j % NS], (j / NS) & 1) && clock64() - t0 < a.wait_limit) {
+                        }
+                    }
+                }
+            }
+        } else if (warp == C::W_MMA) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
+                constexpr uint32_t idO = tc::idesc_bf16(BM, D, false, true);
+                const uint32_t q_addr = smem_u32(sQ);
+                auto issue_s = [&](int i, int j) {          // S_i = Q_i K_j^T
+                    const uint32_t k_addr = smem_u32(sKV + (j % NS) * C::STAGE);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk & 3) * 32;   // 16 bf16 along K inside the 128-B row
+                        const uint64_t ad = tc::smem_desc(q_addr + i * C::Q_BYTES + (kk >> 2) * (BM * 128) + off, 16, 1024,
+                                                          tc::LAYOUT_SW128);
+                        const uint64_t bd = tc::smem_desc(k_addr + (kk >> 2) * C::HALF_T + off, 16, 1024, tc::LAYOUT_SW128);
+                        tc::mma_ss(tS(i), ad, bd, idS, kk > 0 ? 1u : 0u);
+                    }
+                    tc::commit(&sy.s_full[i]);
+                };
+                auto issue_pv = [&](int i, int j) {         // O_i += P_i V_j, P_i read from TMEM
+                    wait_cta(sy, &sy.p_full[i], j & 1, a.wait_limit, a.err);
+                    tc::fence_after();
+                    const uint32_t v_addr = smem_u32(sKV + (j % NS) * C::STAGE + C::TILE);
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk) {
+                        const uint64_t bd = tc::smem_desc(v_addr + kk * 16 * 128, C::HALF_T, 1024, tc::LAYOUT_SW128);
+                        tc::mma_ts(tO(i), tS(i) + kk * 8, bd, idO, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                };
+                auto wait_kv = [&](int j) {
+                    wait_cta(sy, MIX ? &sy.kv_ready[j % NS] : &sy.kv_full[j % NS], (j / NS) & 1, a.wait_limit, a.err);
+                    tc::fence_after();
+                };
+                wait_cta(sy, &sy.q_full, 0, a.wait_limit, a.err);
+                wait_kv(0);
+                if (nq[0] > 0) issue_s(0, 0);
+                if (nq[1] > 0) issue_s(1, 0);
+                for (int j = 0; j < n_kv && !sy.abort; ++j) {
+                    const bool next = j + 1 < n_kv;
+                    if (j < nq[0]) issue_pv(0, j);
+                    if (next) wait_kv(j + 1);
+                    if (next && j + 1 < nq[0]) issue_s(0, j + 1);
+                    if (j < nq[1]) issue_pv(1, j);
+                    tc::commit(&sy.kv_empty[j % NS]);
+                    if (next && j + 1 < nq[1]) issue_s(1, j + 1);
+                }
+                tc::commit(&sy.o_full);
+            }
+        }
     }
 
     tc::fence_before();
@@ -423,6 +446,12 @@ cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
+        // the register split assumes the block is launched with LAUNCH_REGS per thread;
+        // with fewer, the softmax warps' setmaxnreg.inc could never be satisfied
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs * C::THREADS < C::REG_SUM) return cudaErrorInvalidConfiguration;
         attr_done = true;
     }
     dim3 grid(a.Hq, a.B, (a.S + NQ * BM - 1) / (NQ * BM));
