@@ -117,6 +117,9 @@ class DecodeRunner:
                                      basis_rank=cfg.basis_rank)
         self.w = None if cfg.lowrank else cfg.make("w")
         K.kvshare_set_map(self.h, cfg.layer_map, self.w)
+        # nothing writes the cache while the timed steps run, so consecutive decode
+        # launches may request their first K/V tiles before the previous one finishes
+        K.kvshare_set_kv_overlap(self.h, True)
         self.out = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim, device="cuda")
         self.lse = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, device="cuda")
         self.stream = torch.cuda.current_stream()
@@ -516,8 +519,25 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--only", choices=["prefill"], default=None,
+                    help="profiling aid: run only the causal prefill workload and print its numbers")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="profiling aid (with --only prefill): batch of the prefill workload")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+
+    if args.only == "prefill":
+        import torch
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        name = "depthgraft_prefill"
+        if args.batch > 0:
+            name = f"depthgraft_prefill_b{args.batch}"
+            BY_NAME[name] = BY_NAME["depthgraft_prefill"].replace(name=name, batch=args.batch)
+        pr = prefill_arm(args, name)
+        print(json.dumps({"workload": name, "tflops": pr["tflops"], "ms_per_step": pr["step_ms"],
+                          "single_source_layer_tflops": pr["single_layer_tflops"],
+                          "mix_layer_tflops": pr["mix_layer_tflops"], "gpu_launches": pr["launches"]}))
+        return
 
     if args.impl == "reference":
         reference_arm(args)

@@ -85,6 +85,7 @@ struct kvshare_ctx {
     unsigned* counters = nullptr;    // [max_batch * Hkv]
     unsigned* err = nullptr;         // status word
     int splits_override = 0;
+    int kv_overlap = 0;
     int grid_override = 0;
     int stall_next = 0;
     long long wait_limit = 4000000000LL;     // ~2 s of SM clock
@@ -213,6 +214,7 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
         c->stall_next = 0;
         // consecutive decode layers overlap launch and prologue with the previous tail
         a.pdl = 1;
+        a.kv_early = c->kv_overlap;
         cudaError_t err;
         if (cf.dtype == KVS_F32) {
             if (e.kind == KVS_SRC_LOWRANK) return KVS_EUNSUPPORTED;
@@ -591,6 +593,12 @@ kvshare_status kvshare_sync_status(kvshare_t ctx, void* stream) {
 kvshare_status kvshare_set_splits(kvshare_t ctx, int splits) {
     if (ctx == nullptr || splits < 0) return KVS_EINVAL;
     ctx->splits_override = splits;
+    return KVS_OK;
+}
+
+kvshare_status kvshare_set_kv_overlap(kvshare_t ctx, int on) {
+    if (ctx == nullptr) return KVS_EINVAL;
+    ctx->kv_overlap = on ? 1 : 0;
     return KVS_OK;
 }
 

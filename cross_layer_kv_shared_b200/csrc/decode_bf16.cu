@@ -76,10 +76,61 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         mbar_init_fence();
     }
     __syncthreads();
-    // under a dependent launch everything above overlapped the previous kernel's tail;
-    // global memory (inputs, workspace, counters) is touched only from here on
+
+    uint8_t* ring = smem + warp * NSW * C::STAGE_BYTES;
+    uint64_t* wb = &bars[warp * NSW];
+    const int my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
+    // (unit, tile) of this warp's first tile; later tiles step by NW without dividing
+    const long long g0 = tb + warp;
+    const int u_w0 = static_cast<int>(g0 / a.n_t);
+    const int t_w0 = static_cast<int>(g0 - static_cast<long long>(u_w0) * a.n_t);
+    auto advance = [&](int& u, int& t) {
+        t += NW;
+        while (t >= a.n_t) {
+            t -= a.n_t;
+            ++u;
+        }
+    };
+    int iu = u_w0, it = t_w0;        // next tile to issue
+
+    auto issue = [&](int k) {
+        (void)k;
+        const int u = iu;
+        const int t = it;
+        advance(iu, it);
+        const int row0 = a.src0 * BH + u;
+        const int row1 = MIX ? a.src1 * BH + u : 0;
+        const int s = k % NSW;
+        uint8_t* st = ring + s * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(&wb[s], C::STAGE_BYTES);
+#pragma unroll
+        for (int h = 0; h < C::HALVES; ++h) {
+            tma_load_3d(st + h * C::HALF_BYTES, &tmK, h * 64, t * TT, row0, &wb[s]);
+            tma_load_3d(st + C::TILE_BYTES + h * C::HALF_BYTES, &tmV, h * 64, t * TT, row0, &wb[s]);
+            if (MIX) {
+                tma_load_3d(st + 2 * C::TILE_BYTES + h * C::HALF_BYTES, &tmK, h * 64, t * TT, row1, &wb[s]);
+                tma_load_3d(st + 3 * C::TILE_BYTES + h * C::HALF_BYTES, &tmV, h * 64, t * TT, row1, &wb[s]);
+            }
+        }
+    };
+    // Under a dependent launch everything up to grid_dep_wait overlaps the previous
+    // kernel's tail. Inputs, workspace and counters are touched only after it; with
+    // kv_early the caller has promised that no kernel ahead on the stream writes the
+    // cache, so the first ring stages are already requested before the wait.
+    if (a.kv_early) {
+        if (lane == 0) {
+            for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
+        }
+        __syncwarp();
+    }
     grid_dep_wait();
     if (threadIdx.x == 0) grid_dep_launch();
+    if (!a.kv_early) {
+        if (lane == 0) {
+            for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
+        }
+        __syncwarp();
+    }
 
     if (a.stall && threadIdx.x == 0) {
         // test hook: nothing ever arrives on the spare barrier; the bounded wait gives up
@@ -145,46 +196,6 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         }
     };
 
-    uint8_t* ring = smem + warp * NSW * C::STAGE_BYTES;
-    uint64_t* wb = &bars[warp * NSW];
-    const int my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
-    // (unit, tile) of this warp's first tile; later tiles step by NW without dividing
-    const long long g0 = tb + warp;
-    const int u_w0 = static_cast<int>(g0 / a.n_t);
-    const int t_w0 = static_cast<int>(g0 - static_cast<long long>(u_w0) * a.n_t);
-    auto advance = [&](int& u, int& t) {
-        t += NW;
-        while (t >= a.n_t) {
-            t -= a.n_t;
-            ++u;
-        }
-    };
-    int iu = u_w0, it = t_w0;        // next tile to issue
-
-    auto issue = [&](int k) {
-        (void)k;
-        const int u = iu;
-        const int t = it;
-        advance(iu, it);
-        const int row0 = a.src0 * BH + u;
-        const int row1 = MIX ? a.src1 * BH + u : 0;
-        const int s = k % NSW;
-        uint8_t* st = ring + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&wb[s], C::STAGE_BYTES);
-#pragma unroll
-        for (int h = 0; h < C::HALVES; ++h) {
-            tma_load_3d(st + h * C::HALF_BYTES, &tmK, h * 64, t * TT, row0, &wb[s]);
-            tma_load_3d(st + C::TILE_BYTES + h * C::HALF_BYTES, &tmV, h * 64, t * TT, row0, &wb[s]);
-            if (MIX) {
-                tma_load_3d(st + 2 * C::TILE_BYTES + h * C::HALF_BYTES, &tmK, h * 64, t * TT, row1, &wb[s]);
-                tma_load_3d(st + 3 * C::TILE_BYTES + h * C::HALF_BYTES, &tmV, h * 64, t * TT, row1, &wb[s]);
-            }
-        }
-    };
-    if (lane == 0) {
-        for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
-    }
-    __syncwarp();
 
     int cur_u = -1, saved_u = -1;
     const int mi = lane >> 3;        // ldmatrix: which 8x8 matrix this lane addresses
@@ -440,7 +451,7 @@ TileShape shape_of() {
 #define KVS_TT_64S 64
 #endif
 #ifndef KVS_NSW_64S
-#define KVS_NSW_64S 2
+#define KVS_NSW_64S 3
 #endif
 #ifndef KVS_TT_64M
 #define KVS_TT_64M 32

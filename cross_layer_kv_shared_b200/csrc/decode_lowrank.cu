@@ -51,6 +51,9 @@ struct LrCfg {
     static constexpr int RING_BYTES = NW * NSW * STAGE_BYTES;
     // per-warp scratch of per-token s_K, s_V (fp32) and rank (int)
     static constexpr int TOK_BYTES = NW * TT * 3 * 4;
+    // per-warp f16 copies of the tile's K and V codes, masked to each token's rank:
+    // [K | V][TT][16] halves, rows of 32 B whose two 16-B halves swap on every 4th row
+    static constexpr int CVT_BYTES = NW * 2 * TT * 32;
     static constexpr int PD = RB + RM;    // coefficient-space partial width
     static constexpr int COMBINE_FLOATS = NW * 16 * PD + 2 * NW * 16 + 32 + 16 * PD + 16 * D + 2 * MAX_GROUP * MAX_SPLITS + 64;
     static constexpr int MERGE_STAGE_OFF = ((COMBINE_FLOATS * 4 + 1023) / 1024) * 1024;   // free smem for the merge
@@ -59,7 +62,7 @@ struct LrCfg {
     static constexpr int STAGE_FACTORS = (RB + RM) * D * 2;
     static constexpr int STAGE_BYTES_TOTAL = STAGE_FACTORS + 16 * D * 2;
     static constexpr int BODY0 = RING_BYTES > COMBINE_FLOATS * 4 ? RING_BYTES : COMBINE_FLOATS * 4;
-    static constexpr int SMEM = BODY0 + TOK_BYTES + QPROJ_FLOATS * 4 + STAGE_BYTES_TOTAL + 1024;
+    static constexpr int SMEM = BODY0 + TOK_BYTES + CVT_BYTES + QPROJ_FLOATS * 4 + STAGE_BYTES_TOTAL + 1024;
     static_assert(TT % 16 == 0 && COEF_BYTES % 1024 == 0, "tile shape");
 };
 
@@ -94,7 +97,7 @@ __device__ __forceinline__ uint32_t i8pair_bf16(uint32_t w16, bool keep0, bool k
 }
 
 template <int D, int RB, int TT, int NSW, int NW, int NH>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, 1)
 decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_constant__ CUtensorMap tmCV,
                       const __grid_constant__ CUtensorMap tmUK, const __grid_constant__ CUtensorMap tmUV,
                       const DecodeArgs a) {
@@ -105,7 +108,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     float* tok = reinterpret_cast<float*>(smem + C::BODY0);                    // [NW][3][TT]: s_K, s_V, rank
-    float* qproj = tok + NW * TT * 3;                                          // [16][RB + RM]
+    uint8_t* cvt = reinterpret_cast<uint8_t*>(tok + NW * TT * 3);              // [NW][K | V][TT][16] f16
+    float* qproj = reinterpret_cast<float*>(cvt + C::CVT_BYTES);               // [16][RB + RM]
     uint8_t* stagebuf = reinterpret_cast<uint8_t*>(qproj + C::QPROJ_FLOATS);   // factors, then q rows
     __shared__ __align__(8) uint64_t bars[NW * NSW + 1];
     __shared__ __align__(8) uint64_t fac_bar[2];    // [0]: B_K, R_K, q   [1]: B_V, R_V
@@ -185,8 +189,10 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     }
     if (a.stall && threadIdx.x == 0) mbar_wait_bounded(&bars[NW * NSW], 0, a.stall_limit, a.err);
 
-    // B fragments of q~^T (RB rows) and q^^T (16 rows): column = head nb*8 + lane/4, as bf16 hi + lo
-    uint32_t qch[RB / 16][NB][2], qcl[RB / 16][NB][2], quh[NB][2], qul[NB][2];
+    // B fragments of q~^T (RB rows, bf16 hi + lo) and q^^T (16 rows, f16: the residual term
+    // is scaled by s_K, far below the basis term, so f16's 11 bits suffice there);
+    // column = head nb*8 + lane/4
+    uint32_t qch[RB / 16][NB][2], qcl[RB / 16][NB][2], quh[NB][2];
     {
         const int cq = 2 * (lane & 3);
 #pragma unroll
@@ -203,8 +209,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 frag(ks * 16 + cq, qch[ks][nb][0], qcl[ks][nb][0]);
                 frag(ks * 16 + 8 + cq, qch[ks][nb][1], qcl[ks][nb][1]);
             }
-            frag(RB + cq, quh[nb][0], qul[nb][0]);
-            frag(RB + 8 + cq, quh[nb][1], qul[nb][1]);
+            quh[nb][0] = pack_f16(qproj[h * C::PD + RB + cq], qproj[h * C::PD + RB + cq + 1]);
+            quh[nb][1] = pack_f16(qproj[h * C::PD + RB + 8 + cq], qproj[h * C::PD + RB + 8 + cq + 1]);
         }
     }
 
@@ -225,6 +231,10 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     uint64_t* wb = &bars[warp * NSW];
     float* tks = tok + warp * TT * 3;     // [3][TT]: s_K, s_V, rank
     int* tkr = reinterpret_cast<int*>(tks + 2 * TT);
+    uint8_t* cvk = cvt + warp * 2 * TT * 32;   // this warp's f16 K codes [TT][16]
+    uint8_t* cvv = cvk + TT * 32;              //                  V codes [TT][16]
+    // byte offset of the 16-B half `seg` (channels 8 seg .. 8 seg + 7) of token row t
+    auto cvt_off = [](int t, int seg) { return static_cast<uint32_t>(t * 32 + ((seg ^ ((t >> 2) & 1)) << 4)); };
     const int span = tile1 - tile0;
     const int my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
 
@@ -291,6 +301,29 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         const uint32_t cvb = ckb + C::COEF_BYTES;
         const uint8_t* ukp = ring + s * C::STAGE_BYTES + 2 * C::COEF_BYTES;
         const uint8_t* uvp = ukp + C::U_BYTES;
+        // the tile's int8 codes -> f16, masked to each token's rank: lane = token row
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            const int tr = lane + 32 * u;
+            const int r = tkr[tr];
+            const uint4 wk = *reinterpret_cast<const uint4*>(ukp + tr * RM);
+            const uint4 wv = *reinterpret_cast<const uint4*>(uvp + tr * RM);
+            const uint32_t m0 = rank_keep(r, 0), m1 = rank_keep(r, 1), m2 = rank_keep(r, 2), m3 = rank_keep(r, 3);
+            uint4 k0, k1, v0, v1;
+            i8x4_f16(wk.x, m0, k0.x, k0.y);
+            i8x4_f16(wk.y, m1, k0.z, k0.w);
+            i8x4_f16(wk.z, m2, k1.x, k1.y);
+            i8x4_f16(wk.w, m3, k1.z, k1.w);
+            i8x4_f16(wv.x, m0, v0.x, v0.y);
+            i8x4_f16(wv.y, m1, v0.z, v0.w);
+            i8x4_f16(wv.z, m2, v1.x, v1.y);
+            i8x4_f16(wv.w, m3, v1.z, v1.w);
+            *reinterpret_cast<uint4*>(cvk + cvt_off(tr, 0)) = k0;
+            *reinterpret_cast<uint4*>(cvk + cvt_off(tr, 1)) = k1;
+            *reinterpret_cast<uint4*>(cvv + cvt_off(tr, 0)) = v0;
+            *reinterpret_cast<uint4*>(cvv + cvt_off(tr, 1)) = v1;
+        }
+        __syncwarp();
 
         float sc[MT][NB][4];
         float su[MT][NB][4];
@@ -316,23 +349,14 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 }
             }
         }
-        // ---- residual part: U_K (masked to each token's rank) q^^T
+        // ---- residual part: U_K (f16 codes masked to each token's rank) q^^T
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-            const int ta = mt * 16 + (lane >> 2);
-            const int ra = tkr[ta], rb = tkr[ta + 8];
-            const uint16_t* ua = reinterpret_cast<const uint16_t*>(ukp + ta * RM);
-            const uint16_t* ub = reinterpret_cast<const uint16_t*>(ukp + (ta + 8) * RM);
+            const int row = mt * 16 + (mi & 1) * 8 + ri;
             uint32_t af[4];
-            af[0] = i8pair_bf16(ua[q4], 2 * q4 < ra, 2 * q4 + 1 < ra);
-            af[1] = i8pair_bf16(ub[q4], 2 * q4 < rb, 2 * q4 + 1 < rb);
-            af[2] = i8pair_bf16(ua[q4 + 4], 2 * q4 + 8 < ra, 2 * q4 + 9 < ra);
-            af[3] = i8pair_bf16(ub[q4 + 4], 2 * q4 + 8 < rb, 2 * q4 + 9 < rb);
+            ldsm_x4(smem_u32(cvk) + cvt_off(row, mi >> 1), af[0], af[1], af[2], af[3]);
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                mma_bf16(su[mt][nb], af, quh[nb][0], quh[nb][1]);
-                mma_bf16(su[mt][nb], af, qul[nb][0], qul[nb][1]);
-            }
+            for (int nb = 0; nb < NB; ++nb) mma_f16(su[mt][nb], af, quh[nb][0], quh[nb][1]);
         }
         // ---- scores, mask, online softmax per head; P^T and (P s_V)^T by movmatrix
         uint32_t pb[MT][NB][2], pvb[MT][NB][2];
@@ -377,8 +401,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 pb[mt][nb][0] = movmatrix_t(lo);
                 pb[mt][nb][1] = movmatrix_t(hi);
                 const float sva = tks[TT + ta], svb = tks[TT + ta + 8];
-                pvb[mt][nb][0] = movmatrix_t(pack_bf16(p0 * sva, p1 * sva));
-                pvb[mt][nb][1] = movmatrix_t(pack_bf16(p2 * svb, p3 * svb));
+                pvb[mt][nb][0] = movmatrix_t(pack_f16(p0 * sva, p1 * sva));
+                pvb[mt][nb][1] = movmatrix_t(pack_f16(p2 * svb, p3 * svb));
             }
         }
         // ---- c^^T += C_V^T P^T
@@ -393,20 +417,15 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 for (int nb = 0; nb < NB; ++nb) mma_bf16(oc[ct][nb], af, pb[mt][nb][0], pb[mt][nb][1]);
             }
         }
-        // ---- u^^T += U_V^T (P s_V)^T, codes masked to each token's rank
+        // ---- u^^T += U_V^T (P s_V)^T: the f16 codes (masked to each token's rank) read
+        // transposed, channels as rows and tokens as k
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-            const int t0 = mt * 16 + 2 * q4;                 // tokens t0, t0+1 and t0+8, t0+9
-            const int r0 = tkr[t0], r1 = tkr[t0 + 1], r8 = tkr[t0 + 8], r9 = tkr[t0 + 9];
-            const int8_t* uv = reinterpret_cast<const int8_t*>(uvp);
-            const int i = lane >> 2;                         // channel rows i and i + 8
+            const int row = mt * 16 + (mi >> 1) * 8 + ri;
             uint32_t af[4];
-            af[0] = pack_bf16(i < r0 ? uv[t0 * RM + i] : 0, i < r1 ? uv[(t0 + 1) * RM + i] : 0);
-            af[1] = pack_bf16(i + 8 < r0 ? uv[t0 * RM + i + 8] : 0, i + 8 < r1 ? uv[(t0 + 1) * RM + i + 8] : 0);
-            af[2] = pack_bf16(i < r8 ? uv[(t0 + 8) * RM + i] : 0, i < r9 ? uv[(t0 + 9) * RM + i] : 0);
-            af[3] = pack_bf16(i + 8 < r8 ? uv[(t0 + 8) * RM + i + 8] : 0, i + 8 < r9 ? uv[(t0 + 9) * RM + i + 8] : 0);
+            ldsm_x4_t(smem_u32(cvv) + cvt_off(row, mi & 1), af[0], af[1], af[2], af[3]);
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) mma_bf16(ou[nb], af, pvb[mt][nb][0], pvb[mt][nb][1]);
+            for (int nb = 0; nb < NB; ++nb) mma_f16(ou[nb], af, pvb[mt][nb][0], pvb[mt][nb][1]);
         }
         __syncwarp();
         if (lane == 0 && k + NSW < my_n) {

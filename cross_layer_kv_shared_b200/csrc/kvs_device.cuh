@@ -140,6 +140,41 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A(16x16 f16, row) * B(16x8 f16, col) + D, fp32 accumulate
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Four int8 codes (one 32-bit word, byte i = code i) -> two f16 pairs, exactly.
+// Byte b becomes the f16 with bit pattern 0x64 | (b ^ 0x80), i.e. 1024 + 128 + code,
+// which f16 holds exactly (its spacing is 1 on [1024, 2048)); subtracting 1152 leaves
+// the code. Codes whose byte is cleared by `keep` come out as 0.
+__device__ __forceinline__ void i8x4_f16(uint32_t word, uint32_t keep, uint32_t& h01, uint32_t& h23) {
+    const uint32_t x = (word & keep) ^ 0x80808080u;
+    const uint32_t lo = __byte_perm(x, 0x64646464u, 0x5140);
+    const uint32_t hi = __byte_perm(x, 0x64646464u, 0x7362);
+    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));   // 1152
+    const __half2 a = __hsub2(*reinterpret_cast<const __half2*>(&lo), bias);
+    const __half2 b = __hsub2(*reinterpret_cast<const __half2*>(&hi), bias);
+    h01 = *reinterpret_cast<const uint32_t*>(&a);
+    h23 = *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// Byte mask of the code bytes 4w .. 4w+3 that lie below `rank` (byte i kept iff i < rank).
+__device__ __forceinline__ uint32_t rank_keep(int rank, int w) {
+    const int n = min(max(rank - 4 * w, 0), 4);
+    return n >= 4 ? 0xffffffffu : ((1u << (8 * n)) - 1u);
+}
+
 // Transpose an 8x8 matrix of 16-bit values held one pair per thread (thread t owns
 // row t/4, columns 2(t%4), 2(t%4)+1) so that thread t owns row t/4 of the transpose.
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {

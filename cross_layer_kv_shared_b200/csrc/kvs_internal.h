@@ -48,6 +48,9 @@ struct DecodeArgs {
     // the previous kernel on the stream drains, and waits (griddepcontrol.wait) before
     // its first global memory access
     int pdl;
+    // the caller guarantees no kernel ahead on the stream writes the cache: the first
+    // K/V tiles may be requested before the wait on the previous kernel
+    int kv_early;
 };
 
 // cudaLaunchKernelEx with the programmatic-stream-serialization attribute when `pdl`

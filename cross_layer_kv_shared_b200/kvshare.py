@@ -63,6 +63,7 @@ def _load():
         "kvshare_pack_residual": ([P, P, P, P, P, P, P, P, P, I, I, V], I),
         "kvshare_sync_status": ([P, V], I),
         "kvshare_set_splits": ([P, I], I),
+        "kvshare_set_kv_overlap": ([P, I], I),
         "kvshare_debug_stall_next": ([P, I], I),
         "kvshare_debug_set_grid": ([P, I], I),
         "kvshare_launch_count": ([P], ctypes.c_uint64),
@@ -208,6 +209,10 @@ def kvshare_sync_status(h, stream=None) -> int:
 
 def kvshare_set_splits(h, splits: int) -> int:
     return _check(_lib.kvshare_set_splits(h, int(splits)), "kvshare_set_splits")
+
+
+def kvshare_set_kv_overlap(h, on: bool = True) -> int:
+    return _check(_lib.kvshare_set_kv_overlap(h, 1 if on else 0), "kvshare_set_kv_overlap")
 
 
 def kvshare_debug_set_grid(h, ctas: int) -> int:

@@ -173,6 +173,17 @@ kvshare_status kvshare_sync_status(kvshare_t ctx, void* stream);
  * (batch, kv head), clamped to the number of token tiles and the workspace. */
 kvshare_status kvshare_set_splits(kvshare_t ctx, int splits);
 
+/* Overlap of consecutive decode launches (default off). Every decode launch may
+ * start (barrier set-up, tensor-map fetch) while the kernel ahead of it on the
+ * stream drains, and waits for that kernel before it reads q or writes anything.
+ * With `on` != 0 the bf16 decode also requests its first K/V tiles before that
+ * wait. Set it only when no kernel that can still be running when kvshare_decode
+ * is called writes the cache regions the call reads (for example: the step's
+ * cache appends were made before the kernels ahead of the decode, or the layers
+ * decoded read sources nothing is appending to); otherwise a tile could be read
+ * before it is written. Results are identical either way. */
+kvshare_status kvshare_set_kv_overlap(kvshare_t ctx, int on);
+
 /* Test hook: force the bf16 decode grid to `ctas` CTAs (0 = automatic). The
  * units' token tiles are cut into that many equal ranges, so a CTA may cover
  * the end of one (batch, kv head) unit and the start of the next; the units'

@@ -31,7 +31,7 @@ def make_ctx(K, cfg, splits=0, max_batch=None, max_context=None):
     return h
 
 
-def decode_gpu(K, cfg, inp, splits=0, layers=None, dev_inputs=None, keep_ctx=False, grid=0):
+def decode_gpu(K, cfg, inp, splits=0, layers=None, dev_inputs=None, keep_ctx=False, grid=0, kv_overlap=False):
     """Run kvshare_decode over all layers (or [l0, l1)) and return (out, lse) as numpy."""
     torch = torch_mod()
     d = dev_inputs if dev_inputs is not None else {n: to_dev(a, cfg.dtype) for n, a in inp.items()}
@@ -39,6 +39,8 @@ def decode_gpu(K, cfg, inp, splits=0, layers=None, dev_inputs=None, keep_ctx=Fal
     try:
         if grid:
             K.kvshare_debug_set_grid(h, grid)
+        if kv_overlap:
+            K.kvshare_set_kv_overlap(h, True)
         K.kvshare_set_map(h, cfg.layer_map, inp.get("w") if inp is not None else None)
         out = torch.full((cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim), float("nan"), device="cuda")
         lse = torch.full((cfg.layers, cfg.batch, cfg.q_heads), float("nan"), device="cuda")

@@ -98,6 +98,17 @@ def test_grids_whose_ranges_straddle_units(K, cfg, grid):
     assert_close(lse, want_lse, TOL_BF16, "lse")
 
 
+@pytest.mark.parametrize("cfg", [CLA_SMALL, DG_SMALL], ids=lambda c: c.name)
+def test_kv_overlap_changes_nothing(K, cfg):
+    # consecutive layers of one call overlap; with kv_overlap they also fetch K/V early
+    inp = cfg.make_all()
+    base, base_lse, _ = decode_gpu(K, cfg, inp)
+    got, got_lse, _ = decode_gpu(K, cfg, inp, kv_overlap=True)
+    assert np.array_equal(base, got) and np.array_equal(base_lse, got_lse)
+    want, want_lse = oracle_decode(cfg, inp)
+    assert_close(got, want, TOL_BF16, "out")
+
+
 def test_cla_layers_sharing_a_slot_match_bitwise(K):
     cfg = CLA_SMALL
     inp = cfg.make_all()
