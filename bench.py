@@ -584,7 +584,7 @@ def main():
     per_launch_bytes = main_res["read_bytes"] / cfg.layers
     achieved = per_launch_bytes / (avg_launch_ms * 1e-3) / 1e9
     kname = ("decode_lowrank_kernel<%d,%d>" % (cfg.head_dim, cfg.basis_rank) if cfg.lowrank else
-             "decode_bf16_kernel<%d,%s>" % (cfg.head_dim, "mix" if cfg.has_mix else "single"))
+             "decode_%s_kernel<%d,%s>" % (cfg.dtype, cfg.head_dim, "mix" if cfg.has_mix else "single"))
     traffic = NCU_TRAFFIC_BYTES.get(cfg.name)
     line = {
         "metric": METRIC,
@@ -597,7 +597,7 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": cfg.dtype,
         "data": "synthetic (seeded Philox, N(0,1)/8 q/k/v)",
         "config": arm_config(cfg, world),
         "kv_gbs": main_res["kv_gbs"],

@@ -257,20 +257,27 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         // ---- scale, mask the ragged tail, online softmax per head, P^T by movmatrix
         uint32_t pb[MT][NB][2];
         uint32_t pb2[MIX ? MT : 1][NB][2];
-        const int tok0 = t * TT + (lane >> 2);
+        const bool tail = (t + 1) * TT > a.T;       // only the last tile holds tokens past T
+        const int lim = a.T - t * TT - (lane >> 2);  // rows r of this lane are valid iff r < lim
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
             float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float v = MIX ? (w * sc[mt][nb][i] + w1 * sc2[mt][nb][i]) : sc[mt][nb][i];
-                    v *= a.scale_log2;
-                    if (tok0 + mt * 16 + (i >> 1) * 8 >= a.T) v = NEG_INF;
-                    sc[mt][nb][i] = v;
-                    if (i & 1) mx1 = fmaxf(mx1, v); else mx0 = fmaxf(mx0, v);
-                }
+                for (int i = 0; i < 4; ++i)
+                    sc[mt][nb][i] = (MIX ? (w * sc[mt][nb][i] + w1 * sc2[mt][nb][i]) : sc[mt][nb][i]) * a.scale_log2;
+            if (tail) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (mt * 16 + (i >> 1) * 8 >= lim) sc[mt][nb][i] = NEG_INF;
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                mx0 = fmaxf(mx0, fmaxf(sc[mt][nb][0], sc[mt][nb][2]));
+                mx1 = fmaxf(mx1, fmaxf(sc[mt][nb][1], sc[mt][nb][3]));
             }
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
@@ -281,8 +288,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             const float mn1 = fmaxf(mrow[nb][1], mx1);
             const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
             const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
-            const float cr0 = exp2f(mrow[nb][0] - ref0);
-            const float cr1 = exp2f(mrow[nb][1] - ref1);
+            const float cr0 = ex2_approx(mrow[nb][0] - ref0);
+            const float cr1 = ex2_approx(mrow[nb][1] - ref1);
             mrow[nb][0] = mn0;
             mrow[nb][1] = mn1;
             lrow[nb][0] *= cr0;
@@ -294,8 +301,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const float p0 = exp2f(sc[mt][nb][0] - ref0), p1 = exp2f(sc[mt][nb][1] - ref1);
-                const float p2 = exp2f(sc[mt][nb][2] - ref0), p3 = exp2f(sc[mt][nb][3] - ref1);
+                const float p0 = ex2_approx(sc[mt][nb][0] - ref0), p1 = ex2_approx(sc[mt][nb][1] - ref1);
+                const float p2 = ex2_approx(sc[mt][nb][2] - ref0), p3 = ex2_approx(sc[mt][nb][3] - ref1);
                 if (!MIX) {
                     const uint32_t lo = pack_bf16(p0, p1), hi = pack_bf16(p2, p3);
                     lrow[nb][0] += bf16_lo(lo) + bf16_lo(hi);

@@ -140,9 +140,28 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         mbar_init(&fac_bar[1], 1);
         mbar_init_fence();
     }
+    __syncthreads();   // every warp's ring barriers are initialised before any warp issues
     // under a dependent launch everything above overlapped the previous kernel's tail;
     // global memory (inputs, workspace, counters) is touched only from here on
     grid_dep_wait();
+    uint8_t* ring = smem + warp * NSW * C::STAGE_BYTES;
+    uint64_t* wb = &bars[warp * NSW];
+    const int span = tile1 - tile0;
+    const int my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
+
+    auto issue = [&](int k) {
+        const int t = tile0 + warp + k * NW;
+        const int s = k % NSW;
+        uint8_t* st = ring + s * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(&wb[s], C::STAGE_BYTES);
+#pragma unroll
+        for (int h = 0; h < LY::HALVES; ++h) {
+            tma_load_3d(st + h * TT * 128, &tmCK, h * 64, t * TT, crow, &wb[s]);
+            tma_load_3d(st + C::COEF_BYTES + h * TT * 128, &tmCV, h * 64, t * TT, crow, &wb[s]);
+        }
+        tma_load_3d(st + 2 * C::COEF_BYTES, &tmUK, 0, t * TT, urow, &wb[s]);
+        tma_load_3d(st + 2 * C::COEF_BYTES + C::U_BYTES, &tmUV, 0, t * TT, urow, &wb[s]);
+    };
     if (threadIdx.x == 0) {
         grid_dep_launch();
         // B_K[j], R_K[j] and the group's query rows, by bulk copy (all contiguous, 16-B aligned)
@@ -153,6 +172,11 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                   RM * D * 2, &fac_bar[0]);
         bulk_load(stagebuf + C::STAGE_FACTORS, qsrc, g * D * 2, &fac_bar[0]);
     }
+    // then every warp's first tiles, which stream while the query is projected
+    if (lane == 0) {
+        for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
+    }
+    __syncwarp();
     for (int idx = g * C::PD + threadIdx.x; idx < 16 * C::PD; idx += blockDim.x) qproj[idx] = 0.f;
     __syncthreads();
     // ---- q~ = B_K q and q^ = R_K q for the g heads: one warp per output, lanes over d
@@ -227,30 +251,13 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) mrow[nb][0] = mrow[nb][1] = NEG_INF, lrow[nb][0] = lrow[nb][1] = 0.f;
 
-    uint8_t* ring = smem + warp * NSW * C::STAGE_BYTES;
-    uint64_t* wb = &bars[warp * NSW];
     float* tks = tok + warp * TT * 3;     // [3][TT]: s_K, s_V, rank
     int* tkr = reinterpret_cast<int*>(tks + 2 * TT);
     uint8_t* cvk = cvt + warp * 2 * TT * 32;   // this warp's f16 K codes [TT][16]
     uint8_t* cvv = cvk + TT * 32;              //                  V codes [TT][16]
     // byte offset of the 16-B half `seg` (channels 8 seg .. 8 seg + 7) of token row t
     auto cvt_off = [](int t, int seg) { return static_cast<uint32_t>(t * 32 + ((seg ^ ((t >> 2) & 1)) << 4)); };
-    const int span = tile1 - tile0;
-    const int my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
 
-    auto issue = [&](int k) {
-        const int t = tile0 + warp + k * NW;
-        const int s = k % NSW;
-        uint8_t* st = ring + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&wb[s], C::STAGE_BYTES);
-#pragma unroll
-        for (int h = 0; h < LY::HALVES; ++h) {
-            tma_load_3d(st + h * TT * 128, &tmCK, h * 64, t * TT, crow, &wb[s]);
-            tma_load_3d(st + C::COEF_BYTES + h * TT * 128, &tmCV, h * 64, t * TT, crow, &wb[s]);
-        }
-        tma_load_3d(st + 2 * C::COEF_BYTES, &tmUK, 0, t * TT, urow, &wb[s]);
-        tma_load_3d(st + 2 * C::COEF_BYTES + C::U_BYTES, &tmUV, 0, t * TT, urow, &wb[s]);
-    };
     // per-token scales and ranks of a tile, loaded by the lanes (tokens lane, lane+32, ...)
     constexpr int TPL = TT / 32;
     float pf_sk[TPL], pf_sv[TPL];
@@ -269,9 +276,6 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             }
         }
     };
-    if (lane == 0) {
-        for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
-    }
     if (my_n > 0) prefetch(0);
     __syncwarp();
 
@@ -308,7 +312,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             const int r = tkr[tr];
             const uint4 wk = *reinterpret_cast<const uint4*>(ukp + tr * RM);
             const uint4 wv = *reinterpret_cast<const uint4*>(uvp + tr * RM);
-            const uint32_t m0 = rank_keep(r, 0), m1 = rank_keep(r, 1), m2 = rank_keep(r, 2), m3 = rank_keep(r, 3);
+            uint32_t m0, m1, m2, m3;
+            rank_keep4(r, m0, m1, m2, m3);
             uint4 k0, k1, v0, v1;
             i8x4_f16(wk.x, m0, k0.x, k0.y);
             i8x4_f16(wk.y, m1, k0.z, k0.w);
@@ -360,19 +365,33 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         }
         // ---- scores, mask, online softmax per head; P^T and (P s_V)^T by movmatrix
         uint32_t pb[MT][NB][2], pvb[MT][NB][2];
+        const bool tail = (t + 1) * TT > a.T;       // only the last tile holds tokens past T
+        const int lim = a.T - t * TT;
+        float skr[MT][2];                            // s_K of this lane's two rows per m tile
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            skr[mt][0] = tks[mt * 16 + (lane >> 2)];
+            skr[mt][1] = tks[mt * 16 + (lane >> 2) + 8];
+        }
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
             float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int tt = mt * 16 + (lane >> 2) + (i >> 1) * 8;
-                    float v = (sc[mt][nb][i] + tks[tt] * su[mt][nb][i]) * a.scale_log2;
-                    if (t * TT + tt >= a.T) v = NEG_INF;
-                    sc[mt][nb][i] = v;
-                    if (i & 1) mx1 = fmaxf(mx1, v); else mx0 = fmaxf(mx0, v);
-                }
+                for (int i = 0; i < 4; ++i)
+                    sc[mt][nb][i] = (sc[mt][nb][i] + skr[mt][i >> 1] * su[mt][nb][i]) * a.scale_log2;
+            if (tail) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (mt * 16 + (lane >> 2) + (i >> 1) * 8 >= lim) sc[mt][nb][i] = NEG_INF;
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                mx0 = fmaxf(mx0, fmaxf(sc[mt][nb][0], sc[mt][nb][2]));
+                mx1 = fmaxf(mx1, fmaxf(sc[mt][nb][1], sc[mt][nb][3]));
             }
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
@@ -382,7 +401,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             const float mn0 = fmaxf(mrow[nb][0], mx0), mn1 = fmaxf(mrow[nb][1], mx1);
             const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
             const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
-            const float cr0 = exp2f(mrow[nb][0] - ref0), cr1 = exp2f(mrow[nb][1] - ref1);
+            const float cr0 = ex2_approx(mrow[nb][0] - ref0), cr1 = ex2_approx(mrow[nb][1] - ref1);
             mrow[nb][0] = mn0;
             mrow[nb][1] = mn1;
             lrow[nb][0] *= cr0;
@@ -393,8 +412,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const int ta = mt * 16 + (lane >> 2);
-                const float p0 = exp2f(sc[mt][nb][0] - ref0), p1 = exp2f(sc[mt][nb][1] - ref1);
-                const float p2 = exp2f(sc[mt][nb][2] - ref0), p3 = exp2f(sc[mt][nb][3] - ref1);
+                const float p0 = ex2_approx(sc[mt][nb][0] - ref0), p1 = ex2_approx(sc[mt][nb][1] - ref1);
+                const float p2 = ex2_approx(sc[mt][nb][2] - ref0), p3 = ex2_approx(sc[mt][nb][3] - ref1);
                 const uint32_t lo = pack_bf16(p0, p1), hi = pack_bf16(p2, p3);
                 lrow[nb][0] += bf16_lo(lo) + bf16_lo(hi);
                 lrow[nb][1] += bf16_hi(lo) + bf16_hi(hi);

@@ -169,10 +169,16 @@ __device__ __forceinline__ void i8x4_f16(uint32_t word, uint32_t keep, uint32_t&
     h23 = *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// Byte mask of the code bytes 4w .. 4w+3 that lie below `rank` (byte i kept iff i < rank).
-__device__ __forceinline__ uint32_t rank_keep(int rank, int w) {
-    const int n = min(max(rank - 4 * w, 0), 4);
-    return n >= 4 ? 0xffffffffu : ((1u << (8 * n)) - 1u);
+// Byte masks of the 16 code bytes of a token (byte i kept iff i < rank, 0 <= rank <= 16),
+// as four 32-bit words: bytes 0-7 and 8-15 each from one 64-bit shift.
+__device__ __forceinline__ void rank_keep4(int rank, uint32_t& m0, uint32_t& m1, uint32_t& m2, uint32_t& m3) {
+    const int lo = min(rank, 8), hi = max(rank - 8, 0);
+    const unsigned long long a = lo >= 8 ? ~0ull : ((1ull << (8 * lo)) - 1ull);
+    const unsigned long long b = hi >= 8 ? ~0ull : ((1ull << (8 * hi)) - 1ull);
+    m0 = static_cast<uint32_t>(a);
+    m1 = static_cast<uint32_t>(a >> 32);
+    m2 = static_cast<uint32_t>(b);
+    m3 = static_cast<uint32_t>(b >> 32);
 }
 
 // Transpose an 8x8 matrix of 16-bit values held one pair per thread (thread t owns
@@ -202,6 +208,13 @@ __device__ __forceinline__ uint32_t swz128(int row, int c) {
 // (rows stay 16-byte aligned so whole partial blocks can move by bulk copy).
 __host__ __device__ constexpr int partial_width(int D) { return D + 4; }
 
+// 2^x by the MUFU unit (ex2.approx, flush-to-zero): one instruction; -inf gives 0.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
@@ -221,10 +234,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 // With one partial per unit the CTA emits it at once. Otherwise it stores its
 // partial and the last CTA of the unit to arrive merges all partials:
 // M = max m_s, l = sum 2^(m_s - M) l_s, v = sum 2^(m_s - M) v_s, then emits
-// (and resets the unit's arrival counter to zero). The merge is parallel:
-// every thread loads (m, l) pairs, one warp per head reduces them, and the
-// partial blocks are bulk-copied into `stage` (free shared memory of
-// `stage_bytes`, 16-B aligned; 0 means read them directly).
+// (and resets the unit's arrival counter to zero). Arrival is one acq_rel
+// atomic per CTA. The last CTA bulk-copies the unit's partials (contiguous) into
+// `stage` (free shared memory of `stage_bytes`, 16-B aligned) in one copy when
+// they fit, in chunks otherwise (0 bytes: read them directly); one warp per head
+// reduces (m, l), then every thread combines its share of the vector.
 // `emit(v, l, m)` writes the unit's outputs from v [g][DV] (shared memory),
 // l[g] and m[g]; it is called by all threads of the CTA.
 // sm_scratch holds at least 2 * g * count floats; sm_v is reused for the merge.
@@ -259,26 +273,56 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         part[tid * PD + DV] = sm_m[tid];
         part[tid * PD + DV + 1] = sm_l[tid];
     }
-    __threadfence();
     __syncthreads();
     __shared__ unsigned s_is_last;
     if (tid == 0) {
-        const unsigned prev = atomicAdd(a.counters + unit, 1u);
+        // one acq_rel atomic: its release publishes this CTA's partial (ordered before it
+        // by the barrier), its acquire lets the last arrival see every other partial
+        unsigned prev;
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;"
+                     : "=r"(prev)
+                     : "l"(a.counters + unit)
+                     : "memory");
         s_is_last = (prev == static_cast<unsigned>(count - 1)) ? 1u : 0u;
     }
     __syncthreads();
     if (!s_is_last) return;
-    __threadfence();
     const int n = count;
     const float* base = a.ws + static_cast<size_t>(slot0) * per;
     float* fm = sm_scratch;            // [n][g]: m, then the factors 2^(m - M)
     float* fl = sm_scratch + n * g;    // [n][g]: l
     __shared__ float hm[MAX_GROUP], hl[MAX_GROUP];
-    for (int idx = tid; idx < n * g; idx += nthr) {
-        const int sp = idx / g;
-        const int h = idx % g;
-        fm[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV);
-        fl[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 1);
+    __shared__ __align__(8) uint64_t mbar;
+    const int chunk = stage_bytes / (per * 4);
+    float* sp_buf = reinterpret_cast<float*>(stage);
+    const bool one_copy = chunk >= n;  // the unit's partials are contiguous: one bulk copy
+    if (chunk >= 1) {
+        if (tid == 0) {
+            mbar_init(&mbar, 1);
+            mbar_init_fence();
+            if (one_copy) {
+                asm volatile("fence.proxy.async;" ::: "memory");
+                mbar_arrive_expect_tx(&mbar, static_cast<unsigned>(n * per * 4));
+                bulk_load(sp_buf, base, static_cast<unsigned>(n * per * 4), &mbar);
+            }
+        }
+        __syncthreads();
+    }
+    if (one_copy) {
+        mbar_wait_bounded(&mbar, 0, a.wait_limit, a.err);
+        for (int idx = tid; idx < n * g; idx += nthr) {
+            const int sp = idx / g;
+            const int h = idx % g;
+            fm[idx] = sp_buf[sp * per + h * PD + DV];
+            fl[idx] = sp_buf[sp * per + h * PD + DV + 1];
+        }
+    } else {
+        for (int idx = tid; idx < n * g; idx += nthr) {
+            const int sp = idx / g;
+            const int h = idx % g;
+            fm[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV);
+            fl[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 1);
+        }
     }
     __syncthreads();
     const int warp = tid >> 5, lane = tid & 31, nwarps = nthr >> 5;
@@ -303,15 +347,19 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
     float acc[MAXO];
 #pragma unroll
     for (int k = 0; k < MAXO; ++k) acc[k] = 0.f;
-    const int chunk = stage_bytes / (per * 4);
-    if (chunk >= 1) {
-        __shared__ __align__(8) uint64_t mbar;
-        if (tid == 0) {
-            mbar_init(&mbar, 1);
-            mbar_init_fence();
+    if (one_copy) {
+#pragma unroll
+        for (int k = 0; k < MAXO; ++k) {
+            const int idx = tid + k * nthr;
+            if (idx < g * DV) {
+                const int h = idx / DV;
+                const int e = idx % DV;
+                float v = 0.f;
+                for (int c = 0; c < n; ++c) v += fm[c * g + h] * sp_buf[c * per + h * PD + e];
+                acc[k] = v;
+            }
         }
-        __syncthreads();
-        float* sp_buf = reinterpret_cast<float*>(stage);
+    } else if (chunk >= 1) {
         unsigned phase = 0;
         for (int s0 = 0; s0 < n; s0 += chunk) {
             const int cnt = min(chunk, n - s0);
