@@ -128,7 +128,12 @@ kvshare_status kvshare_set_map(kvshare_t ctx, const kvshare_layer* map, const fl
  *   q:   [L][batch][Hq][d] in the config dtype (layer l at offset l*batch*Hq*d)
  *   out: [L][batch][Hq][d] fp32
  *   lse: [L][batch][Hq] fp32 natural-log sum of exp of the scaled scores, or NULL
- * Only rows of layers [l0, l1) are written. */
+ * Only rows of layers [l0, l1) are written. Each launch uses programmatic
+ * dependent launch: it may be scheduled while the kernel ahead of it on the
+ * stream drains, but reads q and writes anything only after that kernel has
+ * completed (see kvshare_set_kv_overlap for the one exception). One
+ * (batch, kv head) unit may be split over several CTAs whose partials merge in
+ * the context's workspace; results agree to fp32 rounding whatever the split. */
 kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const void* q,
                               float* out, float* lse, int l0, int l1, void* stream);
 

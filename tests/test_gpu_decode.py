@@ -178,33 +178,18 @@ def _device_inputs(cfg):
     return {n: sgpu.make_device(cfg, n) for n in cfg.recipe()}
 
 
-def _sampled_oracle(cfg, q_host, w, layers, batches):
-    """Oracle outputs at (layer, batch) pairs, drawing only the needed cache slices on the host."""
-    cache = {}
-
-    def get(name, index):
-        key = (name, index)
-        if key not in cache:
-            cache[key] = cfg.make(name, index)
-        from oracle import kvshare_ref as ref
-        return ref.to_f64(cache[key], cfg.dtype)
-    from oracle import kvshare_ref as ref
-    res = {}
-    for l in layers:
-        for b in batches:
-            for j in range(cfg.kv_heads):
-                g = cfg.group
-                o, s = ref.decode_head_group(cfg.layer_map, l, b, j, ref.to_f64(q_host[l, b, j * g:(j + 1) * g], cfg.dtype),
-                                             get, w=w)
-                res[(l, b, j)] = (o, s)
-    return res
+def _sampled_batches(cfg):
+    """Batch 0 plus four seeded batches (all batches when there are at most four)."""
+    if cfg.batch <= 4:
+        return list(range(cfg.batch))
+    rng = np.random.default_rng(cfg.seed)
+    return [0] + sorted(int(x) for x in rng.choice(np.arange(1, cfg.batch), 4, replace=False))
 
 
-@pytest.mark.parametrize("cfg,layers,batches", [
-    (CLA2_1P1B, list(range(22)), [0, 17]),
-    (DEPTHGRAFT_DECODE, [0, 3, 8, 11, 16, 19, 23], [5]),
-], ids=["cla2_1p1b", "depthgraft_decode"])
-def test_full_size_sampled(K, cfg, layers, batches):
+@pytest.mark.parametrize("cfg", [CLA2_1P1B, DEPTHGRAFT_DECODE], ids=lambda c: c.name)
+def test_full_size_sampled(K, cfg):
+    # every layer and kv head (all query heads) of batch 0 and four seeded batches
+    layers, batches = list(range(cfg.layers)), _sampled_batches(cfg)
     import torch
     d = _device_inputs(cfg)
     q_host = cfg.make("q")
@@ -219,11 +204,36 @@ def test_full_size_sampled(K, cfg, layers, batches):
         cache = K.Cache(batch=cfg.batch, context=cfg.context, k=d["k"], v=d["v"], slots=cfg.slots)
         K.kvshare_decode(h, cache, d["q"], out, lse)
         assert K.kvshare_sync_status(h) == K.KVS_OK
+        # the launch configuration bench.py times: per-layer calls in cold order, early
+        # K/V requests across launches, captured once as a CUDA graph and replayed
+        import bench
+        K.kvshare_set_kv_overlap(h, True)
+        out2 = torch.full_like(out, float("nan"))
+        lse2 = torch.full_like(lse, float("nan"))
+        order = bench.cold_order(cfg)
+        for l in order:           # eager pass: attributes and tensor maps set up outside the capture
+            K.kvshare_decode(h, cache, d["q"], out2, lse2, l, l + 1)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            cap = torch.cuda.current_stream()
+            for l in order:
+                K.kvshare_decode(h, cache, d["q"], out2, lse2, l, l + 1, cap)
+        out2.fill_(float("nan"))
+        graph.replay()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert K.kvshare_sync_status(h) == K.KVS_OK
+        del graph
+        assert torch.equal(out, out2) and torch.equal(lse, lse2)
     finally:
         K.kvshare_destroy(h)
     out = out.cpu().numpy()
     lse = lse.cpu().numpy()
-    want = _sampled_oracle(cfg, q_host, w, layers, batches)
+    import oracle_pool
+    units = [(l, b, j) for l in layers for b in batches for j in range(cfg.kv_heads)]
+    res = oracle_pool.run(oracle_pool.decode_unit, [(cfg.name, l, b, j) for (l, b, j) in units])
+    want = dict(zip(units, res))
     g = cfg.group
     worst = 0.0
     for (l, b, j), (o, s) in want.items():

@@ -118,26 +118,19 @@ def test_full_size_sampled(K):
         assert K.kvshare_sync_status(h) == K.KVS_OK
     finally:
         K.kvshare_destroy(h)
+    # every layer and q head of batch 0 and one seeded batch, at rows {0, 1, 127, 128,
+    # 2047, 4095} plus 26 seeded rows
     rng = np.random.default_rng(99)
     rows = np.unique(np.concatenate([[0, 1, 127, 128, 2047, 4095], rng.integers(0, S, 26)]))
-    g = cfg.group
+    batches = [0, int(rng.integers(1, cfg.batch))]
+    import oracle_pool
+    units = [(l, b, hh) for l in range(cfg.layers) for b in batches for hh in range(cfg.q_heads)]
+    res = oracle_pool.run(oracle_pool.prefill_unit, [(cfg.name, l, b, hh, rows) for (l, b, hh) in units])
+    out_h = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    lse_h = lse.cpu().numpy()
     worst = 0.0
-    for l in range(cfg.layers):
-        b = int(rng.integers(cfg.batch))
-        hh = int(rng.integers(cfg.q_heads))
-        kind, s0, s1 = cfg.layer_map[l]
-        j = hh // g
-        K1 = ref.bf16_bits_to_f64(cfg.make("k", (s0, b, j)))
-        V1 = ref.bf16_bits_to_f64(cfg.make("v", (s0, b, j)))
-        if kind == MIX:
-            K2 = ref.bf16_bits_to_f64(cfg.make("k", (s1, b, j)))
-            V2 = ref.bf16_bits_to_f64(cfg.make("v", (s1, b, j)))
-            Kt, Vt = ref.kv_mix(w[l][j], K1, K2), ref.kv_mix(w[l][j], V1, V2)
-        else:
-            Kt, Vt = K1, V1
-        q = ref.bf16_bits_to_f64(cfg.make("q", (l, b, hh)))[rows]
-        o, s, _ = ref.attend(q, Kt, Vt, 1 / np.sqrt(cfg.head_dim), visible=rows + 1)
-        got = ref.bf16_bits_to_f64(out[l, b, hh].view(torch.int16).cpu().numpy().view(np.uint16))[rows]
+    for (l, b, hh), (o, s) in zip(units, res):
+        got = ref.bf16_bits_to_f64(out_h[l, b, hh][rows])
         worst = max(worst, assert_close(got, o, TOL, f"l{l} b{b} h{hh}")[0])
-        assert_close(lse[l, b, hh].cpu().numpy()[rows], s, TOL, f"lse l{l}")
+        assert_close(lse_h[l, b, hh][rows], s, TOL, f"lse l{l} b{b} h{hh}")
     print(f"depthgraft_prefill: worst max|d| {worst:.3e}")
