@@ -249,7 +249,7 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
             a.r_k = static_cast<const uint16_t*>(k->r_k) + static_cast<size_t>(l) * Hkv * 16 * D;
             a.r_v = static_cast<const uint16_t*>(k->r_v) + static_cast<size_t>(l) * Hkv * 16 * D;
             a.rank = k->rank + static_cast<size_t>(l) * B * T;
-            CUtensorMap maps[7];
+            CUtensorMap maps[4];
             const int crows = k->pairs * B * Hkv;
             const int box0 = Rb < 64 ? Rb : 64;
             const CUtensorMapSwizzle sw = Rb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
@@ -260,20 +260,6 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
                 !get_map(c, a.u_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, T, B * Hkv, 16, tt,
                          CU_TENSOR_MAP_SWIZZLE_NONE, &maps[3]))
                 return KVS_ECUDA;
-            // per-token scales [B*Hkv][T] fp16 and ranks [B][T] u8 by TMA when their rows
-            // are 16-B multiples and the layer's arrays start 16-B aligned
-            const bool al = T % 16 == 0 && (reinterpret_cast<uintptr_t>(a.s_k) & 15) == 0 &&
-                            (reinterpret_cast<uintptr_t>(a.s_v) & 15) == 0 &&
-                            (reinterpret_cast<uintptr_t>(a.rank) & 15) == 0;
-            a.tok_tma = 0;
-            maps[4] = maps[5] = maps[6] = maps[0];
-            if (al && get_map(c, a.s_k, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, T, B * Hkv, 1, tt, 1,
-                              CU_TENSOR_MAP_SWIZZLE_NONE, &maps[4]) &&
-                get_map(c, a.s_v, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, T, B * Hkv, 1, tt, 1,
-                        CU_TENSOR_MAP_SWIZZLE_NONE, &maps[5]) &&
-                get_map(c, a.rank, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, B, 1, tt, 1,
-                        CU_TENSOR_MAP_SWIZZLE_NONE, &maps[6]))
-                a.tok_tma = 1;
             err = launch_decode_lowrank(D, Rb, a, maps, st);
         } else {
             const bool mix = e.kind == KVS_SRC_MIX;

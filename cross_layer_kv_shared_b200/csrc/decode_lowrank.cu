@@ -47,18 +47,12 @@ struct LrCfg {
     using L = CoefLayout<RB>;
     static constexpr int COEF_BYTES = TT * RB * 2;
     static constexpr int U_BYTES = TT * RM;
-    // per-token s_K, s_V (fp16) and rank (u8) of the tile, when they come by TMA; every
-    // TMA destination in shared memory starts on a 128-byte boundary
+    // every TMA destination in shared memory starts on a 128-byte boundary
     static constexpr int ALIGN128(int x) { return (x + 127) / 128 * 128; }
     static constexpr int OFF_UK = 2 * COEF_BYTES;
     static constexpr int OFF_UV = OFF_UK + ALIGN128(U_BYTES);
-    static constexpr int OFF_SK = OFF_UV + ALIGN128(U_BYTES);
-    static constexpr int OFF_SV = OFF_SK + ALIGN128(TT * 2);
-    static constexpr int OFF_RK = OFF_SV + ALIGN128(TT * 2);
-    static constexpr int TOK_TX = TT * 2 * 2 + TT;
-    static constexpr int STAGE_BYTES = ((OFF_RK + TT + 1023) / 1024) * 1024;   // keeps swizzled tiles aligned
-    static_assert(COEF_BYTES % 128 == 0 && OFF_UK % 128 == 0 && OFF_UV % 128 == 0 && OFF_SK % 128 == 0 &&
-                      OFF_SV % 128 == 0 && OFF_RK % 128 == 0,
+    static constexpr int STAGE_BYTES = ((OFF_UV + U_BYTES + 1023) / 1024) * 1024;   // keeps swizzled tiles aligned
+    static_assert(COEF_BYTES % 128 == 0 && OFF_UK % 128 == 0 && OFF_UV % 128 == 0,
                   "TMA destinations must be 128-byte aligned");
     static constexpr int RING_BYTES = NW * NSW * STAGE_BYTES;
     // per-warp scratch of per-token s_K, s_V (fp32) and rank (int)
@@ -108,14 +102,11 @@ __device__ __forceinline__ uint32_t i8pair_bf16(uint32_t w16, bool keep0, bool k
     return pack_bf16(static_cast<float>(x0), static_cast<float>(x1));
 }
 
-// TOKTMA: the tile's per-token scales and ranks arrive by TMA with the tile (the
-// context is a multiple of 16 tokens); otherwise each lane loads its tokens' values.
-template <int D, int RB, int TT, int NSW, int NW, int NH, bool TOKTMA>
+template <int D, int RB, int TT, int NSW, int NW, int NH>
 __global__ void __launch_bounds__(NW * 32, 1)
 decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_constant__ CUtensorMap tmCV,
                       const __grid_constant__ CUtensorMap tmUK, const __grid_constant__ CUtensorMap tmUV,
-                      const __grid_constant__ CUtensorMap tmSK, const __grid_constant__ CUtensorMap tmSV,
-                      const __grid_constant__ CUtensorMap tmRK, const DecodeArgs a) {
+                      const DecodeArgs a) {
     using C = LrCfg<D, RB, TT, NSW, NW>;
     using LY = typename C::L;
     constexpr int MT = TT / 16;
@@ -150,11 +141,6 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         prefetch_tmap(&tmCV);
         prefetch_tmap(&tmUK);
         prefetch_tmap(&tmUV);
-        if (TOKTMA) {
-            prefetch_tmap(&tmSK);
-            prefetch_tmap(&tmSV);
-            prefetch_tmap(&tmRK);
-        }
         for (int i = 0; i < NW * NSW + 1; ++i) mbar_init(&bars[i], 1);
         mbar_init(&fac_bar[0], 1);
         mbar_init(&fac_bar[1], 1);
@@ -173,7 +159,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         const int t = tile0 + warp + k * NW;
         const int s = k % NSW;
         uint8_t* st = ring + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&wb[s], 2 * C::COEF_BYTES + 2 * C::U_BYTES + (TOKTMA ? C::TOK_TX : 0));
+        mbar_arrive_expect_tx(&wb[s], 2 * C::COEF_BYTES + 2 * C::U_BYTES);
 #pragma unroll
         for (int h = 0; h < LY::HALVES; ++h) {
             tma_load_3d(st + h * TT * 128, &tmCK, h * 64, t * TT, crow, &wb[s]);
@@ -181,11 +167,6 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         }
         tma_load_3d(st + C::OFF_UK, &tmUK, 0, t * TT, urow, &wb[s]);
         tma_load_3d(st + C::OFF_UV, &tmUV, 0, t * TT, urow, &wb[s]);
-        if (TOKTMA) {
-            tma_load_3d(st + C::OFF_SK, &tmSK, t * TT, urow, 0, &wb[s]);
-            tma_load_3d(st + C::OFF_SV, &tmSV, t * TT, urow, 0, &wb[s]);
-            tma_load_3d(st + C::OFF_RK, &tmRK, t * TT, b, 0, &wb[s]);
-        }
     };
     if (threadIdx.x == 0) {
         grid_dep_launch();
@@ -301,7 +282,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             }
         }
     };
-    if (!TOKTMA && my_n > 0) prefetch(0);
+    if (my_n > 0) prefetch(0);
     __syncwarp();
 
     const int mi = lane >> 3;
@@ -311,15 +292,13 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         const int s = k % NSW;
         // publish this tile's per-token values, start fetching the next tile's
         __syncwarp();
-        if (!TOKTMA) {
 #pragma unroll
-            for (int u = 0; u < TPL; ++u) {
-                tks[lane + 32 * u] = pf_sk[u];
-                tks[TT + lane + 32 * u] = pf_sv[u];
-                tkr[lane + 32 * u] = pf_r[u];
-            }
-            if (k + 1 < my_n) prefetch(k + 1);
+        for (int u = 0; u < TPL; ++u) {
+            tks[lane + 32 * u] = pf_sk[u];
+            tks[TT + lane + 32 * u] = pf_sv[u];
+            tkr[lane + 32 * u] = pf_r[u];
         }
+        if (k + 1 < my_n) prefetch(k + 1);
         __syncwarp();
         const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&wb[s], (k / NSW) & 1, a.wait_limit, a.err));
         if (!ok) {
@@ -332,17 +311,11 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         const uint32_t cvb = ckb + C::COEF_BYTES;
         const uint8_t* ukp = ring + s * C::STAGE_BYTES + C::OFF_UK;
         const uint8_t* uvp = ring + s * C::STAGE_BYTES + C::OFF_UV;
-        const uint16_t* tsk = reinterpret_cast<const uint16_t*>(ring + s * C::STAGE_BYTES + C::OFF_SK);
-        const uint16_t* tsv = reinterpret_cast<const uint16_t*>(ring + s * C::STAGE_BYTES + C::OFF_SV);
-        const uint8_t* trk = ring + s * C::STAGE_BYTES + C::OFF_RK;
-        auto tok_sk = [&](int tt) { return TOKTMA ? __half2float(__ushort_as_half(tsk[tt])) : tks[tt]; };
-        auto tok_sv = [&](int tt) { return TOKTMA ? __half2float(__ushort_as_half(tsv[tt])) : tks[TT + tt]; };
-        auto tok_rank = [&](int tt) { return TOKTMA ? static_cast<int>(trk[tt]) : tkr[tt]; };
         // the tile's int8 codes -> f16, masked to each token's rank: lane = token row
 #pragma unroll
         for (int u = 0; u < TPL; ++u) {
             const int tr = lane + 32 * u;
-            const int r = tok_rank(tr);
+            const int r = tkr[tr];
             const uint4 wk = *reinterpret_cast<const uint4*>(ukp + tr * RM);
             const uint4 wv = *reinterpret_cast<const uint4*>(uvp + tr * RM);
             uint32_t m0, m1, m2, m3;
@@ -403,8 +376,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         float skr[MT][2];                            // s_K of this lane's two rows per m tile
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-            skr[mt][0] = tok_sk(mt * 16 + (lane >> 2));
-            skr[mt][1] = tok_sk(mt * 16 + (lane >> 2) + 8);
+            skr[mt][0] = tks[mt * 16 + (lane >> 2)];
+            skr[mt][1] = tks[mt * 16 + (lane >> 2) + 8];
         }
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
@@ -452,7 +425,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 lrow[nb][1] += bf16_hi(lo) + bf16_hi(hi);
                 pb[mt][nb][0] = movmatrix_t(lo);
                 pb[mt][nb][1] = movmatrix_t(hi);
-                const float sva = tok_sv(ta), svb = tok_sv(ta + 8);
+                const float sva = tks[TT + ta], svb = tks[TT + ta + 8];
                 pvb[mt][nb][0] = movmatrix_t(pack_f16(p0 * sva, p1 * sva));
                 pvb[mt][nb][1] = movmatrix_t(pack_f16(p2 * svb, p3 * svb));
             }
@@ -560,10 +533,10 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 smem + C::MERGE_STAGE_OFF, C::BODY0 > C::MERGE_STAGE_OFF ? C::BODY0 - C::MERGE_STAGE_OFF : 0, emit);
 }
 
-template <int D, int RB, int TT, int NSW, int NW, int NH, bool TOKTMA>
+template <int D, int RB, int TT, int NSW, int NW, int NH>
 cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
     using C = LrCfg<D, RB, TT, NSW, NW>;
-    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, NH, TOKTMA>;
+    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, NH>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -571,23 +544,18 @@ cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t
         attr_done = true;
     }
     dim3 grid(a.splits, a.Hkv, a.B);
-    return launch_kernel(kern, grid, dim3(NW * 32), C::SMEM, st, a.pdl != 0, maps[0], maps[1], maps[2], maps[3],
-                         maps[4], maps[5], maps[6], a);
+    return launch_kernel(kern, grid, dim3(NW * 32), C::SMEM, st, a.pdl != 0, maps[0], maps[1], maps[2], maps[3], a);
 }
 
 template <int D, int RB, int TT, int NSW, int NW>
 cudaError_t launch_one(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
-    if (a.tok_tma)
-        return a.g <= 8 ? launch_nh<D, RB, TT, NSW, NW, 8, true>(a, maps, st)
-                        : launch_nh<D, RB, TT, NSW, NW, 16, true>(a, maps, st);
-    return a.g <= 8 ? launch_nh<D, RB, TT, NSW, NW, 8, false>(a, maps, st)
-                    : launch_nh<D, RB, TT, NSW, NW, 16, false>(a, maps, st);
+    return a.g <= 8 ? launch_nh<D, RB, TT, NSW, NW, 8>(a, maps, st) : launch_nh<D, RB, TT, NSW, NW, 16>(a, maps, st);
 }
 
 template <int D, int RB, int TT, int NSW, int NW>
 int occupancy_of() {
     using C = LrCfg<D, RB, TT, NSW, NW>;
-    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, 8, false>;
+    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, 8>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NW * 32, C::SMEM) != cudaSuccess) return 1;

@@ -51,8 +51,6 @@ struct DecodeArgs {
     // the caller guarantees no kernel ahead on the stream writes the cache: the first
     // K/V tiles may be requested before the wait on the previous kernel
     int kv_early;
-    // form (c): the per-token scales and ranks come by TMA (maps 4-6 are valid)
-    int tok_tma;
 };
 
 // cudaLaunchKernelEx with the programmatic-stream-serialization attribute when `pdl`

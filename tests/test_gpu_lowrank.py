@@ -78,12 +78,12 @@ def oracle_lowrank(cfg, inp, packed):
     return ref.decode(cfg.layer_map, ref.bf16_bits_to_f64(inp["q"]), lambda n, i: arrs[n][i])
 
 
-# contexts that are multiples of 16 take the path where per-token scales and ranks
-# arrive by TMA with each tile (208: a half-empty last tile of 32); the others load them per lane
+# ragged and aligned contexts: 1, 17, 129, 300 tokens; 64 and 512 (whole 32-token tiles);
+# 208 (a half-empty last tile)
 SMALL = [lr_cfg("dw_small", 4, 8, 2, 128, 2, 300), lr_cfg("dw_d64_g16", 2, 16, 1, 64, 1, 129),
          lr_cfg("dw_t1", 2, 4, 4, 128, 3, 1), lr_cfg("dw_t17_g1", 2, 2, 2, 64, 1, 17),
-         lr_cfg("dw_t512_tma", 2, 8, 2, 128, 2, 512), lr_cfg("dw_t208_tma", 2, 8, 2, 128, 1, 208),
-         lr_cfg("dw_t64_g16_tma", 2, 16, 1, 64, 1, 64)]
+         lr_cfg("dw_t512", 2, 8, 2, 128, 2, 512), lr_cfg("dw_t208", 2, 8, 2, 128, 1, 208),
+         lr_cfg("dw_t64_g16", 2, 16, 1, 64, 1, 64)]
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
