@@ -37,8 +37,13 @@ from synth.configs import BY_NAME, LOWRANK, MIX  # noqa: E402
 METRIC = "decode tok/s and KV GB/s (% of HBM peak); prefill TFLOP/s, 1×B200"
 
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel,
-# for the kernel as currently built (None until captured for this build)
-NCU_TRAFFIC_BYTES = {"cla2_1p1b": None}
+# for the kernel as currently built (None until captured for this build): mean over the
+# 22 launches of one replayed step, captured without cache control
+# (ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
+#  --cache-control none --clock-control none -k regex:decode_bf16 -s 88 -c 22
+#  python bench.py --steps 1 --warmup 3 --no-secondary --no-cpu-baseline):
+# 67,254,575 B read + 1,409,990 B written
+NCU_TRAFFIC_BYTES = {"cla2_1p1b": 68664565}
 
 
 def load_peaks():
