@@ -15,7 +15,7 @@
 //                 that the tensor core computes one tile's product while the other
 //                 tile's softmax runs:  S = Q K^T  (A, B from shared memory)
 //                                       O += P V  (A = P straight from TMEM, B = V from shared)
-//   warpgroup 2   (two-source layers only) mixers: K~ = w K1 + (1-w) K2 and the
+//   warpgroups 2, 3 (two-source layers only) mixers: K~ = w K1 + (1-w) K2 and the
 //                 same for V, in fp32, rounded once to bf16, written in place over
 //                 the first source's tile, so the MMA reads the mixed operand and
 //                 the mixed K/V never reach HBM ("DepthGraft: Structural
@@ -46,17 +46,18 @@ struct PfCfg {
     static constexpr int STAGE = 2 * NSRC * TILE;
     static constexpr int SMEM = NQ * Q_BYTES + NS * STAGE + 1024;
     static constexpr uint32_t TMEM_COLS = 512;     // S0 | S1 | O0 | O1
-    // warpgroups: 0, 1 softmax; MIX: 2 mixers, 3 TMA + MMA (+2 idle); single: 2 TMA + MMA (+2 idle)
-    static constexpr int THREADS = MIX ? 512 : 384;
+    // warpgroups: 0, 1 softmax; MIX: 2, 3 mixers, 4 TMA + MMA (+2 idle); single: 2 TMA + MMA (+2 idle)
+    static constexpr int MIXERS = 256;                      // mixer threads (two warpgroups)
+    static constexpr int THREADS = MIX ? 640 : 384;
     static constexpr int W_MIX = 8;
-    static constexpr int W_TMA = MIX ? 12 : 8, W_MMA = W_TMA + 1;
+    static constexpr int W_TMA = MIX ? 16 : 8, W_MMA = W_TMA + 1;
     // per-thread registers after the split (setmaxnreg): the softmax threads hold a whole
     // S row; the sum over the block must not exceed what the block was launched with
-    static constexpr int LAUNCH_REGS = MIX ? 128 : 168;
-    static constexpr int REG_SOFTMAX = MIX ? 192 : 224;
-    static constexpr int REG_MIXER = 64;
-    static constexpr int REG_CTRL = 56;
-    static constexpr int REG_SUM = 2 * 128 * REG_SOFTMAX + (MIX ? 128 * REG_MIXER : 0) + 128 * REG_CTRL;
+    static constexpr int LAUNCH_REGS = MIX ? 96 : 168;
+    static constexpr int REG_SOFTMAX = MIX ? 160 : 224;
+    static constexpr int REG_MIXER = 48;
+    static constexpr int REG_CTRL = MIX ? 48 : 56;
+    static constexpr int REG_SUM = 2 * 128 * REG_SOFTMAX + (MIX ? MIXERS * REG_MIXER : 0) + 128 * REG_CTRL;
     static_assert(REG_SUM <= THREADS * LAUNCH_REGS, "register split exceeds the launch allocation");
     static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
 };
@@ -154,7 +155,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mbar_init(&sy.q_full, 1);
         for (int s = 0; s < NS; ++s) {
             mbar_init(&sy.kv_full[s], 1);
-            mbar_init(&sy.kv_ready[s], 128);
+            mbar_init(&sy.kv_ready[s], C::MIXERS);
             mbar_init(&sy.kv_empty[s], 1);
         }
         for (int i = 0; i < NQ; ++i) {
@@ -314,7 +315,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 bulk_wait_read0();
             }
         }
-    } else if (MIX && wg == C::W_MIX / 4) {
+    } else if (MIX && wg >= C::W_MIX / 4 && wg < C::W_MIX / 4 + C::MIXERS / 128) {
         tc::reg_dec<C::REG_MIXER>();
         // ------------------------------------------------------------ mixers (two-source layers)
         const int t = threadIdx.x - 32 * C::W_MIX;
@@ -325,15 +326,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             wait_cta(sy, &sy.kv_full[s], (j / NS) & 1, a.wait_limit, a.err);
             uint4* dst = reinterpret_cast<uint4*>(sKV + s * C::STAGE);                          // K1 | V1
             const uint4* src = reinterpret_cast<const uint4*>(sKV + s * C::STAGE + 2 * C::TILE);   // K2 | V2
-            for (int idx = t; idx < 2 * C::TILE / 16; idx += 128) {
-                const uint4 x = dst[idx];
-                const uint4 y = src[idx];
-                uint4 r;
-                r.x = pack_bf16(w * bf16_lo(x.x) + w1 * bf16_lo(y.x), w * bf16_hi(x.x) + w1 * bf16_hi(y.x));
-                r.y = pack_bf16(w * bf16_lo(x.y) + w1 * bf16_lo(y.y), w * bf16_hi(x.y) + w1 * bf16_hi(y.y));
-                r.z = pack_bf16(w * bf16_lo(x.z) + w1 * bf16_lo(y.z), w * bf16_hi(x.z) + w1 * bf16_hi(y.z));
-                r.w = pack_bf16(w * bf16_lo(x.w) + w1 * bf16_lo(y.w), w * bf16_hi(x.w) + w1 * bf16_hi(y.w));
-                dst[idx] = r;
+            // 16-B chunks of K1|V1 and K2|V2, four per thread in flight before any is mixed
+            constexpr int NIT = 2 * C::TILE / 16 / C::MIXERS;
+            static_assert(NIT % 4 == 0, "mixer batches");
+#pragma unroll
+            for (int it0 = 0; it0 < NIT; it0 += 4) {
+                uint4 x[4], y[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    x[u] = dst[t + (it0 + u) * C::MIXERS];
+                    y[u] = src[t + (it0 + u) * C::MIXERS];
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint4 r;
+                    r.x = pack_bf16(w * bf16_lo(x[u].x) + w1 * bf16_lo(y[u].x), w * bf16_hi(x[u].x) + w1 * bf16_hi(y[u].x));
+                    r.y = pack_bf16(w * bf16_lo(x[u].y) + w1 * bf16_lo(y[u].y), w * bf16_hi(x[u].y) + w1 * bf16_hi(y[u].y));
+                    r.z = pack_bf16(w * bf16_lo(x[u].z) + w1 * bf16_lo(y[u].z), w * bf16_hi(x[u].z) + w1 * bf16_hi(y[u].z));
+                    r.w = pack_bf16(w * bf16_lo(x[u].w) + w1 * bf16_lo(y[u].w), w * bf16_hi(x[u].w) + w1 * bf16_hi(y[u].w));
+                    dst[t + (it0 + u) * C::MIXERS] = r;
+                }
             }
             fence_proxy_async();
             mbar_arrive(&sy.kv_ready[s]);
