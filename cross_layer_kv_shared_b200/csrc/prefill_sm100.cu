@@ -9,8 +9,10 @@
 //                 in TMEM only when a row max grows by more than 2^8), P as bf16
 //                 written back over the row's S columns; epilogue O / l -> bf16
 //                 through shared memory and a TMA store
-//   last warpgroup  one warp TMA producer (Q0, Q1 once, then K/V tiles into a
-//                 2-stage ring), one warp TMEM owner and MMA issuer (one thread),
+//   last warpgroup  one warp TMA producer (Q0, Q1 once, then K/V tiles: a 2-stage
+//                 ring; two-source layers: a 3-stage ring for the first source and a
+//                 2-stage ring for the second, which the mixers free as soon as they
+//                 have read it), one warp TMEM owner and MMA issuer (one thread),
 //                 in the order S0_j, S1_j, PV0_j, S0_{j+1}, PV1_j, S1_{j+1}, ... so
 //                 that the tensor core computes one tile's product while the other
 //                 tile's softmax runs:  S = Q K^T  (A, B from shared memory)
@@ -33,7 +35,7 @@ namespace {
 
 constexpr int BM = 128;   // rows per query tile
 constexpr int NQ = 2;     // query tiles per CTA
-constexpr int NS = 2;     // K/V stages
+constexpr int NS_MAX = 3;   // K/V stages of the first-source ring, at most
 
 template <int D, bool MIX>
 struct PfCfg {
@@ -43,8 +45,15 @@ struct PfCfg {
     static constexpr int Q_BYTES = BM * D * 2;     // one query tile
     static constexpr int TILE = BN * D * 2;        // one K or V tile
     static constexpr int HALF_T = BN * 128;        // one 64-column half of it
-    static constexpr int STAGE = 2 * NSRC * TILE;
-    static constexpr int SMEM = NQ * Q_BYTES + NS * STAGE + 1024;
+    // ring A: [K | V] (the first source, mixed in place on two-source layers), NS stages;
+    // ring B (two-source layers): [K2 | V2], NSB stages, freed by the mixers as soon as
+    // they have read it, so the copies of the second source run ahead of the MMA
+    static constexpr int NS = MIX ? 3 : 2;
+    static constexpr int NSB = MIX ? 2 : 0;
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int SMEM = NQ * Q_BYTES + (NS + NSB) * STAGE + 1024;
+    static_assert(NS <= NS_MAX, "ring A depth");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
     static constexpr uint32_t TMEM_COLS = 512;     // S0 | S1 | O0 | O1
     // warpgroups: 0, 1 softmax; MIX: 2, 3 mixers, 4 TMA + MMA (+2 idle); single: 2 TMA + MMA (+2 idle)
     static constexpr int MIXERS = 256;                      // mixer threads (two warpgroups)
@@ -54,8 +63,8 @@ struct PfCfg {
     // per-thread registers after the split (setmaxnreg): the softmax threads hold a whole
     // S row; the sum over the block must not exceed what the block was launched with
     static constexpr int LAUNCH_REGS = MIX ? 96 : 168;
-    static constexpr int REG_SOFTMAX = MIX ? 160 : 224;
-    static constexpr int REG_MIXER = 48;
+    static constexpr int REG_SOFTMAX = MIX ? 152 : 224;
+    static constexpr int REG_MIXER = 56;
     static constexpr int REG_CTRL = MIX ? 48 : 56;
     static constexpr int REG_SUM = 2 * 128 * REG_SOFTMAX + (MIX ? MIXERS * REG_MIXER : 0) + 128 * REG_CTRL;
     static_assert(REG_SUM <= THREADS * LAUNCH_REGS, "register split exceeds the launch allocation");
@@ -64,9 +73,11 @@ struct PfCfg {
 
 struct Sync {
     uint64_t q_full;
-    uint64_t kv_full[NS];
-    uint64_t kv_ready[NS];
-    uint64_t kv_empty[NS];
+    uint64_t kv_full[NS_MAX];
+    uint64_t kv_ready[NS_MAX];
+    uint64_t kv_empty[NS_MAX];
+    uint64_t kvb_full[2];
+    uint64_t kvb_empty[2];
     uint64_t s_full[NQ];
     uint64_t p_full[NQ];
     uint64_t o_full;
@@ -131,7 +142,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;                                  // [NQ][HALVES][BM][64]
-    uint8_t* sKV = smem + NQ * C::Q_BYTES;               // [NS][K1 | V1 (| K2 | V2)]
+    uint8_t* sKV = smem + NQ * C::Q_BYTES;               // ring A [NS][K | V]
+    uint8_t* sKV2 = sKV + C::NS * C::STAGE;              // ring B [NSB][K2 | V2] (two-source layers)
+    constexpr int NS = C::NS;
+    constexpr int NSB = C::NSB;
     __shared__ __align__(8) Sync sy;
 
     const int warp = threadIdx.x >> 5;
@@ -153,6 +167,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         prefetch_tmap(&tmV);
         prefetch_tmap(&tmO);
         mbar_init(&sy.q_full, 1);
+        for (int s = 0; s < NSB; ++s) {
+            mbar_init(&sy.kvb_full[s], 1);
+            mbar_init(&sy.kvb_empty[s], C::MIXERS);
+        }
         for (int s = 0; s < NS; ++s) {
             mbar_init(&sy.kv_full[s], 1);
             mbar_init(&sy.kv_ready[s], C::MIXERS);
@@ -323,9 +341,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const float w1 = 1.f - w;
         for (int j = 0; j < n_kv; ++j) {
             const int s = j % NS;
+            const int sb = j % (NSB > 0 ? NSB : 1);
             wait_cta(sy, &sy.kv_full[s], (j / NS) & 1, a.wait_limit, a.err);
-            uint4* dst = reinterpret_cast<uint4*>(sKV + s * C::STAGE);                          // K1 | V1
-            const uint4* src = reinterpret_cast<const uint4*>(sKV + s * C::STAGE + 2 * C::TILE);   // K2 | V2
+            wait_cta(sy, &sy.kvb_full[sb], (j / (NSB > 0 ? NSB : 1)) & 1, a.wait_limit, a.err);
+            uint4* dst = reinterpret_cast<uint4*>(sKV + s * C::STAGE);                    // K1 | V1
+            const uint4* src = reinterpret_cast<const uint4*>(sKV2 + sb * C::STAGE);     // K2 | V2
             // 16-B chunks of K1|V1 and K2|V2, four per thread in flight before any is mixed
             constexpr int NIT = 2 * C::TILE / 16 / C::MIXERS;
             static_assert(NIT % 4 == 0, "mixer batches");
@@ -349,6 +369,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             }
             fence_proxy_async();
             mbar_arrive(&sy.kv_ready[s]);
+            mbar_arrive(&sy.kvb_empty[sb]);   // ring B slot read: the next copy may land
         }
     } else {
         tc::reg_dec<C::REG_CTRL>();
@@ -367,6 +388,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 const int r1 = a.src1 * BH + b * a.Hkv + jkv;
                 for (int j = 0; j < n_kv; ++j) {
                     const int s = j % NS;
+                    if (MIX) {
+                        // the second source first: its ring is freed by the mixers, not the MMA
+                        const int sb = j % NSB;
+                        if (j >= NSB) wait_cta(sy, &sy.kvb_empty[sb], ((j / NSB) - 1) & 1, a.wait_limit, a.err);
+                        if (sy.abort) break;
+                        uint8_t* st2 = sKV2 + sb * C::STAGE;
+                        mbar_arrive_expect_tx(&sy.kvb_full[sb], C::STAGE);
+#pragma unroll
+                        for (int hh = 0; hh < C::HALVES; ++hh) {
+                            tma_load_3d(st2 + hh * C::HALF_T, &tmK, hh * 64, j * BN, r1, &sy.kvb_full[sb]);
+                            tma_load_3d(st2 + C::TILE + hh * C::HALF_T, &tmV, hh * 64, j * BN, r1, &sy.kvb_full[sb]);
+                        }
+                    }
                     if (j >= NS) wait_cta(sy, &sy.kv_empty[s], ((j / NS) - 1) & 1, a.wait_limit, a.err);
                     if (sy.abort) break;
                     uint8_t* st = sKV + s * C::STAGE;
@@ -375,10 +409,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     for (int hh = 0; hh < C::HALVES; ++hh) {
                         tma_load_3d(st + hh * C::HALF_T, &tmK, hh * 64, j * BN, r0, &sy.kv_full[s]);
                         tma_load_3d(st + C::TILE + hh * C::HALF_T, &tmV, hh * 64, j * BN, r0, &sy.kv_full[s]);
-                        if (MIX) {
-                            tma_load_3d(st + 2 * C::TILE + hh * C::HALF_T, &tmK, hh * 64, j * BN, r1, &sy.kv_full[s]);
-                            tma_load_3d(st + 3 * C::TILE + hh * C::HALF_T, &tmV, hh * 64, j * BN, r1, &sy.kv_full[s]);
-                        }
                     }
                 }
                 if (sy.abort) {
@@ -387,6 +417,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     for (int j = first; j < n_kv; ++j) {
                         const long long t0 = clock64();
                         while (!mbar_try_wait(&sy.kv_full[j % NS], (j / NS) & 1) && clock64() - t0 < a.wait_limit) {
+                        }
+                    }
+                    if (MIX) {
+                        const int firstb = n_kv > NSB ? n_kv - NSB : 0;
+                        for (int j = firstb; j < n_kv; ++j) {
+                            const long long t0 = clock64();
+                            while (!mbar_try_wait(&sy.kvb_full[j % NSB], (j / NSB) & 1) &&
+                                   clock64() - t0 < a.wait_limit) {
+                            }
                         }
                     }
                 }
