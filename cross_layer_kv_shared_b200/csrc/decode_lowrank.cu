@@ -266,19 +266,20 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
 
     // per-token scales and ranks of a tile, loaded by the lanes (tokens lane, lane+32, ...)
     constexpr int TPL = TT / 32;
-    float pf_sk[TPL], pf_sv[TPL];
-    int pf_r[TPL];
+    // raw 16-bit scales and 8-bit ranks: converted only when published, a tile later, so
+    // nothing waits on these loads until then
+    unsigned pf_sk[TPL], pf_sv[TPL], pf_r[TPL];
     auto prefetch = [&](int k) {
         const int t0 = (tile0 + warp + k * NW) * TT;
 #pragma unroll
         for (int u = 0; u < TPL; ++u) {
             const int t = t0 + lane + 32 * u;
             if (t < a.T) {
-                pf_sk[u] = __half2float(__ushort_as_half(__ldg(a.s_k + tokrow + t)));
-                pf_sv[u] = __half2float(__ushort_as_half(__ldg(a.s_v + tokrow + t)));
-                pf_r[u] = static_cast<int>(__ldg(rank_row + t));
+                pf_sk[u] = __ldg(a.s_k + tokrow + t);
+                pf_sv[u] = __ldg(a.s_v + tokrow + t);
+                pf_r[u] = __ldg(rank_row + t);
             } else {
-                pf_sk[u] = 0.f; pf_sv[u] = 0.f; pf_r[u] = 0;
+                pf_sk[u] = 0u; pf_sv[u] = 0u; pf_r[u] = 0u;
             }
         }
     };
@@ -294,9 +295,9 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         __syncwarp();
 #pragma unroll
         for (int u = 0; u < TPL; ++u) {
-            tks[lane + 32 * u] = pf_sk[u];
-            tks[TT + lane + 32 * u] = pf_sv[u];
-            tkr[lane + 32 * u] = pf_r[u];
+            tks[lane + 32 * u] = __half2float(__ushort_as_half(static_cast<unsigned short>(pf_sk[u])));
+            tks[TT + lane + 32 * u] = __half2float(__ushort_as_half(static_cast<unsigned short>(pf_sv[u])));
+            tkr[lane + 32 * u] = static_cast<int>(pf_r[u]);
         }
         if (k + 1 < my_n) prefetch(k + 1);
         __syncwarp();
