@@ -416,12 +416,11 @@ cudaError_t launch_nh(const CUtensorMap& tmK, const CUtensorMap& tmV, const Deco
     using C = DecodeCfg<D, MIX, TT, NSW, NW>;
     auto kern = decode_bf16_kernel<D, MIX, TT, NSW, NW, NH, STRADDLE>;
     constexpr int smem = STRADDLE ? C::SMEM : C::SMEM_ALIGNED;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = once_per_device(attr_done, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (e != cudaSuccess) return e;
     return launch_kernel(kern, dim3(a.splits), dim3(NW * 32), smem, st, a.pdl != 0, tmK, tmV, a);
 }
 

@@ -538,12 +538,11 @@ template <int D, int RB, int TT, int NSW, int NW, int NH>
 cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
     using C = LrCfg<D, RB, TT, NSW, NW>;
     auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, NH>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = once_per_device(attr_done, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    });
+    if (e != cudaSuccess) return e;
     dim3 grid(a.splits, a.Hkv, a.B);
     return launch_kernel(kern, grid, dim3(NW * 32), C::SMEM, st, a.pdl != 0, maps[0], maps[1], maps[2], maps[3], a);
 }

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace kvs {
 
 // bits of the device status word
@@ -52,6 +54,21 @@ struct DecodeArgs {
     // K/V tiles may be requested before the wait on the previous kernel
     int kv_early;
 };
+
+// One-time set-up of a kernel on the current device (the dynamic shared-memory limit is
+// a per-device function attribute): `setup()` runs the first time this kernel is
+// launched on each device; `done` is the kernel's own device bit mask.
+template <typename Setup>
+inline cudaError_t once_per_device(std::atomic<unsigned long long>& done, Setup setup) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    e = setup();
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 // cudaLaunchKernelEx with the programmatic-stream-serialization attribute when `pdl`
 template <typename... KArgs, typename... Args>

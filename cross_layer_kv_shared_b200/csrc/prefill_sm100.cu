@@ -493,18 +493,18 @@ cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        const PrefillArgs& a, cudaStream_t st) {
     using C = PfCfg<D, MIX>;
     auto kern = prefill_kernel<D, MIX>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return e;
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = once_per_device(attr_done, [&] {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (r != cudaSuccess) return r;
         // the register split assumes the block is launched with LAUNCH_REGS per thread;
         // with fewer, the softmax warps' setmaxnreg.inc could never be satisfied
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, kern);
-        if (e != cudaSuccess) return e;
-        if (fa.numRegs * C::THREADS < C::REG_SUM) return cudaErrorInvalidConfiguration;
-        attr_done = true;
-    }
+        r = cudaFuncGetAttributes(&fa, kern);
+        if (r != cudaSuccess) return r;
+        return fa.numRegs * C::THREADS < C::REG_SUM ? cudaErrorInvalidConfiguration : cudaSuccess;
+    });
+    if (e != cudaSuccess) return e;
     dim3 grid(a.Hq, a.B, (a.S + NQ * BM - 1) / (NQ * BM));
     kern<<<grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, to, a);
     return cudaGetLastError();
