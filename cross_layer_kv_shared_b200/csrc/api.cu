@@ -96,6 +96,12 @@ struct kvshare_ctx {
     void* q_stage = nullptr;
     float* out_stage = nullptr;
     float* lse_stage = nullptr;
+    // kvshare_decode_host: copy streams (host to device, device to host) and events that
+    // pipeline chunks of layers (copies of one chunk under the decode of another)
+    static constexpr int HOST_CHUNKS = 8;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_done = nullptr;
+    cudaEvent_t ev_in[HOST_CHUNKS] = {}, ev_out[HOST_CHUNKS] = {};
 };
 
 namespace {
@@ -400,6 +406,14 @@ kvshare_status kvshare_destroy(kvshare_t ctx) {
     cudaFree(ctx->q_stage);
     cudaFree(ctx->out_stage);
     cudaFree(ctx->lse_stage);
+    if (ctx->h2d != nullptr) cudaStreamDestroy(ctx->h2d);
+    if (ctx->d2h != nullptr) cudaStreamDestroy(ctx->d2h);
+    for (cudaEvent_t ev : {ctx->ev_start, ctx->ev_done})
+        if (ev != nullptr) cudaEventDestroy(ev);
+    for (int c = 0; c < kvshare_ctx::HOST_CHUNKS; ++c) {
+        if (ctx->ev_in[c] != nullptr) cudaEventDestroy(ctx->ev_in[c]);
+        if (ctx->ev_out[c] != nullptr) cudaEventDestroy(ctx->ev_out[c]);
+    }
     cudaSetDevice(prev);
     delete ctx;
     return KVS_OK;
@@ -468,22 +482,59 @@ kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, co
             return KVS_ENOMEM;
         }
     }
+    if (ctx->h2d == nullptr) {
+        bool ok = cudaStreamCreateWithFlags(&ctx->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&ctx->d2h, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&ctx->ev_start, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&ctx->ev_done, cudaEventDisableTiming) == cudaSuccess;
+        for (int c = 0; ok && c < kvshare_ctx::HOST_CHUNKS; ++c)
+            ok = cudaEventCreateWithFlags(&ctx->ev_in[c], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&ctx->ev_out[c], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            cudaGetLastError();
+            return KVS_ECUDA;
+        }
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t lay = static_cast<size_t>(cache->batch) * cf.num_q_heads * cf.head_dim;   // elements per layer
     const size_t layh = static_cast<size_t>(cache->batch) * cf.num_q_heads;
-    const size_t nl = static_cast<size_t>(l1 - l0);
+    const int nl = l1 - l0;
     if (nl == 0) return KVS_OK;
-    cudaError_t e = cudaMemcpyAsync(static_cast<char*>(ctx->q_stage) + l0 * lay * es,
-                                    static_cast<const char*>(q_host) + l0 * lay * es, nl * lay * es,
-                                    cudaMemcpyHostToDevice, st);
+    // Chunks of layers: chunk c's q is copied in on h2d while earlier chunks decode on
+    // `stream`, and its outputs are copied out on d2h while later chunks decode. The
+    // copy streams first wait for work already on `stream` (an earlier call may still be
+    // using the staging buffers), and `stream` waits for the last copy out, so the call
+    // is ordered on `stream` exactly like one that ran everything there.
+    const int nch = nl < kvshare_ctx::HOST_CHUNKS ? nl : kvshare_ctx::HOST_CHUNKS;
+    auto chunk_begin = [&](int c) { return l0 + static_cast<int>((static_cast<long long>(nl) * c) / nch); };
+    cudaError_t e = cudaEventRecord(ctx->ev_start, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->h2d, ctx->ev_start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->d2h, ctx->ev_start, 0);
+    for (int c = 0; c < nch && e == cudaSuccess; ++c) {
+        const size_t a = chunk_begin(c), n = chunk_begin(c + 1) - a;
+        e = cudaMemcpyAsync(static_cast<char*>(ctx->q_stage) + a * lay * es,
+                            static_cast<const char*>(q_host) + a * lay * es, n * lay * es, cudaMemcpyHostToDevice,
+                            ctx->h2d);
+        if (e == cudaSuccess) e = cudaEventRecord(ctx->ev_in[c], ctx->h2d);
+    }
     if (e != cudaSuccess) return KVS_ECUDA;
-    s = decode_layers(ctx, cache, ctx->q_stage, ctx->out_stage, lse_host ? ctx->lse_stage : nullptr, l0, l1, st);
-    if (s != KVS_OK) return s;
-    e = cudaMemcpyAsync(out_host + l0 * lay, ctx->out_stage + l0 * lay, nl * lay * sizeof(float),
-                        cudaMemcpyDeviceToHost, st);
-    if (e == cudaSuccess && lse_host != nullptr)
-        e = cudaMemcpyAsync(lse_host + l0 * layh, ctx->lse_stage + l0 * layh, nl * layh * sizeof(float),
-                            cudaMemcpyDeviceToHost, st);
+    for (int c = 0; c < nch; ++c) {
+        const int a = chunk_begin(c), b = chunk_begin(c + 1);
+        if (cudaStreamWaitEvent(st, ctx->ev_in[c], 0) != cudaSuccess) return KVS_ECUDA;
+        s = decode_layers(ctx, cache, ctx->q_stage, ctx->out_stage, lse_host ? ctx->lse_stage : nullptr, a, b, st);
+        if (s != KVS_OK) return s;
+        e = cudaEventRecord(ctx->ev_out[c], st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->d2h, ctx->ev_out[c], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(out_host + a * lay, ctx->out_stage + a * lay, (b - a) * lay * sizeof(float),
+                                cudaMemcpyDeviceToHost, ctx->d2h);
+        if (e == cudaSuccess && lse_host != nullptr)
+            e = cudaMemcpyAsync(lse_host + a * layh, ctx->lse_stage + a * layh, (b - a) * layh * sizeof(float),
+                                cudaMemcpyDeviceToHost, ctx->d2h);
+        if (e != cudaSuccess) return KVS_ECUDA;
+    }
+    e = cudaEventRecord(ctx->ev_done, ctx->d2h);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ctx->ev_done, 0);
     return cuda_status(e);
 }
 

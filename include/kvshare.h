@@ -142,7 +142,12 @@ kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const v
  * out/lse of those layers back to `out_host`/`lse_host` (same layouts as
  * kvshare_decode, host memory; pinned memory makes the copies asynchronous).
  * The cache stays on the device. Results are valid after the stream has
- * synchronised. The staging buffers are allocated on the first call and reused. */
+ * synchronised. The staging buffers, two copy streams and their events are
+ * created on the first call and reused: the layers run in up to 8 chunks, each
+ * chunk's q copied in on one copy stream while earlier chunks decode on
+ * `stream`, its outputs copied out on the other while later chunks decode. The
+ * copy streams wait for work already on `stream` first, and `stream` waits for
+ * the last copy out, so the call is ordered on `stream` like a serial one. */
 kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, const void* q_host,
                                    float* out_host, float* lse_host, int l0, int l1, void* stream);
 
