@@ -367,20 +367,28 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     const float* save_ml = save + NW * 16 * D;
     for (int uu = u_first; uu <= u_last && span > 0; ++uu) {
         const int u = uu;
-        // the warps' contributions to unit u: final states, and states saved at a unit switch
+        // the warps' contributions to unit u: final states, and states saved at a unit switch;
+        // one weight 2^(m_w - M) per (warp, head), so the vector combine is FMAs only
+        __shared__ float fac_f[NW][16], fac_s[NW][16];
         if (threadIdx.x < g) {
             const int h = threadIdx.x;
             float M = NEG_INF;
             for (int ww = 0; ww < NW; ++ww) {
                 if (fin_unit[ww] == u) M = fmaxf(M, comb_ml[ww * 32 + h]);
-                if (sav_unit[ww] == u) M = fmaxf(M, save_ml[ww * 32 + h]);
+                if (STRADDLE && sav_unit[ww] == u) M = fmaxf(M, save_ml[ww * 32 + h]);
             }
             float L = 0.f;
             for (int ww = 0; ww < NW; ++ww) {
-                if (fin_unit[ww] == u && comb_ml[ww * 32 + h] != NEG_INF)
-                    L += exp2f(comb_ml[ww * 32 + h] - M) * comb_ml[ww * 32 + 16 + h];
-                if (sav_unit[ww] == u && save_ml[ww * 32 + h] != NEG_INF)
-                    L += exp2f(save_ml[ww * 32 + h] - M) * save_ml[ww * 32 + 16 + h];
+                const float mf = comb_ml[ww * 32 + h];
+                const float ff = (fin_unit[ww] == u && mf != NEG_INF) ? ex2_approx(mf - M) : 0.f;
+                fac_f[ww][h] = ff;
+                L += ff * comb_ml[ww * 32 + 16 + h];
+                if (STRADDLE) {
+                    const float ms = save_ml[ww * 32 + h];
+                    const float fs = (sav_unit[ww] == u && ms != NEG_INF) ? ex2_approx(ms - M) : 0.f;
+                    fac_s[ww][h] = fs;
+                    L += fs * save_ml[ww * 32 + 16 + h];
+                }
             }
             fin_m[h] = M;
             fin_l[h] = L;
@@ -392,10 +400,13 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             float acc = 0.f;
 #pragma unroll
             for (int ww = 0; ww < NW; ++ww) {
-                if (fin_unit[ww] == u && comb_ml[ww * 32 + h] != NEG_INF)
-                    acc += exp2f(comb_ml[ww * 32 + h] - fin_m[h]) * comb_o[(ww * 16 + h) * D + e];
-                if (sav_unit[ww] == u && save_ml[ww * 32 + h] != NEG_INF)
-                    acc += exp2f(save_ml[ww * 32 + h] - fin_m[h]) * save_o[(ww * 16 + h) * D + e];
+                // a warp without a state for u left whatever its slot held: skip it, never 0 * x
+                const float ff = fac_f[ww][h];
+                if (ff != 0.f) acc = fmaf(ff, comb_o[(ww * 16 + h) * D + e], acc);
+                if (STRADDLE) {
+                    const float fs = fac_s[ww][h];
+                    if (fs != 0.f) acc = fmaf(fs, save_o[(ww * 16 + h) * D + e], acc);
+                }
             }
             fin_o[idx] = acc;
         }

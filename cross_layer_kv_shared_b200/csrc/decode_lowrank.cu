@@ -503,13 +503,19 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         }
     }
     __syncthreads();
+    // one weight 2^(m_w - M) per (warp, head), so the vector combine is FMAs only
+    __shared__ float fac[NW][16];
     if (threadIdx.x < g) {
         const int h = threadIdx.x;
         float M = NEG_INF;
         for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, comb_m[ww * 16 + h]);
         float L = 0.f;
-        for (int ww = 0; ww < NW; ++ww)
-            if (comb_m[ww * 16 + h] != NEG_INF) L += exp2f(comb_m[ww * 16 + h] - M) * comb_l[ww * 16 + h];
+        for (int ww = 0; ww < NW; ++ww) {
+            const float m = comb_m[ww * 16 + h];
+            const float f = m != NEG_INF ? ex2_approx(m - M) : 0.f;
+            fac[ww][h] = f;
+            L += f * comb_l[ww * 16 + h];
+        }
         fin_m[h] = M;
         fin_l[h] = L;
     }
@@ -518,9 +524,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         const int h = idx / PD;
         float acc = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww)
-            if (comb_m[ww * 16 + h] != NEG_INF)
-                acc += exp2f(comb_m[ww * 16 + h] - fin_m[h]) * comb[(ww * 16 + h) * PD + (idx % PD)];
+        for (int ww = 0; ww < NW; ++ww) acc = fmaf(fac[ww][h], comb[(ww * 16 + h) * PD + (idx % PD)], acc);
         fin_c[idx] = acc;
     }
     __syncthreads();

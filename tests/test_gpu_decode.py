@@ -98,6 +98,29 @@ def test_grids_whose_ranges_straddle_units(K, cfg, grid):
     assert_close(lse, want_lse, TOL_BF16, "lse")
 
 
+# other sharing topologies the layer table expresses: CLA3 / CLA4 groups reading the
+# lowest layer of each group, a single-anchor map (the upper half reads one slot), and
+# MQA (one kv head) at group sizes 8 and 16
+OTHER_MAPS = [
+    small("cla3", "bf16", 6, [(SINGLE, l // 3, 0) for l in range(6)], 2, 8, 2, 64, 2, 257, 0.125),
+    small("cla4", "bf16", 8, [(SINGLE, l // 4, 0) for l in range(8)], 2, 16, 4, 128, 1, 300),
+    small("single_anchor", "bf16", 6, [(SINGLE, 0, 0), (SINGLE, 1, 0), (SINGLE, 2, 0)] + [(SINGLE, 2, 0)] * 3,
+          3, 8, 2, 64, 2, 200, 0.125),
+    small("mqa_g8", "bf16", 2, [(SINGLE, 0, 0), (SINGLE, 0, 0)], 1, 8, 1, 128, 2, 333),
+    small("mqa_g16", "bf16", 2, [(SINGLE, 0, 0), (MIX, 0, 1)], 2, 16, 1, 64, 1, 129),
+]
+
+
+@pytest.mark.parametrize("cfg", OTHER_MAPS, ids=lambda c: c.name)
+def test_other_sharing_maps_every_output(K, cfg):
+    inp = cfg.make_all()
+    out, lse, launches = decode_gpu(K, cfg, inp)
+    want, want_lse = oracle_decode(cfg, inp)
+    assert_close(out, want, TOL_BF16, "out")
+    assert_close(lse, want_lse, TOL_BF16, "lse")
+    assert launches == cfg.layers
+
+
 @pytest.mark.parametrize("cfg", [CLA_SMALL, DG_SMALL], ids=lambda c: c.name)
 def test_kv_overlap_changes_nothing(K, cfg):
     # consecutive layers of one call overlap; with kv_overlap they also fetch K/V early
