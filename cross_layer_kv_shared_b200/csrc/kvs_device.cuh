@@ -332,7 +332,7 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         M = warp_max(M);
         float L = 0.f;
         for (int sp = lane; sp < n; sp += 32) {
-            const float f = exp2f(fm[sp * g + h] - M);
+            const float f = ex2_approx(fm[sp * g + h] - M);
             fm[sp * g + h] = f;
             L += f * fl[sp * g + h];
         }
