@@ -64,12 +64,14 @@ struct LrCfg {
     static constexpr int COMBINE_FLOATS = NW * 16 * PD + 2 * NW * 16 + 32 + 16 * PD + 16 * D + 2 * MAX_GROUP * MAX_SPLITS + 64;
     static constexpr int MERGE_STAGE_OFF = ((COMBINE_FLOATS * 4 + 1023) / 1024) * 1024;   // free smem for the merge
     static constexpr int QPROJ_FLOATS = 16 * PD;
-    // staging: basis [RB][D] + residual factor [RM][D] (bf16), then the query rows [<=16][D]
+    // staging: B_K [RB][D] + R_K [RM][D] (bf16), the query rows [<=16][D], then B_V + R_V
     static constexpr int STAGE_FACTORS = (RB + RM) * D * 2;
-    static constexpr int STAGE_BYTES_TOTAL = STAGE_FACTORS + 16 * D * 2;
+    static constexpr int OFF_VFAC = STAGE_FACTORS + 16 * D * 2;
+    static constexpr int STAGE_BYTES_TOTAL = OFF_VFAC + STAGE_FACTORS;
     static constexpr int BODY0 = RING_BYTES > COMBINE_FLOATS * 4 ? RING_BYTES : COMBINE_FLOATS * 4;
     static constexpr int SMEM = BODY0 + TOK_BYTES + CVT_BYTES + QPROJ_FLOATS * 4 + STAGE_BYTES_TOTAL + 1024;
     static_assert(TT % 16 == 0 && COEF_BYTES % 1024 == 0, "tile shape");
+    static_assert(SMEM + 4096 <= 227 * 1024, "shared memory (dynamic + the kernel's static arrays)");
 };
 
 // Writes out = (c^ B_V + u^ R_V) / l from the merged coefficient-space sums v [g][RB + 16].
@@ -116,7 +118,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     float* tok = reinterpret_cast<float*>(smem + C::BODY0);                    // [NW][3][TT]: s_K, s_V, rank
     uint8_t* cvt = reinterpret_cast<uint8_t*>(tok + NW * TT * 3);              // [NW][K | V][TT][16] f16
     float* qproj = reinterpret_cast<float*>(cvt + C::CVT_BYTES);               // [16][RB + RM]
-    uint8_t* stagebuf = reinterpret_cast<uint8_t*>(qproj + C::QPROJ_FLOATS);   // factors, then q rows
+    uint8_t* stagebuf = reinterpret_cast<uint8_t*>(qproj + C::QPROJ_FLOATS);   // K factors, q rows, V factors
+    uint8_t* vfac = stagebuf + C::OFF_VFAC;
     __shared__ __align__(8) uint64_t bars[NW * NSW + 1];
     __shared__ __align__(8) uint64_t fac_bar[2];    // [0]: B_K, R_K, q   [1]: B_V, R_V
 
@@ -147,9 +150,6 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         mbar_init_fence();
     }
     __syncthreads();   // every warp's ring barriers are initialised before any warp issues
-    // under a dependent launch everything above overlapped the previous kernel's tail;
-    // global memory (inputs, workspace, counters) is touched only from here on
-    grid_dep_wait();
     uint8_t* ring = smem + warp * NSW * C::STAGE_BYTES;
     uint64_t* wb = &bars[warp * NSW];
     const int span = tile1 - tile0;
@@ -168,55 +168,77 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         tma_load_3d(st + C::OFF_UK, &tmUK, 0, t * TT, urow, &wb[s]);
         tma_load_3d(st + C::OFF_UV, &tmUV, 0, t * TT, urow, &wb[s]);
     };
-    if (threadIdx.x == 0) {
-        grid_dep_launch();
-        // B_K[j], R_K[j] and the group's query rows, by bulk copy (all contiguous, 16-B aligned)
-        mbar_arrive_expect_tx(&fac_bar[0], C::STAGE_FACTORS + g * D * 2);
-        bulk_load(stagebuf, static_cast<const uint16_t*>(a.basis_k) + static_cast<size_t>(j) * RB * D, RB * D * 2,
-                  &fac_bar[0]);
-        bulk_load(stagebuf + RB * D * 2, static_cast<const uint16_t*>(a.r_k) + static_cast<size_t>(j) * RM * D,
-                  RM * D * 2, &fac_bar[0]);
-        bulk_load(stagebuf + C::STAGE_FACTORS, qsrc, g * D * 2, &fac_bar[0]);
-    }
-    // then every warp's first tiles, which stream while the query is projected
-    if (lane == 0) {
-        for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
-    }
-    __syncwarp();
+    // per-token scales and ranks of a tile, loaded by the lanes (tokens lane, lane+32, ...)
+    constexpr int TPL = TT / 32;
+    // raw 16-bit scales and 8-bit ranks: converted only when published, a tile later, so
+    // nothing waits on these loads until then
+    unsigned pf_sk[TPL], pf_sv[TPL], pf_r[TPL];
+    auto prefetch = [&](int k) {
+        const int t0 = (tile0 + warp + k * NW) * TT;
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            const int t = t0 + lane + 32 * u;
+            if (t < a.T) {
+                pf_sk[u] = __ldg(a.s_k + tokrow + t);
+                pf_sv[u] = __ldg(a.s_v + tokrow + t);
+                pf_r[u] = __ldg(rank_row + t);
+            } else {
+                pf_sk[u] = 0u; pf_sv[u] = 0u; pf_r[u] = 0u;
+            }
+        }
+    };
+    // Cache reads only (bases, residual factors, this warp's first tiles and scales).
+    // Under a dependent launch the kernel ahead on the stream may still be running; with
+    // kv_early the caller has promised that it writes none of the cache, so these are
+    // requested before the wait. The query and everything written come after it.
+    auto request_cache = [&] {
+        if (threadIdx.x == 0) {
+            mbar_arrive_expect_tx(&fac_bar[0], C::STAGE_FACTORS + g * D * 2);   // q lands on it too
+            bulk_load(stagebuf, static_cast<const uint16_t*>(a.basis_k) + static_cast<size_t>(j) * RB * D,
+                      RB * D * 2, &fac_bar[0]);
+            bulk_load(stagebuf + RB * D * 2, static_cast<const uint16_t*>(a.r_k) + static_cast<size_t>(j) * RM * D,
+                      RM * D * 2, &fac_bar[0]);
+            mbar_arrive_expect_tx(&fac_bar[1], C::STAGE_FACTORS);
+            bulk_load(vfac, static_cast<const uint16_t*>(a.basis_v) + static_cast<size_t>(j) * RB * D, RB * D * 2,
+                      &fac_bar[1]);
+            bulk_load(vfac + RB * D * 2, static_cast<const uint16_t*>(a.r_v) + static_cast<size_t>(j) * RM * D,
+                      RM * D * 2, &fac_bar[1]);
+        }
+        if (lane == 0) {
+            for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
+        }
+        __syncwarp();
+        if (my_n > 0) prefetch(0);
+    };
+    if (a.kv_early) request_cache();
+    grid_dep_wait();
+    if (threadIdx.x == 0) grid_dep_launch();
+    if (!a.kv_early) request_cache();
+    if (threadIdx.x == 0) bulk_load(stagebuf + C::STAGE_FACTORS, qsrc, g * D * 2, &fac_bar[0]);
     for (int idx = g * C::PD + threadIdx.x; idx < 16 * C::PD; idx += blockDim.x) qproj[idx] = 0.f;
-    __syncthreads();
-    // ---- q~ = B_K q and q^ = R_K q for the g heads: one warp per output, lanes over d
+    // ---- q~ = B_K q and q^ = R_K q for the g heads: one thread per output; lane l starts
+    // its walk over d at pair l, so the 32 lanes of a warp read 32 different banks
     mbar_wait_bounded(&fac_bar[0], 0, a.wait_limit, a.err);
     {
-        const uint16_t* fac = reinterpret_cast<const uint16_t*>(stagebuf);
-        const uint16_t* qs = reinterpret_cast<const uint16_t*>(stagebuf + C::STAGE_FACTORS);
-        for (int idx = warp; idx < g * C::PD; idx += NW) {
-            const int h = idx / C::PD;
-            const int i = idx % C::PD;
-            float acc = 0.f;
-            {
-                const uint16_t* row = fac + static_cast<size_t>(i) * D;     // basis rows, then factor rows
-                for (int e = 2 * lane; e < D; e += 64) {
-                    const uint32_t bw = *reinterpret_cast<const uint32_t*>(row + e);
-                    const uint32_t qw = *reinterpret_cast<const uint32_t*>(qs + h * D + e);
-                    acc += bf16_lo(bw) * bf16_lo(qw) + bf16_hi(bw) * bf16_hi(qw);
-                }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        constexpr int W = D / 2;   // bf16 pairs per row
+        const uint32_t* fac = reinterpret_cast<const uint32_t*>(stagebuf);   // basis rows, then factor rows
+        const uint32_t* qs = reinterpret_cast<const uint32_t*>(stagebuf + C::STAGE_FACTORS);
+        for (int idx = threadIdx.x; idx < g * C::PD; idx += blockDim.x) {
+            const uint32_t* row = fac + (idx % C::PD) * W;
+            const uint32_t* qr = qs + (idx / C::PD) * W;
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+            for (int k = 0; k < W; ++k) {
+                const int w = (k + lane) & (W - 1);
+                const uint32_t bw = row[w];
+                const uint32_t qw = qr[w];
+                acc0 = fmaf(bf16_lo(bw), bf16_lo(qw), acc0);
+                acc1 = fmaf(bf16_hi(bw), bf16_hi(qw), acc1);
             }
-            if (lane == 0) qproj[idx] = acc;
+            qproj[idx] = acc0 + acc1;
         }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        // B_V[j], R_V[j] for the final projection, landing while the tiles stream
-        fence_proxy_async();
-        mbar_arrive_expect_tx(&fac_bar[1], C::STAGE_FACTORS);
-        bulk_load(stagebuf, static_cast<const uint16_t*>(a.basis_v) + static_cast<size_t>(j) * RB * D, RB * D * 2,
-                  &fac_bar[1]);
-        bulk_load(stagebuf + RB * D * 2, static_cast<const uint16_t*>(a.r_v) + static_cast<size_t>(j) * RM * D,
-                  RM * D * 2, &fac_bar[1]);
-    }
     if (a.stall && threadIdx.x == 0) mbar_wait_bounded(&bars[NW * NSW], 0, a.stall_limit, a.err);
 
     // B fragments of q~^T (RB rows, bf16 hi + lo) and q^^T (16 rows, f16: the residual term
@@ -264,27 +286,6 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     // byte offset of the 16-B half `seg` (channels 8 seg .. 8 seg + 7) of token row t
     auto cvt_off = [](int t, int seg) { return static_cast<uint32_t>(t * 32 + ((seg ^ ((t >> 2) & 1)) << 4)); };
 
-    // per-token scales and ranks of a tile, loaded by the lanes (tokens lane, lane+32, ...)
-    constexpr int TPL = TT / 32;
-    // raw 16-bit scales and 8-bit ranks: converted only when published, a tile later, so
-    // nothing waits on these loads until then
-    unsigned pf_sk[TPL], pf_sv[TPL], pf_r[TPL];
-    auto prefetch = [&](int k) {
-        const int t0 = (tile0 + warp + k * NW) * TT;
-#pragma unroll
-        for (int u = 0; u < TPL; ++u) {
-            const int t = t0 + lane + 32 * u;
-            if (t < a.T) {
-                pf_sk[u] = __ldg(a.s_k + tokrow + t);
-                pf_sv[u] = __ldg(a.s_v + tokrow + t);
-                pf_r[u] = __ldg(rank_row + t);
-            } else {
-                pf_sk[u] = 0u; pf_sv[u] = 0u; pf_r[u] = 0u;
-            }
-        }
-    };
-    if (my_n > 0) prefetch(0);
-    __syncwarp();
 
     const int mi = lane >> 3;
     const int ri = lane & 7;
@@ -531,7 +532,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     // partials stay in coefficient space (RB + 16 values per head); the CTA that
     // finishes the unit projects once: o = (c^ B_V + u^ R_V) / l
     mbar_wait_bounded(&fac_bar[1], 0, a.wait_limit, a.err);
-    const uint16_t* Bv = reinterpret_cast<const uint16_t*>(stagebuf);
+    const uint16_t* Bv = reinterpret_cast<const uint16_t*>(vfac);
     const EmitProject<D, RB> emit{a, static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g, Bv, Bv + RB * D};
     const int unit = b * a.Hkv + j;
     finish_unit(a, PD, unit, split, a.splits, static_cast<long long>(unit) * a.splits, fin_m, fin_l, fin_c, scratch,

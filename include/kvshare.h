@@ -187,7 +187,8 @@ kvshare_status kvshare_set_splits(kvshare_t ctx, int splits);
  * start (barrier set-up, tensor-map fetch) while the kernel ahead of it on the
  * stream drains, and waits for that kernel before it reads q or writes anything.
  * With `on` != 0 the bf16 decode also requests its first K/V tiles before that
- * wait. Set it only when no kernel that can still be running when kvshare_decode
+ * wait, and the low-rank decode its bases, residual factors, first coefficient
+ * and code tiles and their per-token scales and ranks. Set it only when no kernel that can still be running when kvshare_decode
  * is called writes the cache regions the call reads (for example: the step's
  * cache appends were made before the kernels ahead of the decode, or the layers
  * decoded read sources nothing is appending to); otherwise a tile could be read

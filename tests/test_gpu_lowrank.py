@@ -47,13 +47,14 @@ def make_ctx(K, cfg):
     return h
 
 
-def run_small(K, cfg, inp=None):
+def run_small(K, cfg, inp=None, kv_overlap=False):
     import torch
     inp = inp or cfg.make_all()
     d = {n: to_dev(a, "bf16") for n, a in inp.items()}
     h = make_ctx(K, cfg)
     try:
         K.kvshare_set_map(h, cfg.layer_map, None)
+        K.kvshare_set_kv_overlap(h, 1 if kv_overlap else 0)
         rank, ck, cv, sk, sv = pack_gpu(K, h, cfg, d["score"], d["u_k"], d["u_v"])
         out = torch.full((cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim), float("nan"), device="cuda")
         lse = torch.full((cfg.layers, cfg.batch, cfg.q_heads), float("nan"), device="cuda")
@@ -147,6 +148,16 @@ def test_full_rank_identity_basis_equals_single_source(K):
     assert_close(out, want, TOL, "identity basis")
 
 
+@pytest.mark.parametrize("cfg", [SMALL[0], SMALL[5]], ids=lambda c: c.name)
+def test_kv_overlap_changes_nothing(K, cfg):
+    # with kv_overlap each layer's launch requests its bases, factors, first tiles and
+    # scales before waiting on the previous layer's kernel; the results are the same bits
+    inp = cfg.make_all()
+    out, lse, _, _ = run_small(K, cfg, inp)
+    out2, lse2, _, _ = run_small(K, cfg, inp, kv_overlap=True)
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+
+
 def test_full_size_sampled(K):
     import torch
     cfg = DEPTHWEAVE_DECODE
@@ -164,8 +175,9 @@ def test_full_size_sampled(K):
         K.kvshare_decode(h, cache, dev["q"], out, lse)
         assert K.kvshare_sync_status(h) == K.KVS_OK
         # the launch configuration bench.py times: per-layer calls in cold order captured
-        # once as a CUDA graph and replayed; same bits as the plain call
+        # once as a CUDA graph and replayed, with kv_overlap; same bits as the plain call
         import bench
+        K.kvshare_set_kv_overlap(h, 1)
         out2 = torch.full_like(out, float("nan"))
         lse2 = torch.full_like(lse, float("nan"))
         order = bench.cold_order(cfg)
