@@ -62,7 +62,6 @@ struct LrCfg {
     static constexpr int CVT_BYTES = NW * 2 * TT * 32;
     static constexpr int PD = RB + RM;    // coefficient-space partial width
     static constexpr int COMBINE_FLOATS = NW * 16 * PD + 2 * NW * 16 + 32 + 16 * PD + 16 * D + 2 * MAX_GROUP * MAX_SPLITS + 64;
-    static constexpr int MERGE_STAGE_OFF = ((COMBINE_FLOATS * 4 + 1023) / 1024) * 1024;   // free smem for the merge
     static constexpr int QPROJ_FLOATS = 16 * PD;
     // staging: B_K [RB][D] + R_K [RM][D] (bf16), the query rows [<=16][D], then B_V + R_V
     static constexpr int STAGE_FACTORS = (RB + RM) * D * 2;
@@ -72,6 +71,7 @@ struct LrCfg {
     static constexpr int SMEM = BODY0 + TOK_BYTES + CVT_BYTES + QPROJ_FLOATS * 4 + STAGE_BYTES_TOTAL + 1024;
     static_assert(TT % 16 == 0 && COEF_BYTES % 1024 == 0, "tile shape");
     static_assert(SMEM + 4096 <= 227 * 1024, "shared memory (dynamic + the kernel's static arrays)");
+    static_assert(BODY0 % 16 == 0, "the split merge stages partials by bulk copy after the body");
 };
 
 // Writes out = (c^ B_V + u^ R_V) / l from the merged coefficient-space sums v [g][RB + 16].
@@ -223,19 +223,32 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         constexpr int W = D / 2;   // bf16 pairs per row
         const uint32_t* fac = reinterpret_cast<const uint32_t*>(stagebuf);   // basis rows, then factor rows
         const uint32_t* qs = reinterpret_cast<const uint32_t*>(stagebuf + C::STAGE_FACTORS);
-        for (int idx = threadIdx.x; idx < g * C::PD; idx += blockDim.x) {
+        // two adjacent lanes per output (each half of d) when the block has the threads
+        const int halves = 2 * g * C::PD <= static_cast<int>(blockDim.x) ? 2 : 1;
+        const int WP = W / halves;
+        const int total = g * C::PD * halves;
+        // whole warps run each pass (the pair sum is a shuffle); lanes past the end idle
+        for (int t = threadIdx.x; t < ((total + 31) & ~31); t += blockDim.x) {
+            const bool valid = t < total;
+            const int idx = valid ? t / halves : 0;
+            const int w0 = (t % halves) * WP;
             const uint32_t* row = fac + (idx % C::PD) * W;
             const uint32_t* qr = qs + (idx / C::PD) * W;
-            float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-            for (int k = 0; k < W; ++k) {
-                const int w = (k + lane) & (W - 1);
-                const uint32_t bw = row[w];
-                const uint32_t qw = qr[w];
-                acc0 = fmaf(bf16_lo(bw), bf16_lo(qw), acc0);
-                acc1 = fmaf(bf16_hi(bw), bf16_hi(qw), acc1);
+            float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll 4
+            for (int k = 0; k < WP; k += 2) {
+                const int wa = w0 + ((k + lane) & (WP - 1));
+                const int wb = w0 + ((k + 1 + lane) & (WP - 1));
+                const uint32_t ba = row[wa], qa = qr[wa];
+                const uint32_t bb = row[wb], qb = qr[wb];
+                acc0 = fmaf(bf16_lo(ba), bf16_lo(qa), acc0);
+                acc1 = fmaf(bf16_hi(ba), bf16_hi(qa), acc1);
+                acc2 = fmaf(bf16_lo(bb), bf16_lo(qb), acc2);
+                acc3 = fmaf(bf16_hi(bb), bf16_hi(qb), acc3);
             }
-            qproj[idx] = acc0 + acc1;
+            float acc = (acc0 + acc1) + (acc2 + acc3);
+            if (halves == 2) acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            if (valid && t % halves == 0) qproj[idx] = acc;
         }
     }
     __syncthreads();
@@ -469,6 +482,9 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         }
 
     // ---- merge warps in coefficient space, project once, finish the split
+    // (the code-conversion buffers, written through the generic proxy in the loop, later
+    // receive the unit's partials by bulk copy)
+    fence_proxy_async();
     __syncthreads();
     constexpr int PD = C::PD;
     float* comb = reinterpret_cast<float*>(smem);   // [NW][16][PD]
@@ -535,8 +551,9 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     const uint16_t* Bv = reinterpret_cast<const uint16_t*>(vfac);
     const EmitProject<D, RB> emit{a, static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g, Bv, Bv + RB * D};
     const int unit = b * a.Hkv + j;
+    // the per-token and code-conversion buffers are free now: they stage the unit's partials
     finish_unit(a, PD, unit, split, a.splits, static_cast<long long>(unit) * a.splits, fin_m, fin_l, fin_c, scratch,
-                smem + C::MERGE_STAGE_OFF, C::BODY0 > C::MERGE_STAGE_OFF ? C::BODY0 - C::MERGE_STAGE_OFF : 0, emit);
+                reinterpret_cast<uint8_t*>(tok), C::TOK_BYTES + C::CVT_BYTES, emit);
 }
 
 template <int D, int RB, int TT, int NSW, int NW, int NH>
