@@ -1,5 +1,6 @@
 // Host side of libkvshare: argument validation, layer-table resolution,
 // split heuristic, TMA descriptors and kernel launches. See include/kvshare.h.
+#include <algorithm>
 #include "kvshare.h"
 
 #include <cuda.h>
@@ -140,7 +141,7 @@ bool get_store_map(kvshare_ctx* c, const void* base, int D, int T, int rows, int
     return get_map(c, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, rows, 64, tt, CU_TENSOR_MAP_SWIZZLE_128B, out);
 }
 
-int choose_splits(const kvshare_ctx* c, int units, int tiles, int ctas_per_sm, int g, int D) {
+int choose_splits(const kvshare_ctx* c, int units, int tiles, int ctas_per_sm, int g, int part_values) {
     int s;
     if (c->splits_override > 0) {
         s = c->splits_override;
@@ -151,8 +152,8 @@ int choose_splits(const kvshare_ctx* c, int units, int tiles, int ctas_per_sm, i
     }
     if (s > tiles) s = tiles;
     if (s > MAX_SPLITS) s = MAX_SPLITS;
-    // workspace capacity: units * splits * g * partial_width(D) floats
-    const size_t per_split = static_cast<size_t>(units) * g * (D + 4);
+    // workspace capacity: units * splits * g * (part_values + 4) floats
+    const size_t per_split = static_cast<size_t>(units) * g * (part_values + 4);
     while (s > 1 && per_split * s > c->ws_floats) --s;
     if (s < 1) s = 1;
     return s;
@@ -237,7 +238,7 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
             int& o = occ_lr[D == 128][Rb == 32 ? 0 : (Rb == 64 ? 1 : 2)];
             if (o == 0) o = decode_lowrank_occupancy(D, Rb);
             const int tiles = (T + tt - 1) / tt;
-            int s = choose_splits(c, B * Hkv, tiles, o, g, D);
+            int s = choose_splits(c, B * Hkv, tiles, o, g, Rb + 16);   // partials of Rb + 16 values
             a.tiles_per_split = (tiles + s - 1) / s;
             a.splits = (tiles + a.tiles_per_split - 1) / a.tiles_per_split;
             const size_t BHT = static_cast<size_t>(B) * Hkv * T;
@@ -372,7 +373,10 @@ kvshare_status kvshare_create(const kvshare_config* cfg, kvshare_t* out) {
     const size_t units = static_cast<size_t>(c.max_batch) * c.num_kv_heads;
     const int max_tiles = (c.max_context + 15) / 16;
     const int ms = max_tiles < MAX_SPLITS ? max_tiles : MAX_SPLITS;
-    ctx->ws_floats = units * ms * g * (c.head_dim + 4);
+    // a split's partial per q head: d values (forms a, b) or Rb + 16 coefficient-space
+    // values (form c), plus m and l, padded to 16 bytes
+    const int part_values = std::max(c.head_dim, ctx->cfg.basis_rank + ctx->cfg.max_resid_rank);
+    ctx->ws_floats = units * ms * g * (part_values + 4);
     ctx->map.assign(c.num_layers, kvshare_layer{KVS_SRC_SINGLE, 0, 0});
     ctx->w_host.assign(static_cast<size_t>(c.num_layers) * c.num_kv_heads, 1.0f);
     if (cudaMalloc(&ctx->ws, ctx->ws_floats * sizeof(float)) != cudaSuccess ||

@@ -47,7 +47,7 @@ def make_ctx(K, cfg):
     return h
 
 
-def run_small(K, cfg, inp=None, kv_overlap=False):
+def run_small(K, cfg, inp=None, kv_overlap=False, splits=0):
     import torch
     inp = inp or cfg.make_all()
     d = {n: to_dev(a, "bf16") for n, a in inp.items()}
@@ -55,6 +55,8 @@ def run_small(K, cfg, inp=None, kv_overlap=False):
     try:
         K.kvshare_set_map(h, cfg.layer_map, None)
         K.kvshare_set_kv_overlap(h, 1 if kv_overlap else 0)
+        if splits:
+            K.kvshare_set_splits(h, splits)
         rank, ck, cv, sk, sv = pack_gpu(K, h, cfg, d["score"], d["u_k"], d["u_v"])
         out = torch.full((cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim), float("nan"), device="cuda")
         lse = torch.full((cfg.layers, cfg.batch, cfg.q_heads), float("nan"), device="cuda")
@@ -146,6 +148,29 @@ def test_full_rank_identity_basis_equals_single_source(K):
     assert np.all(packed[0] == 0)
     want = ref.decode(kvcfg.layer_map, ref.bf16_bits_to_f64(kv["q"]), lambda n, i: ref.bf16_bits_to_f64(kv[n][i]))[0]
     assert_close(out, want, TOL, "identity basis")
+
+
+# g = 16 with more splits than the merge's staging buffer holds partials: the last CTA of
+# a unit reads them in several bulk copies (11 per copy at Rb = 32, one at a time at
+# Rb = 128), instead of the single copy the other tests take
+# (the last case: partials of Rb + 16 = 144 values, more than d = 128, and one unit split
+# 148 ways with one tile each: the workspace must hold 148 partials of that width)
+@pytest.mark.parametrize("cfg,splits", [(lr_cfg("dw_g16_s16", 2, 16, 1, 128, 1, 1024), 16),
+                                        (lr_cfg("dw_rb128_g16_s6", 2, 16, 1, 128, 1, 400, Rb=128), 6),
+                                        (lr_cfg("dw_rb128_t4736_auto", 2, 4, 1, 128, 1, 4736, Rb=128), 0)],
+                         ids=lambda x: getattr(x, "name", str(x)))
+def test_merge_in_several_copies(K, cfg, splits):
+    out, lse, packed, inp = run_small(K, cfg, splits=splits)
+    want = qr.pack_residual(inp["score"], inp["u_k"], inp["u_v"])
+    for got, exp in zip(packed, want):
+        assert np.array_equal(got.view(exp.dtype), exp)
+    o, l = oracle_lowrank(cfg, inp, want)
+    assert_close(out, o, TOL, "out")
+    assert_close(lse, l, TOL, "lse")
+    # P is rounded to bf16 against each split's own running max: the split count moves
+    # the output by at most the bf16 precision of the weights
+    one, _, _, _ = run_small(K, cfg, inp, splits=1)
+    assert np.max(np.abs(out - one)) <= 2.0 ** -8 * np.max(np.abs(one))
 
 
 @pytest.mark.parametrize("cfg", [SMALL[0], SMALL[5]], ids=lambda c: c.name)
