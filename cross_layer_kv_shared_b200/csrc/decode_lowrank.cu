@@ -552,7 +552,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     const EmitProject<D, RB> emit{a, static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g, Bv, Bv + RB * D};
     const int unit = b * a.Hkv + j;
     // the per-token and code-conversion buffers are free now: they stage the unit's partials
-    finish_unit(a, PD, unit, split, a.splits, static_cast<long long>(unit) * a.splits, fin_m, fin_l, fin_c, scratch,
+    finish_unit<(PD > D ? PD : D)>(a, PD, unit, split, a.splits, static_cast<long long>(unit) * a.splits, fin_m, fin_l,
+                                   fin_c, scratch,
                 reinterpret_cast<uint8_t*>(tok), C::TOK_BYTES + C::CVT_BYTES, emit);
 }
 

@@ -253,7 +253,9 @@ struct EmitPlain {
     }
 };
 
-template <typename Emit>
+// MAXDV bounds DV (values per head of a partial): each thread holds up to
+// MAX_GROUP * MAXDV / 128 merged values, as every caller runs at least 128 threads.
+template <int MAXDV = 128, typename Emit>
 __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int index, int count, long long slot0,
                                    const float* sm_m, const float* sm_l, float* sm_v, float* sm_scratch,
                                    uint8_t* stage, int stage_bytes, const Emit& emit) {
@@ -343,7 +345,7 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         }
     }
     __syncthreads();
-    constexpr int MAXO = (MAX_GROUP * 128 + 127) / 128;   // values per thread at >= 128 threads
+    constexpr int MAXO = (MAX_GROUP * MAXDV + 127) / 128;   // values per thread at >= 128 threads
     float acc[MAXO];
 #pragma unroll
     for (int k = 0; k < MAXO; ++k) acc[k] = 0.f;

@@ -165,7 +165,8 @@ def test_merge_in_several_copies(K, cfg, splits):
     for got, exp in zip(packed, want):
         assert np.array_equal(got.view(exp.dtype), exp)
     o, l = oracle_lowrank(cfg, inp, want)
-    assert_close(out, o, TOL, "out")
+    _, rel = assert_close(out, o, TOL, "out")
+    assert rel < 2e-2          # these outputs can be far below O(1): bound the relative error too
     assert_close(lse, l, TOL, "lse")
     # P is rounded to bf16 against each split's own running max: the split count moves
     # the output by at most the bf16 precision of the weights
