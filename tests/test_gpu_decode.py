@@ -9,7 +9,7 @@ import pytest
 from synth.configs import CLA2_1P1B, DEPTHGRAFT_DECODE, MIX, SINGLE, TINY_CLA2, Config
 import synth.gpu as sgpu
 
-from gpu_helpers import assert_close, decode_gpu, oracle_decode, to_dev, make_ctx
+from gpu_helpers import assert_scaled, assert_close, decode_gpu, oracle_decode, to_dev, make_ctx
 
 pytestmark = pytest.mark.gpu
 
@@ -258,9 +258,11 @@ def test_full_size_sampled(K, cfg):
     res = oracle_pool.run(oracle_pool.decode_unit, [(cfg.name, l, b, j) for (l, b, j) in units])
     want = dict(zip(units, res))
     g = cfg.group
-    worst = 0.0
+    worst = scale = 0.0
     for (l, b, j), (o, s) in want.items():
         got = out[l, b, j * g:(j + 1) * g]
         worst = max(worst, assert_close(got, o, TOL_BF16, f"l{l} b{b} j{j}")[0])
+        scale = max(scale, float(np.max(np.abs(o))))
         assert_close(lse[l, b, j * g:(j + 1) * g], s, TOL_BF16, f"lse l{l} b{b} j{j}")
-    print(f"{cfg.name}: worst max|d| {worst:.3e}")
+    print(f"{cfg.name}: worst max|d| {worst:.3e}, max|want| {scale:.3e}")
+    assert_scaled(worst, scale, cfg.name)
