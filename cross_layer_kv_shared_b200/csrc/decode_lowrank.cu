@@ -586,9 +586,9 @@ int occupancy_of() {
 }
 
 // token tile, stages per warp and warps per CTA by basis rank (the full-rank basis only serves tests)
-// (defaults: the fastest of a measured sweep on the 64K-token, Rb = 32 workload; the
-// kernel is issue-latency bound, so 16 warps with one 32-token stage each beat deeper
-// rings on fewer warps)
+// (defaults: the fastest of a measured sweep on the 64K-token, Rb = 32 workload:
+// 16 warps with one 32-token stage each beat deeper rings on fewer warps, two stages
+// on 16 warps, and 18 to 20 warps)
 #ifndef KVS_LR_TT
 #define KVS_LR_TT 32
 #endif
