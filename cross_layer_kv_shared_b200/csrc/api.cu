@@ -1,11 +1,12 @@
 // Host side of libkvshare: argument validation, layer-table resolution,
 // split heuristic, TMA descriptors and kernel launches. See include/kvshare.h.
-#include <algorithm>
 #include "kvshare.h"
 
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -234,9 +235,14 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
         } else if (e.kind == KVS_SRC_LOWRANK) {
             const int Rb = cf.basis_rank;
             const int tt = decode_lowrank_tile(Rb);
-            static int occ_lr[2][3] = {{0, 0, 0}, {0, 0, 0}};
-            int& o = occ_lr[D == 128][Rb == 32 ? 0 : (Rb == 64 ? 1 : 2)];
-            if (o == 0) o = decode_lowrank_occupancy(D, Rb);
+            // occupancy per kernel shape, computed once (racing threads compute the same value)
+            static std::atomic<int> occ_lr[2][3];
+            std::atomic<int>& occ_slot = occ_lr[D == 128][Rb == 32 ? 0 : (Rb == 64 ? 1 : 2)];
+            int o = occ_slot.load(std::memory_order_relaxed);
+            if (o == 0) {
+                o = decode_lowrank_occupancy(D, Rb);
+                occ_slot.store(o, std::memory_order_relaxed);
+            }
             const int tiles = (T + tt - 1) / tt;
             int s = choose_splits(c, B * Hkv, tiles, o, g, Rb + 16);   // partials of Rb + 16 values
             a.tiles_per_split = (tiles + s - 1) / s;
@@ -271,9 +277,13 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
         } else {
             const bool mix = e.kind == KVS_SRC_MIX;
             const TileShape ts = decode_bf16_shape(D, mix);
-            static int occ[2][2] = {{0, 0}, {0, 0}};
-            int& o = occ[D == 128][mix];
-            if (o == 0) o = decode_bf16_ctas_per_sm(D, mix);
+            static std::atomic<int> occ[2][2];
+            std::atomic<int>& occ_slot = occ[D == 128][mix];
+            int o = occ_slot.load(std::memory_order_relaxed);
+            if (o == 0) {
+                o = decode_bf16_ctas_per_sm(D, mix);
+                occ_slot.store(o, std::memory_order_relaxed);
+            }
             // balanced grid: the units' token tiles cut into G equal ranges, one CTA each
             const int units = B * Hkv;
             const int n_t = (T + ts.tt - 1) / ts.tt;
