@@ -7,7 +7,8 @@
 * I5: brute force at 50 digits (mpmath, pure-Python loops) on tiny inputs, all
   three forms; the absorbed low-rank algebra the kernels use agrees.
 * I6: decode is invariant under a joint permutation of the cached tokens.
-* I8: causal prefill row i equals decode over tokens 0..i.
+* I8: causal prefill row i equals decode over tokens 0..i; an identity map's
+  prefill equals torch's causal SDPA (fp64).
 * closed forms: equal keys average V; two tokens give a logistic weight.
 * planted mistakes: each pin fails when a plausible bug is planted in the oracle.
 """
@@ -312,6 +313,33 @@ def test_prefill_row_equals_decode_over_prefix():
         assert np.max(np.abs(o[i] - d[0])) < 1e-13 and abs(lse[i] - ld[0]) < 1e-13
 
 
+def check_prefill_identity_map_is_causal_sdpa(L=2, B=2, Hq=8, Hkv=2, T=29, d=16):
+    g = Hq // Hkv
+    cache = rand_cache(L, B, Hkv, T, d, seed=21)
+    q = np.random.default_rng(22).standard_normal((L, B, Hq, T, d))
+    lmap = tuple((SINGLE, l, 0) for l in range(L))
+    rows = np.arange(T)
+    for l in range(L):
+        k = torch.from_numpy(cache["k"][l]).repeat_interleave(g, dim=1)     # [B, Hq, T, d]
+        v = torch.from_numpy(cache["v"][l]).repeat_interleave(g, dim=1)
+        qq = torch.from_numpy(q[l])
+        want = torch.nn.functional.scaled_dot_product_attention(qq, k, v, is_causal=True).numpy()
+        z = torch.einsum("bhid,bhtd->bhit", qq, k) / math.sqrt(d)
+        z = z.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), 1), float("-inf"))
+        want_lse = torch.logsumexp(z, dim=-1).numpy()
+        for b in range(B):
+            for h in range(Hq):
+                o, lse = ref.prefill_rows(lmap, l, b, h, g, q[l, b, h], rows, dict_get(cache))
+                assert np.max(np.abs(o - want[b, h])) < 1e-12
+                assert np.max(np.abs(lse - want_lse[b, h])) < 1e-12
+
+
+def test_prefill_identity_map_is_causal_sdpa():
+    # independent of the decode oracle: causal GQA attention by torch in fp64, each
+    # q head h reading kv head h // g, position i seeing tokens 0..i
+    check_prefill_identity_map_is_causal_sdpa()
+
+
 # ----------------------------------------------------------------------------- I9
 def test_stored_bytes_reproduce_the_pages_ratios():
     # Cross-Layer Attention, Abstract: CLA2 halves the cache.
@@ -363,3 +391,13 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(ref, "layer_kv", wrong_group)
     with pytest.raises(AssertionError):
         check_identity_map_is_sdpa()
+    with pytest.raises(AssertionError):
+        check_prefill_identity_map_is_causal_sdpa()
+    monkeypatch.setattr(ref, "layer_kv", orig_layer_kv)
+
+    def one_future_token(q, K, V, s, visible=None):                                # sees 0..i+1
+        return orig_attend(q, K, V, s, None if visible is None else np.asarray(visible) + 1)
+    monkeypatch.setattr(ref, "attend", one_future_token)
+    with pytest.raises(AssertionError):
+        check_prefill_identity_map_is_causal_sdpa()
+    monkeypatch.setattr(ref, "attend", orig_attend)
