@@ -486,6 +486,18 @@ def cpu_baseline(cfg, seconds=12.0):
                       f"{cfg.layers} layers x {cfg.batch} batch"}
 
 
+def data_desc(cfg):
+    """The synthetic input recipe of a workload, for the JSON line's "data" key."""
+    s = cfg.qkv_scale
+    if s == 1.0:
+        dist = "N(0,1)"
+    elif (1.0 / s).is_integer():
+        dist = f"N(0,1)/{1.0 / s:g}"
+    else:
+        dist = f"{s:g} x N(0,1)"
+    return f"synthetic (seeded Philox, q/k/v {dist})"
+
+
 def reference_arm(args):
     cfg = BY_NAME[args.config]
     rank = int(os.environ.get("RANK", "0"))
@@ -505,7 +517,7 @@ def reference_arm(args):
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tok/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox, N(0,1))",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": data_desc(cfg),
         "config": arm_config(cfg, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": val, "unit": "tok/s", "cores": threads, "kind": "oracle",
                          "sample": f"{units_total} (layer, batch) units over {args.steps} steps, extrapolated"},
@@ -603,7 +615,7 @@ def main():
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": cfg.dtype,
-        "data": "synthetic (seeded Philox, N(0,1)/8 q/k/v)",
+        "data": data_desc(cfg),
         "config": arm_config(cfg, world),
         "kv_gbs": main_res["kv_gbs"],
         "hbm_frac": main_res["kv_gbs"] / hbm_peak,

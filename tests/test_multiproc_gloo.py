@@ -47,3 +47,22 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
     monkeypatch.setenv("RANK", "1")
     bench.reference_arm(argparse.Namespace(config="cla2_1p1b", steps=1, warmup=3, gpus=2))
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_rank0_prints_one_contract_line(monkeypatch, capsys):
+    import argparse
+    import json
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    bench.reference_arm(argparse.Namespace(config="cla2_1p1b", steps=1, warmup=3, gpus=1))
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "tok/s"
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["n_gpus"] == 1
+    assert d["steps"] == 1 and d["warmup"] == 3 and d["config"]["workload"] == "cla2_1p1b"
+    assert d["data"] == "synthetic (seeded Philox, q/k/v N(0,1)/8)"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
