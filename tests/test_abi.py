@@ -71,3 +71,25 @@ def test_null_arguments_are_rejected_without_touching_the_gpu():
     assert lib.kvshare_create(ctypes.byref(bad), ctypes.byref(h)) == K.KVS_EUNSUPPORTED
     bad = K.kvshare_config(4, 64, 2, 64, K.KVS_BF16, 0.0, 32, 16, 1, 128)     # group of 32 > 16
     assert lib.kvshare_create(ctypes.byref(bad), ctypes.byref(h)) == K.KVS_EUNSUPPORTED
+
+
+def test_unsupported_low_rank_and_scale_settings_are_rejected_without_touching_the_gpu():
+    from cross_layer_kv_shared_b200 import kvshare as K
+    lib = K._lib
+    h = ctypes.c_void_p()
+
+    def create(**kw):
+        f = dict(L=4, Hq=8, Hkv=4, d=64, dt=K.KVS_BF16, scale=0.0, rb=32, rm=16, B=1, T=128)
+        f.update(kw)
+        c = K.kvshare_config(f["L"], f["Hq"], f["Hkv"], f["d"], f["dt"], f["scale"], f["rb"], f["rm"], f["B"], f["T"])
+        return lib.kvshare_create(ctypes.byref(c), ctypes.byref(h))
+
+    assert create(rb=48) == K.KVS_EUNSUPPORTED             # basis rank: 32 or head_dim only
+    assert create(d=64, rb=128) == K.KVS_EUNSUPPORTED      # full rank means Rb = d
+    assert create(rm=8) == K.KVS_EUNSUPPORTED              # residual rank fixed at 16
+    assert create(scale=-1.0) == K.KVS_EINVAL
+    assert create(scale=float("nan")) == K.KVS_EINVAL
+    assert create(scale=float("inf")) == K.KVS_EINVAL
+    assert create(dt=7) == K.KVS_EINVAL
+    assert create(B=0) == K.KVS_EINVAL and create(T=0) == K.KVS_EINVAL and create(L=0) == K.KVS_EINVAL
+    assert not h.value
