@@ -93,3 +93,20 @@ def test_unsupported_low_rank_and_scale_settings_are_rejected_without_touching_t
     assert create(dt=7) == K.KVS_EINVAL
     assert create(B=0) == K.KVS_EINVAL and create(T=0) == K.KVS_EINVAL and create(L=0) == K.KVS_EINVAL
     assert not h.value
+
+
+def test_noalloc_shape_and_source_checks_run_before_any_cuda_call():
+    from cross_layer_kv_shared_b200 import kvshare as K
+    f = K._lib.kvshare_decode_layer_noalloc
+
+    def call(B=2, Hq=8, Hkv=2, d=64, T=64, slots=2, s0=0, s1=-1):
+        return f(None, None, None, None, None, None, B, Hq, Hkv, d, T, slots, s0, s1, None)
+
+    assert call(B=0) == K.KVS_EINVAL and call(T=0) == K.KVS_EINVAL and call(slots=0) == K.KVS_EINVAL
+    assert call(Hq=6, Hkv=4) == K.KVS_EINVAL                 # Hq % Hkv != 0
+    assert call(d=96) == K.KVS_EUNSUPPORTED
+    assert call(Hq=64, Hkv=2) == K.KVS_EUNSUPPORTED          # group of 32 > 16
+    assert call(s0=2) == K.KVS_EINVAL and call(s0=-1) == K.KVS_EINVAL
+    assert call(s1=2) == K.KVS_EINVAL and call(s1=0) == K.KVS_EINVAL   # mix source out of range / same as src0
+    assert call(B=2049, Hkv=2, Hq=2) == K.KVS_EINVAL          # 4098 units > 4096
+    assert call() == K.KVS_EINVAL                             # valid shape, but null (non-device) pointers
