@@ -89,6 +89,7 @@ struct kvshare_ctx {
     int splits_override = 0;
     int kv_overlap = 0;
     int grid_override = 0;
+    std::vector<int> order;          // layer order of decode calls (a permutation of 0..L-1)
     int stall_next = 0;
     long long wait_limit = 4000000000LL;     // ~2 s of SM clock
     long long stall_limit = 20000000LL;      // ~10 ms
@@ -183,8 +184,29 @@ kvshare_status check_layer_sources(const kvshare_ctx* c, const kvshare_cache* k,
     return KVS_OK;
 }
 
+// Prefill fills a slot when its owner runs: the first layer (lowest index) of the map that
+// reads the slot as a SINGLE source. A two-source target rebuilds its K/V from slots its
+// own forward pass has already produced, so each source needs an owner shallower than the
+// target ("DepthGraft: Structural Regularization through Hierarchical Cross-Layer KV
+// Reconstruction", Abstract: deep layers rebuilt from shallow and middle sources, prefill
+// keeping its early completion).
+bool prefill_source_ready(const kvshare_ctx* c, int slot, int target) {
+    for (int l = 0; l < target; ++l)
+        if (c->map[l].kind == KVS_SRC_SINGLE && c->map[l].src0 == slot) return true;
+    return false;
+}
+
+// The layers of [l0, l1) in the context's decode order.
+std::vector<int> ordered_layers(const kvshare_ctx* c, int l0, int l1) {
+    std::vector<int> ls;
+    ls.reserve(l1 - l0);
+    for (int l : c->order)
+        if (l >= l0 && l < l1) ls.push_back(l);
+    return ls;
+}
+
 kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void* q, float* out, float* lse,
-                             int l0, int l1, cudaStream_t st) {
+                             const int* layers, int n_layers, cudaStream_t st) {
     const kvshare_config& cf = c->cfg;
     const int D = cf.head_dim;
     const int B = k->batch;
@@ -195,7 +217,8 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
     const size_t es = elem_size(cf.dtype);
     if (cudaSetDevice(c->device) != cudaSuccess) return KVS_ECUDA;
 
-    for (int l = l0; l < l1; ++l) {
+    for (int li = 0; li < n_layers; ++li) {
+        const int l = layers[li];
         const kvshare_layer& e = c->map[l];
         DecodeArgs a;
         std::memset(&a, 0, sizeof(a));
@@ -388,6 +411,8 @@ kvshare_status kvshare_create(const kvshare_config* cfg, kvshare_t* out) {
     const int part_values = std::max(c.head_dim, ctx->cfg.basis_rank + ctx->cfg.max_resid_rank);
     ctx->ws_floats = units * ms * g * (part_values + 4);
     ctx->map.assign(c.num_layers, kvshare_layer{KVS_SRC_SINGLE, 0, 0});
+    ctx->order.resize(c.num_layers);
+    for (int l = 0; l < c.num_layers; ++l) ctx->order[l] = l;
     ctx->w_host.assign(static_cast<size_t>(c.num_layers) * c.num_kv_heads, 1.0f);
     if (cudaMalloc(&ctx->ws, ctx->ws_floats * sizeof(float)) != cudaSuccess ||
         cudaMalloc(&ctx->counters, units * sizeof(unsigned)) != cudaSuccess ||
@@ -476,7 +501,9 @@ kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const v
                               int l0, int l1, void* stream) {
     kvshare_status s = validate_decode(ctx, cache, q, out, lse, l0, l1, false);
     if (s != KVS_OK) return s;
-    return decode_layers(ctx, cache, q, out, lse, l0, l1, static_cast<cudaStream_t>(stream));
+    const std::vector<int> ls = ordered_layers(ctx, l0, l1);
+    return decode_layers(ctx, cache, q, out, lse, ls.data(), static_cast<int>(ls.size()),
+                         static_cast<cudaStream_t>(stream));
 }
 
 kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, const void* q_host, float* out_host,
@@ -514,13 +541,20 @@ kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, co
     const size_t layh = static_cast<size_t>(cache->batch) * cf.num_q_heads;
     const int nl = l1 - l0;
     if (nl == 0) return KVS_OK;
-    // Chunks of layers: chunk c's q is copied in on h2d while earlier chunks decode on
-    // `stream`, and its outputs are copied out on d2h while later chunks decode. The
-    // copy streams first wait for work already on `stream` (an earlier call may still be
-    // using the staging buffers), and `stream` waits for the last copy out, so the call
-    // is ordered on `stream` exactly like one that ran everything there.
+    // q is copied in as up to 8 contiguous chunks of layers on h2d; the layers decode on
+    // `stream` in the context's order, each after the chunk holding its q has landed; a
+    // chunk's out and lse are copied back on d2h as soon as its last layer has decoded.
+    // The copy streams first wait for work already on `stream` (an earlier call may still
+    // be using the staging buffers), and `stream` waits for the last copy out, so the call
+    // is ordered on `stream` exactly like one that ran everything there. In model order
+    // this pipelines the copies of one chunk under the decode of the others.
     const int nch = nl < kvshare_ctx::HOST_CHUNKS ? nl : kvshare_ctx::HOST_CHUNKS;
     auto chunk_begin = [&](int c) { return l0 + static_cast<int>((static_cast<long long>(nl) * c) / nch); };
+    auto chunk_of = [&](int l) {
+        int c = 0;
+        while (c + 1 < nch && chunk_begin(c + 1) <= l) ++c;
+        return c;
+    };
     cudaError_t e = cudaEventRecord(ctx->ev_start, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->h2d, ctx->ev_start, 0);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->d2h, ctx->ev_start, 0);
@@ -532,11 +566,23 @@ kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, co
         if (e == cudaSuccess) e = cudaEventRecord(ctx->ev_in[c], ctx->h2d);
     }
     if (e != cudaSuccess) return KVS_ECUDA;
+    const std::vector<int> ls = ordered_layers(ctx, l0, l1);
+    int remaining[kvshare_ctx::HOST_CHUNKS];
+    bool waited[kvshare_ctx::HOST_CHUNKS];
     for (int c = 0; c < nch; ++c) {
-        const int a = chunk_begin(c), b = chunk_begin(c + 1);
-        if (cudaStreamWaitEvent(st, ctx->ev_in[c], 0) != cudaSuccess) return KVS_ECUDA;
-        s = decode_layers(ctx, cache, ctx->q_stage, ctx->out_stage, lse_host ? ctx->lse_stage : nullptr, a, b, st);
+        remaining[c] = chunk_begin(c + 1) - chunk_begin(c);
+        waited[c] = false;
+    }
+    for (int l : ls) {
+        const int c = chunk_of(l);
+        if (!waited[c]) {
+            if (cudaStreamWaitEvent(st, ctx->ev_in[c], 0) != cudaSuccess) return KVS_ECUDA;
+            waited[c] = true;
+        }
+        s = decode_layers(ctx, cache, ctx->q_stage, ctx->out_stage, lse_host ? ctx->lse_stage : nullptr, &l, 1, st);
         if (s != KVS_OK) return s;
+        if (--remaining[c] > 0) continue;
+        const size_t a = chunk_begin(c), b = chunk_begin(c + 1);
         e = cudaEventRecord(ctx->ev_out[c], st);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->d2h, ctx->ev_out[c], 0);
         if (e == cudaSuccess)
@@ -566,6 +612,9 @@ kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const 
     for (int l = l0; l < l1; ++l) {
         s = check_layer_sources(ctx, cache, l, &need_kv, &need_lr);
         if (s != KVS_OK) return s;
+        if (ctx->map[l].kind == KVS_SRC_MIX && !(prefill_source_ready(ctx, ctx->map[l].src0, l) &&
+                                                  prefill_source_ready(ctx, ctx->map[l].src1, l)))
+            return KVS_EINVAL;
     }
     if (need_lr || cf.dtype != KVS_BF16) return KVS_EUNSUPPORTED;
     if (need_kv && (cache->slots < 1 || !dev_ok(cache->k) || !dev_ok(cache->v))) return KVS_EINVAL;
@@ -664,6 +713,25 @@ kvshare_status kvshare_set_splits(kvshare_t ctx, int splits) {
 kvshare_status kvshare_set_kv_overlap(kvshare_t ctx, int on) {
     if (ctx == nullptr) return KVS_EINVAL;
     ctx->kv_overlap = on ? 1 : 0;
+    return KVS_OK;
+}
+
+kvshare_status kvshare_set_layer_order(kvshare_t ctx, const int* order) {
+    if (ctx == nullptr) return KVS_EINVAL;
+    const int L = ctx->cfg.num_layers;
+    std::vector<int> o(L);
+    if (order == nullptr) {
+        for (int l = 0; l < L; ++l) o[l] = l;
+    } else {
+        std::vector<char> seen(L, 0);
+        for (int i = 0; i < L; ++i) {
+            const int l = order[i];
+            if (l < 0 || l >= L || seen[l]) return KVS_EINVAL;
+            seen[l] = 1;
+            o[i] = l;
+        }
+    }
+    ctx->order.swap(o);
     return KVS_OK;
 }
 

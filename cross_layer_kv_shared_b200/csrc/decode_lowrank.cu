@@ -18,7 +18,7 @@
 //   - tokens are the MMA's M rows and the g heads its N columns (S^T = C q~^T),
 //     so a group of up to 8 heads wastes nothing on padding; P^T reaches the
 //     PV MMAs through an in-register transpose (movmatrix);
-//   - int8 codes convert exactly to bf16 operands, masked by the token's rank;
+//   - int8 codes convert exactly to f16 operands, masked by the token's rank;
 //   - c^ and u^ accumulate in fp32 MMA accumulators; split partials stay in this
 //     coefficient space and the CTA that merges a unit projects it once.
 #include "kvs_device.cuh"

@@ -19,6 +19,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -125,14 +126,27 @@ extern "C" kvshare_status kvshare_decode_layer_noalloc(const void* q, const void
 
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // resident CTAs per SM of each kernel variant, looked up once (racing threads store
+    // the same value)
+    static std::atomic<int> occ[2][2];
+    std::atomic<int>& occ_slot = occ[head_dim == 128][mix];
+    int ctas_per_sm = occ_slot.load(std::memory_order_relaxed);
+    if (ctas_per_sm == 0) {
+        ctas_per_sm = decode_bf16_ctas_per_sm(head_dim, mix);
+        occ_slot.store(ctas_per_sm, std::memory_order_relaxed);
+    }
     const TileShape ts = decode_bf16_shape(head_dim, mix);
     // balanced grid: the units' token tiles cut into G equal ranges, one CTA each; a
     // unit spread over several CTAs keeps one partial per CTA in the array
     const int n_t = (context + ts.tt - 1) / ts.tt;
     const long long W = units * n_t;
-    const long long per_unit = (static_cast<long long>(sms) * decode_bf16_ctas_per_sm(head_dim, mix)) / units;
+    const long long per_unit = (static_cast<long long>(sms) * ctas_per_sm) / units;
     long long G = units * (per_unit > 1 ? per_unit : 1);
     if (G > W) G = W;
+    // partial slots run up to units + G; lower G until they fit the array. With one CTA
+    // per unit (G == units) no partial is written at all. On a 148-SM B200 with one
+    // resident CTA per SM the default grid always fits (at most 222 slots of
+    // 16 x (128 + 4) floats, 1.9 MB), so the loop guards other devices and tile shapes.
     const size_t per = static_cast<size_t>(g) * (head_dim + 4);
     while (G > units && (static_cast<size_t>(units) + G) * per > PARTIAL_FLOATS) --G;
 

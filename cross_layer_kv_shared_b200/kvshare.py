@@ -64,6 +64,7 @@ def _load():
         "kvshare_sync_status": ([P, V], I),
         "kvshare_set_splits": ([P, I], I),
         "kvshare_set_kv_overlap": ([P, I], I),
+        "kvshare_set_layer_order": ([P, P], I),
         "kvshare_debug_stall_next": ([P, I], I),
         "kvshare_debug_set_grid": ([P, I], I),
         "kvshare_launch_count": ([P], ctypes.c_uint64),
@@ -213,6 +214,17 @@ def kvshare_set_splits(h, splits: int) -> int:
 
 def kvshare_set_kv_overlap(h, on: bool = True) -> int:
     return _check(_lib.kvshare_set_kv_overlap(h, 1 if on else 0), "kvshare_set_kv_overlap")
+
+
+def kvshare_set_layer_order(h, order=None, check: bool = True) -> int:
+    """order: sequence of num_layers distinct layer indices, or None for model order."""
+    keep = None
+    if order is not None:
+        keep = (ctypes.c_int * len(order))(*[int(x) for x in order])
+    st = _lib.kvshare_set_layer_order(h, keep)
+    if check:
+        _check(st, "kvshare_set_layer_order")
+    return st
 
 
 def kvshare_debug_set_grid(h, ctas: int) -> int:

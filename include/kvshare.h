@@ -124,7 +124,8 @@ kvshare_status kvshare_destroy(kvshare_t ctx);
  *        entry is MIX. Rows of non-MIX layers are ignored. */
 kvshare_status kvshare_set_map(kvshare_t ctx, const kvshare_layer* map, const float* w);
 
-/* One decode step for layers [l0, l1), launched in layer order on `stream`.
+/* One decode step for layers [l0, l1), launched on `stream` in the context's
+ * layer order (model order unless kvshare_set_layer_order changed it).
  *   q:   [L][batch][Hq][d] in the config dtype (layer l at offset l*batch*Hq*d)
  *   out: [L][batch][Hq][d] fp32
  *   lse: [L][batch][Hq] fp32 natural-log sum of exp of the scaled scores, or NULL
@@ -143,17 +144,26 @@ kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const v
  * kvshare_decode, host memory; pinned memory makes the copies asynchronous).
  * The cache stays on the device. Results are valid after the stream has
  * synchronised. The staging buffers, two copy streams and their events are
- * created on the first call and reused: the layers run in up to 8 chunks, each
- * chunk's q copied in on one copy stream while earlier chunks decode on
- * `stream`, its outputs copied out on the other while later chunks decode. The
- * copy streams wait for work already on `stream` first, and `stream` waits for
- * the last copy out, so the call is ordered on `stream` like a serial one. */
+ * created on the first call and reused. q is copied in as up to 8 contiguous
+ * chunks of layers on one copy stream; the layers decode on `stream` in the
+ * context's layer order (kvshare_set_layer_order), each once its chunk has
+ * landed; a chunk's out and lse are copied back on the other copy stream once its
+ * last layer has decoded (in model order: copies of one chunk under the decode of
+ * the others). The copy streams wait for work already on `stream` first, and
+ * `stream` waits for the last copy out, so the call is ordered on `stream` like a
+ * serial one. */
 kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, const void* q_host,
                                    float* out_host, float* lse_host, int l0, int l1, void* stream);
 
 /* Causal prefill of `seqlen` tokens for layers [l0, l1) (bf16 only; SINGLE and
  * MIX layers, LOWRANK gives KVS_EUNSUPPORTED). A MIX layer's K/V operands are
  * mixed from its two source slots inside the kernel and never written to HBM.
+ * In a forward pass a slot is filled by its owner, the first layer of the map that
+ * reads it as a SINGLE source, so a MIX layer's two sources must each be read as
+ * SINGLE by some layer shallower than it; otherwise KVS_EINVAL ("DepthGraft:
+ * Structural Regularization through Hierarchical Cross-Layer KV Reconstruction",
+ * Abstract: deep layers rebuilt from shallow and middle sources). The check covers
+ * the whole map, not only [l0, l1).
  *   q:   [L][batch][Hq][seqlen][d] bf16
  *   out: [L][batch][Hq][seqlen][d] bf16
  *   lse: [L][batch][Hq][seqlen] fp32 or NULL
@@ -195,6 +205,15 @@ kvshare_status kvshare_set_splits(kvshare_t ctx, int splits);
  * before it is written. Results are identical either way. */
 kvshare_status kvshare_set_kv_overlap(kvshare_t ctx, int on);
 
+/* Order in which kvshare_decode and kvshare_decode_host launch the layers of a
+ * call: `order` is a HOST array of num_layers distinct layer indices (a
+ * permutation, copied); a call over [l0, l1) runs the layers of that range in the
+ * order they appear in it. NULL restores model order 0, 1, ..., L-1. Each layer's
+ * attention depends only on its own q and sources, so results do not change; the
+ * order decides which shared sources are still in L2 when a layer reads them.
+ * KVS_EINVAL if an entry is out of range or repeated. */
+kvshare_status kvshare_set_layer_order(kvshare_t ctx, const int* order);
+
 /* Test hook: force the bf16 decode grid to `ctas` CTAs (0 = automatic). The
  * units' token tiles are cut into that many equal ranges, so a CTA may cover
  * the end of one (batch, kv head) unit and the start of the next; the units'
@@ -224,7 +243,9 @@ uint64_t kvshare_launch_count(kvshare_t ctx);
  *   w: [Hkv] fp32 device weights in [0, 1] (ignored for a single source).
  *   Softmax scale 1/sqrt(d); d is 64 or 128; Hq / Hkv <= 16.
  * Limits: batch * Hkv <= 4096, else KVS_EINVAL; the split count is lowered
- * until the partials fit the array. The first call on each device looks up
+ * until the partials fit the array. Every pointer must be device (or managed)
+ * memory, checked with cudaPointerGetAttributes: host memory, mapped pinned
+ * memory included, gives KVS_EINVAL. The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) and should come before
  * any stream capture. Every call shares the array and keeps the previous
  * call's contents; the call clears the counters and status word on `stream`

@@ -41,7 +41,8 @@ def decode_unit(cfg_name, l, b, j):
 # ---------------------------------------------------------------- decode, low-rank form
 def lowrank_unit(cfg_name, l, j):
     """Low-rank decode of layer l, kv head j at batch 0, with the packer rule run on the
-    host: returns (o [g][d], lse [g], rank [T], codes_k [T][16], scale_v bits [T])."""
+    host: returns (o [g][d], lse [g], rank [T], codes_k [T][16], codes_v [T][16],
+    scale_k bits [T], scale_v bits [T])."""
     from oracle import kvshare_ref as ref
     from oracle import quant_ref as qr
     from synth.configs import BY_NAME
@@ -60,7 +61,7 @@ def lowrank_unit(cfg_name, l, j):
                                  ref.bf16_bits_to_f64(cfg.make("r_" + s, (l, j))), r))
     q = ref.bf16_bits_to_f64(cfg.make("q", (l, 0))[j * g:(j + 1) * g])
     o, lse, _ = ref.attend(q, kv[0], kv[1], 1 / np.sqrt(cfg.head_dim))
-    return o, lse, r, codes_k, scv
+    return o, lse, r, codes_k, codes_v, sck, scv
 
 
 # ---------------------------------------------------------------- causal prefill

@@ -176,8 +176,12 @@ def test_layer_range_writes_only_its_rows(K):
     assert_close(out[1:3], want[1:3], TOL_BF16)
 
 
-def test_decode_host_matches_device_call(K):
+@pytest.mark.parametrize("order", ["model", "cold", "reversed"])
+def test_decode_host_matches_device_call(K, order):
+    # the host-buffer call, with the layers launched in model order, in the bench's cold
+    # order or reversed: the same bits as the device call in model order
     import torch
+    import bench
     cfg = DG_SMALL
     inp = cfg.make_all()
     out, lse, _ = decode_gpu(K, cfg, inp)
@@ -185,15 +189,36 @@ def test_decode_host_matches_device_call(K):
     h = make_ctx(K, cfg)
     try:
         K.kvshare_set_map(h, cfg.layer_map, inp["w"])
+        perm = {"model": None, "cold": bench.cold_order(cfg), "reversed": list(range(cfg.layers))[::-1]}[order]
+        K.kvshare_set_layer_order(h, perm)
         qh = torch.from_numpy(np.ascontiguousarray(inp["q"]).view(np.int16)).pin_memory()
-        oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-        lh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        oh = torch.full(out.shape, float("nan"), dtype=torch.float32).pin_memory()
+        lh = torch.full(lse.shape, float("nan"), dtype=torch.float32).pin_memory()
         cache = K.Cache(batch=cfg.batch, context=cfg.context, k=d["k"], v=d["v"], slots=cfg.slots)
-        K.kvshare_decode_host(h, cache, qh, oh, lh)
+        for _ in range(2):     # a second call reuses the staging buffers
+            K.kvshare_decode_host(h, cache, qh, oh, lh)
+            assert K.kvshare_sync_status(h) == K.KVS_OK
+            assert np.array_equal(oh.numpy(), out) and np.array_equal(lh.numpy(), lse)
+        # a partial range in that order writes only its layers
+        oh.fill_(float("nan"))
+        K.kvshare_decode_host(h, cache, qh, oh, lh, 1, 3)
         assert K.kvshare_sync_status(h) == K.KVS_OK
+        assert np.array_equal(oh.numpy()[1:3], out[1:3]) and np.all(np.isnan(oh.numpy()[0]))
     finally:
         K.kvshare_destroy(h)
-    assert np.array_equal(oh.numpy(), out) and np.array_equal(lh.numpy(), lse)
+
+
+def test_layer_order_validation(K):
+    cfg = DG_SMALL
+    h = make_ctx(K, cfg)
+    try:
+        L = cfg.layers
+        assert K.kvshare_set_layer_order(h, [0] * L, check=False) == K.KVS_EINVAL          # repeated
+        assert K.kvshare_set_layer_order(h, list(range(1, L + 1)), check=False) == K.KVS_EINVAL   # out of range
+        assert K.kvshare_set_layer_order(h, list(range(L))[::-1], check=False) == K.KVS_OK
+        assert K.kvshare_set_layer_order(h, None, check=False) == K.KVS_OK
+    finally:
+        K.kvshare_destroy(h)
 
 
 # ----------------------------------------------------------------------------- full sizes, sampled

@@ -1,5 +1,4 @@
 """Host validation, unsupported combinations and the bounded device wait (no GPU fault)."""
-import ctypes
 
 import numpy as np
 import pytest
@@ -115,8 +114,58 @@ def test_bounded_wait_in_the_bf16_kernel(K):
         K.kvshare_destroy(h)
 
 
-def test_unsupported_prefill_for_now_or_lowrank(K, setup):
+def test_prefill_rejects_fp32_with_unsupported(K, setup):
+    # the fp32 tiny workload: prefill runs on bf16 operands only
     cfg, h, d, out, cache = setup
-    lib = K._lib
-    st = lib.kvshare_prefill(h, ctypes.byref(cache.as_c()), d["q"].data_ptr(), out.data_ptr(), None, 0, 1, 1, None)
-    assert st in (K.KVS_EUNSUPPORTED, K.KVS_EINVAL)
+    n0 = K.kvshare_launch_count(h)
+    st = K.kvshare_prefill(h, cache, d["q"], out, None, 0, 1, seqlen=1, check=False)
+    assert st == K.KVS_EUNSUPPORTED
+    assert K.kvshare_launch_count(h) == n0
+
+
+def prefill_ctx(K, layer_map, L=3, Hq=4, Hkv=2, d=64, T=32, w=None):
+    import torch
+    _, h = K.kvshare_create(L, Hq, Hkv, d, K.KVS_BF16, 1, T)
+    w = np.full((L, Hkv), 0.5, np.float32) if w is None else w
+    q = torch.zeros(L, 1, Hq, T, d, dtype=torch.bfloat16, device="cuda")
+    o = torch.zeros_like(q)
+    kv = torch.zeros(3, 1, Hkv, T, d, dtype=torch.bfloat16, device="cuda")
+    cache = K.Cache(batch=1, context=T, k=kv, v=kv, slots=3)
+    return h, q, o, cache, w
+
+
+def test_prefill_lowrank_layer_is_unsupported(K):
+    h, q, o, cache, w = prefill_ctx(K, None)
+    try:
+        K.kvshare_set_map(h, [(SINGLE, 0, 0), (SINGLE, 1, 0), (LOWRANK, 0, 0)], None)
+        n0 = K.kvshare_launch_count(h)
+        st = K.kvshare_prefill(h, cache, q, o, None, 0, 3, seqlen=32, check=False)
+        assert st == K.KVS_EUNSUPPORTED
+        assert K.kvshare_launch_count(h) == n0
+    finally:
+        K.kvshare_destroy(h)
+
+
+@pytest.mark.parametrize("layer_map,ok", [
+    ([(SINGLE, 0, 0), (SINGLE, 1, 0), (MIX, 0, 1)], True),      # both sources owned by shallower layers
+    ([(SINGLE, 0, 0), (MIX, 0, 1), (SINGLE, 1, 0)], False),     # slot 1 is filled deeper than the target
+    ([(SINGLE, 0, 0), (SINGLE, 0, 0), (MIX, 0, 2)], False),     # slot 2 has no owner at all
+    ([(MIX, 0, 1), (SINGLE, 0, 0), (SINGLE, 1, 0)], False),     # both sources deeper
+], ids=["owned", "deeper_source", "unowned_slot", "both_deeper"])
+def test_prefill_mix_sources_must_be_owned_by_shallower_layers(K, layer_map, ok):
+    h, q, o, cache, w = prefill_ctx(K, None)
+    try:
+        K.kvshare_set_map(h, layer_map, w)
+        n0 = K.kvshare_launch_count(h)
+        mix_l = [l for l, e in enumerate(layer_map) if e[0] == MIX][0]
+        # the rule covers the map, so a call over the target layer alone is judged the same
+        st = K.kvshare_prefill(h, cache, q, o, None, mix_l, mix_l + 1, seqlen=32, check=False)
+        if ok:
+            assert st == K.KVS_OK
+            assert K.kvshare_launch_count(h) == n0 + 1
+            assert K.kvshare_sync_status(h) == K.KVS_OK
+        else:
+            assert st == K.KVS_EINVAL
+            assert K.kvshare_launch_count(h) == n0
+    finally:
+        K.kvshare_destroy(h)

@@ -227,6 +227,8 @@ def test_full_size_sampled(K):
     lse = lse.cpu().numpy()
     rank_d = rank.cpu().numpy()
     ck_d = ck.cpu().numpy()
+    cv_d = cv.cpu().numpy()
+    sk_d = sk.cpu().numpy().view(np.uint16)
     sv_d = sv.cpu().numpy().view(np.uint16)
     # every layer and kv head (batch 1): the packer's bits and the decode against the oracle
     import oracle_pool
@@ -234,9 +236,11 @@ def test_full_size_sampled(K):
     res = oracle_pool.run(oracle_pool.lowrank_unit, [(cfg.name, l, j) for (l, j) in units])
     g = cfg.group
     worst = scale = 0.0
-    for (l, j), (o, s_, r, codes_k, scv) in zip(units, res):
+    for (l, j), (o, s_, r, codes_k, codes_v, sck, scv) in zip(units, res):
         assert np.array_equal(rank_d[l, 0], r)
         assert np.array_equal(ck_d[l, 0, j], codes_k)
+        assert np.array_equal(cv_d[l, 0, j], codes_v)
+        assert np.array_equal(sk_d[l, 0, j], sck)
         assert np.array_equal(sv_d[l, 0, j], scv)
         worst = max(worst, assert_close(out[l, 0, j * g:(j + 1) * g], o, TOL, f"l{l} j{j}")[0])
         scale = max(scale, float(np.max(np.abs(o))))
