@@ -11,6 +11,9 @@ Modules
 ``kvshare_ref``  layer-map resolution, K/V reconstruction for the three
                  sharing forms, softmax attention (decode and causal prefill),
                  stored-byte counts.
+``router_ref``   attention statistics of a decode step (per-head entropy and
+                 peak, per-kv-head attention mass each cached token receives)
+                 and the fp32 router score that feeds the rank rule.
 ``quant_ref``    the write side of the low-rank form: per-token rank routing and
                  symmetric int8 quantisation with an fp16 per-token scale,
                  evaluated in fp32 with correctly rounded IEEE operations.
@@ -18,4 +21,4 @@ Modules
 Every function is pinned by tests under ``tests/`` against closed forms,
 invariants, a library routine (torch SDPA in fp64) or high-precision brute force.
 """
-from . import kvshare_ref, quant_ref  # noqa: F401
+from . import kvshare_ref, quant_ref, router_ref  # noqa: F401

@@ -143,19 +143,31 @@ def layer_kv(layer_map, l: int, b: int, j: int, get, w=None):
     raise ValueError(f"unknown layer kind {kind}")
 
 
-def decode_head_group(layer_map, l, b, j, q_group, get, w=None, scale=None):
-    """Decode outputs of the q heads of kv head j: q_group [g, d] -> (o [g, d], lse [g])."""
+def decode_head_group(layer_map, l, b, j, q_group, get, w=None, scale=None, length=None):
+    """Decode outputs of the q heads of kv head j: q_group [g, d] -> (o [g, d], lse [g]).
+
+    ``length`` (optional) is the sequence's own token count: only cached tokens
+    0 .. length-1 are attended to. A sequence with no tokens has an empty softmax:
+    its outputs are 0 and its lse is -inf.
+    """
     K, V = layer_kv(layer_map, l, b, j, get, w)
+    if length is not None:
+        K, V = K[:int(length)], V[:int(length)]
+    q_group = np.atleast_2d(q_group)
+    if K.shape[0] == 0:
+        return np.zeros((q_group.shape[0], V.shape[1])), np.full(q_group.shape[0], -np.inf)
     d = K.shape[1]
     sc = 1.0 / np.sqrt(d) if scale is None else scale
     o, lse, _ = attend(q_group, K, V, sc)
     return o, lse
 
 
-def decode(layer_map, q, get, w=None, scale=None, layers=None, batches=None):
+def decode(layer_map, q, get, w=None, scale=None, layers=None, batches=None, lengths=None):
     """Full decode step: q [L][B][Hq][d] (fp64) -> out [L][B][Hq][d], lse [L][B][Hq].
 
-    Query head h reads kv head h // g (contiguous GQA groups).
+    Query head h reads kv head h // g (contiguous GQA groups). ``lengths`` [B]
+    (optional) gives each sequence's own token count; without it every sequence
+    attends to all cached tokens.
     """
     q = np.asarray(q, dtype=np.float64)
     L, B, Hq, d = q.shape
@@ -168,7 +180,8 @@ def decode(layer_map, q, get, w=None, scale=None, layers=None, batches=None):
                 Hkv = _kv_heads(get, layer_map, l)
             g = Hq // Hkv
             for j in range(Hkv):
-                o, s = decode_head_group(layer_map, l, b, j, q[l, b, j * g:(j + 1) * g], get, w, scale)
+                o, s = decode_head_group(layer_map, l, b, j, q[l, b, j * g:(j + 1) * g], get, w, scale,
+                                         None if lengths is None else lengths[b])
                 out[l, b, j * g:(j + 1) * g] = o
                 lse[l, b, j * g:(j + 1) * g] = s
     return out, lse
