@@ -95,6 +95,8 @@ struct kvshare_ctx {
     long long stall_limit = 20000000LL;      // ~10 ms
     uint64_t launches = 0;
     std::unordered_map<MapKey, CUtensorMap, MapKeyHash> maps;
+    // kept scores of one layer for the attention statistics [max_batch][Hq][max_context]
+    float* sscore = nullptr;
     // staging for kvshare_decode_host
     void* q_stage = nullptr;
     float* out_stage = nullptr;
@@ -205,8 +207,16 @@ std::vector<int> ordered_layers(const kvshare_ctx* c, int l0, int l1) {
     return ls;
 }
 
+// Optional statistics outputs of a decode call (all [L]-major, see kvshare_decode_stats).
+struct StatsOut {
+    float* mass;
+    float* score;
+    float* entropy;
+    float* peak;
+};
+
 kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void* q, float* out, float* lse,
-                             const int* layers, int n_layers, cudaStream_t st) {
+                             const int* layers, int n_layers, cudaStream_t st, const StatsOut* stats = nullptr) {
     const kvshare_config& cf = c->cfg;
     const int D = cf.head_dim;
     const int B = k->batch;
@@ -235,6 +245,8 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
         a.Hkv = Hkv;
         a.T = T;
         a.g = g;
+        a.lens = k->lengths;
+        a.sscore = stats != nullptr ? c->sscore : nullptr;
         a.scale_log2 = c->scale * 1.4426950408889634f;
         a.ws = c->ws;
         a.counters = c->counters;
@@ -338,6 +350,31 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
         }
         if (err != cudaSuccess) return KVS_ECUDA;
         ++c->launches;
+        if (stats != nullptr) {
+            StatsArgs sa;
+            std::memset(&sa, 0, sizeof(sa));
+            sa.sscore = c->sscore;
+            sa.lse = a.lse;
+            sa.lens = k->lengths;
+            const size_t lbt = static_cast<size_t>(l) * B;
+            sa.mass = stats->mass ? stats->mass + lbt * Hkv * T : nullptr;
+            sa.score = stats->score ? stats->score + lbt * T : nullptr;
+            sa.entropy = stats->entropy ? stats->entropy + lbt * Hq : nullptr;
+            sa.peak = stats->peak ? stats->peak + lbt * Hq : nullptr;
+            sa.err = c->err;
+            sa.B = B;
+            sa.Hq = Hq;
+            sa.Hkv = Hkv;
+            sa.T = T;
+            sa.g = g;
+            // entropy and peak accumulate: start each layer's rows at zero
+            if (sa.entropy && cudaMemsetAsync(sa.entropy, 0, static_cast<size_t>(B) * Hq * sizeof(float), st) != cudaSuccess)
+                return KVS_ECUDA;
+            if (sa.peak && cudaMemsetAsync(sa.peak, 0, static_cast<size_t>(B) * Hq * sizeof(float), st) != cudaSuccess)
+                return KVS_ECUDA;
+            if (launch_router_stats(sa, st) != cudaSuccess) return KVS_ECUDA;
+            ++c->launches;
+        }
     }
     return KVS_OK;
 }
@@ -359,6 +396,8 @@ kvshare_status validate_decode(kvshare_ctx* c, const kvshare_cache* k, const voi
         if (s != KVS_OK) return s;
         if (c->map[l].kind == KVS_SRC_LOWRANK && c->cfg.dtype != KVS_BF16) return KVS_EUNSUPPORTED;
     }
+    if (k->lengths != nullptr && (!is_device_ptr(k->lengths) || (reinterpret_cast<uintptr_t>(k->lengths) & 3u)))
+        return KVS_EINVAL;
     if (need_kv) {
         if (k->slots < 1 || !dev_ok(k->k) || !dev_ok(k->v)) return KVS_EINVAL;
     }
@@ -442,6 +481,7 @@ kvshare_status kvshare_destroy(kvshare_t ctx) {
     cudaFree(ctx->counters);
     cudaFree(ctx->err);
     cudaFree(ctx->w_dev);
+    cudaFree(ctx->sscore);
     cudaFree(ctx->q_stage);
     cudaFree(ctx->out_stage);
     cudaFree(ctx->lse_stage);
@@ -504,6 +544,32 @@ kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const v
     const std::vector<int> ls = ordered_layers(ctx, l0, l1);
     return decode_layers(ctx, cache, q, out, lse, ls.data(), static_cast<int>(ls.size()),
                          static_cast<cudaStream_t>(stream));
+}
+
+kvshare_status kvshare_decode_stats(kvshare_t ctx, const kvshare_cache* cache, const void* q, float* out, float* lse,
+                                    float* mass, float* score, float* entropy, float* peak, int l0, int l1,
+                                    void* stream) {
+    kvshare_status s = validate_decode(ctx, cache, q, out, lse, l0, l1, false);
+    if (s != KVS_OK) return s;
+    if (lse == nullptr) return KVS_EINVAL;
+    for (const float* p : {mass, score, entropy, peak})
+        if (p != nullptr && (!is_device_ptr(p) || (reinterpret_cast<uintptr_t>(p) & 3u))) return KVS_EINVAL;
+    const std::vector<int> ls = ordered_layers(ctx, l0, l1);
+    if (mass == nullptr && score == nullptr && entropy == nullptr && peak == nullptr)
+        return decode_layers(ctx, cache, q, out, lse, ls.data(), static_cast<int>(ls.size()),
+                             static_cast<cudaStream_t>(stream));
+    if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
+    if (ctx->sscore == nullptr) {
+        const size_t n = static_cast<size_t>(ctx->cfg.max_batch) * ctx->cfg.num_q_heads * ctx->cfg.max_context;
+        if (cudaMalloc(&ctx->sscore, n * sizeof(float)) != cudaSuccess) {
+            cudaGetLastError();
+            ctx->sscore = nullptr;
+            return KVS_ENOMEM;
+        }
+    }
+    const StatsOut so{mass, score, entropy, peak};
+    return decode_layers(ctx, cache, q, out, lse, ls.data(), static_cast<int>(ls.size()),
+                         static_cast<cudaStream_t>(stream), &so);
 }
 
 kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, const void* q_host, float* out_host,
@@ -606,9 +672,12 @@ kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const 
     const kvshare_config& cf = ctx->cfg;
     if (l0 < 0 || l1 > cf.num_layers || l0 > l1) return KVS_EINVAL;
     if (seqlen < 1 || seqlen > cache->context) return KVS_EINVAL;
+    if (cache->lengths != nullptr) return KVS_EUNSUPPORTED;   // one seqlen for every sequence
     if (!dev_ok(q) || !dev_ok(out) || (lse != nullptr && (!is_device_ptr(lse) || (reinterpret_cast<uintptr_t>(lse) & 3u))))
         return KVS_EINVAL;
     bool need_kv = false, need_lr = false;
+    for (int l = l0; l < l1; ++l)
+        if (ctx->map[l].kind == KVS_SRC_LOWRANK) return KVS_EUNSUPPORTED;
     for (int l = l0; l < l1; ++l) {
         s = check_layer_sources(ctx, cache, l, &need_kv, &need_lr);
         if (s != KVS_OK) return s;
@@ -700,6 +769,7 @@ kvshare_status kvshare_sync_status(kvshare_t ctx, void* stream) {
     if (word != 0) {
         if (cudaMemset(ctx->err, 0, sizeof(unsigned)) != cudaSuccess) return KVS_ECUDA;
         if (word & ERR_TIMEOUT) return KVS_ETIMEOUT;
+        if (word & ERR_RANGE) return KVS_EINVAL;
     }
     return KVS_OK;
 }

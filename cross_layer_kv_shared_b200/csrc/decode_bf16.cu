@@ -32,11 +32,11 @@ struct DecodeCfg {
     static constexpr int NSRC = MIX ? 2 : 1;
     static constexpr int STAGE_BYTES = 2 * NSRC * TILE_BYTES;
     static constexpr int RING_BYTES = NW * NSW * STAGE_BYTES;
-    static constexpr int COMBINE_FLOATS = NW * 16 * D + 2 * NW * 16 + 32 + 16 * D + 2 * MAX_GROUP * MAX_SPLITS + 64;
+    static constexpr int COMBINE_FLOATS = NW * 16 * D + 3 * NW * 16 + 48 + 16 * D + 3 * MAX_GROUP * MAX_SPLITS + 64;
     static constexpr int MERGE_STAGE_OFF = ((COMBINE_FLOATS * 4 + 1023) / 1024) * 1024;   // free smem for the merge
     static constexpr int BODY = RING_BYTES > COMBINE_FLOATS * 4 ? RING_BYTES : COMBINE_FLOATS * 4;
     // per-warp state of the first unit when a warp's tiles cross into the second one
-    static constexpr int SAVE_FLOATS = NW * (16 * D + 32);
+    static constexpr int SAVE_FLOATS = NW * (16 * D + 48);
     static constexpr int SMEM = BODY + SAVE_FLOATS * 4 + 1024;  // + slack to align the ring to 1024 B
     static constexpr int SMEM_ALIGNED = BODY + 1024;             // grids whose ranges never straddle
     static_assert(TT % 16 == 0, "token tile must hold whole m16 tiles");
@@ -52,7 +52,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     constexpr int NB = NH / 8;       // n8 head blocks
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    float* save = reinterpret_cast<float*>(smem + C::BODY);    // [NW][16][D] O, then [NW][16] m, [NW][16] l
+    float* save = reinterpret_cast<float*>(smem + C::BODY);    // [NW][16][D] O, then [NW][48]: m, l, lx
     __shared__ __align__(8) uint64_t bars[NW * NSW + 1];
     __shared__ int fin_unit[NW], sav_unit[NW];
 
@@ -64,10 +64,15 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     const long long W = static_cast<long long>(a.units) * a.n_t;
     const long long tb = (static_cast<long long>(cta) * W + G - 1) / G;
     const long long te = (static_cast<long long>(cta + 1) * W + G - 1) / G;
-    const int span = static_cast<int>(te - tb);
+    const int cap_span = static_cast<int>(te - tb);        // tiles of the range in store capacity
     const int u_first = static_cast<int>(tb / a.n_t);
     const int u_last = static_cast<int>((te - 1) / a.n_t);
     const int BH = a.B * a.Hkv;
+    // token tiles of unit u's own sequence
+    auto unit_tiles = [&](int u) { return (seq_len(a, u / a.Hkv) + TT - 1) / TT; };
+    // A range inside one unit is clipped to the unit's sequence; a range that may cross
+    // units keeps its tiles and skips those past their sequence one by one.
+    int span = cap_span;
 
     if (threadIdx.x == 0) {
         prefetch_tmap(&tmK);
@@ -79,7 +84,16 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 
     uint8_t* ring = smem + warp * NSW * C::STAGE_BYTES;
     uint64_t* wb = &bars[warp * NSW];
-    const int my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
+    int my_n = 0;
+    // with per-sequence lengths the range depends on them: read them where the first
+    // tiles are requested (before the dependent-launch wait only under kv_early)
+    auto set_range = [&] {
+        if (!STRADDLE && a.lens != nullptr) {
+            const long long u_end = static_cast<long long>(u_first) * a.n_t + unit_tiles(u_first);
+            span = te <= u_end ? cap_span : (u_end > tb ? static_cast<int>(u_end - tb) : 0);
+        }
+        my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
+    };
     // (unit, tile) of this warp's first tile; later tiles step by NW without dividing
     const long long g0 = tb + warp;
     const int u_w0 = static_cast<int>(g0 / a.n_t);
@@ -102,6 +116,10 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         const int row1 = MIX ? a.src1 * BH + u : 0;
         const int s = k % NSW;
         uint8_t* st = ring + s * C::STAGE_BYTES;
+        if (STRADDLE && a.lens != nullptr && t >= unit_tiles(u)) {
+            mbar_arrive(&wb[s]);      // a tile past its sequence: the stage completes empty
+            return;
+        }
         mbar_arrive_expect_tx(&wb[s], C::STAGE_BYTES);
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h) {
@@ -118,6 +136,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     // kv_early the caller has promised that no kernel ahead on the stream writes the
     // cache, so the first ring stages are already requested before the wait.
     if (a.kv_early) {
+        set_range();
         if (lane == 0) {
             for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
         }
@@ -126,6 +145,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     grid_dep_wait();
     if (threadIdx.x == 0) grid_dep_launch();
     if (!a.kv_early) {
+        set_range();
         if (lane == 0) {
             for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
         }
@@ -140,7 +160,10 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     uint32_t qb[D / 16][NB][2];      // B fragments of Q^T: column n = head nb*8 + lane/4
     float o[D / 16][NB][4];          // O^T: rows = channels, columns = heads nb*8 + 2(lane%4) (+1)
     float mrow[NB][2], lrow[NB][2];  // softmax statistics of those two heads
+    float lxrow[NB][2];              // sums of the unrounded weights (for the lse)
     float w = 1.f, w1 = 0.f;
+    int tlen = a.T;                  // tokens of the current unit's sequence
+    float* srow = nullptr;           // the current unit's kept scores [g][T], if requested
     auto begin_unit = [&](int u) {
         const int b = u / a.Hkv;
         const int j = u % a.Hkv;
@@ -157,13 +180,18 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             }
             mrow[nb][0] = mrow[nb][1] = NEG_INF;
             lrow[nb][0] = lrow[nb][1] = 0.f;
+            lxrow[nb][0] = lxrow[nb][1] = 0.f;
 #pragma unroll
             for (int i = 0; i < D / 16; ++i) o[i][nb][0] = o[i][nb][1] = o[i][nb][2] = o[i][nb][3] = 0.f;
         }
         w = MIX ? a.w[j] : 1.f;
         w1 = 1.f - w;
+        tlen = seq_len(a, b);
+        srow = a.sscore != nullptr ? a.sscore + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g) * a.T
+                                   : nullptr;
     };
-    // write this warp's statistics and O^T for heads < g: O to dst_o [16][D], m, l to dst_ml [32]
+    // write this warp's statistics and O^T for heads < g: O to dst_o [16][D], m, l, lx to
+    // dst_ml [48]
     auto store_state = [&](float* dst_o, float* dst_ml) {
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
@@ -171,6 +199,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             for (int off = 4; off < 32; off <<= 1) {
                 lrow[nb][0] += __shfl_xor_sync(0xffffffffu, lrow[nb][0], off);
                 lrow[nb][1] += __shfl_xor_sync(0xffffffffu, lrow[nb][1], off);
+                lxrow[nb][0] += __shfl_xor_sync(0xffffffffu, lxrow[nb][0], off);
+                lxrow[nb][1] += __shfl_xor_sync(0xffffffffu, lxrow[nb][1], off);
             }
         const int e0 = lane >> 2;
 #pragma unroll
@@ -192,6 +222,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                 dst_ml[h0 + 1] = mrow[nb][1];
                 dst_ml[16 + h0] = lrow[nb][0];
                 dst_ml[16 + h0 + 1] = lrow[nb][1];
+                dst_ml[32 + h0] = lxrow[nb][0];
+                dst_ml[32 + h0 + 1] = lxrow[nb][1];
             }
         }
     };
@@ -209,7 +241,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     for (int k = 0; k < my_n; ++k, advance(u, t)) {
         if (STRADDLE && u != cur_u) {
             if (cur_u >= 0) {
-                store_state(save + warp * 16 * D, save + NW * 16 * D + warp * 32);
+                store_state(save + warp * 16 * D, save + NW * 16 * D + warp * 48);
                 saved_u = cur_u;
             }
             begin_unit(u);
@@ -222,6 +254,19 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             const int issued = min(my_n, k + NSW);
             for (int kk = k + 1; kk < issued; ++kk) mbar_wait_bounded(&wb[kk % NSW], (kk / NSW) & 1, a.wait_limit, a.err);
             break;
+        }
+        if (STRADDLE && t * TT >= tlen) {
+            // a tile past the sequence: its stage completed empty; hand it on
+            __syncwarp();
+            if (lane == 0 && k + NSW < my_n) issue(k + NSW);
+            __syncwarp();
+            continue;
+        }
+        if (a.lens != nullptr && (t + 1) * TT > tlen) {
+            uint8_t* vt = ring + s * C::STAGE_BYTES + C::TILE_BYTES;
+            zero_tile_rows(vt, 128, C::HALVES, C::HALF_BYTES, tlen - t * TT, TT, lane);
+            if (MIX) zero_tile_rows(vt + 2 * C::TILE_BYTES, 128, C::HALVES, C::HALF_BYTES, tlen - t * TT, TT, lane);
+            __syncwarp();
         }
         const uint32_t kb = smem_u32(ring + s * C::STAGE_BYTES);
         const uint32_t vb = kb + C::TILE_BYTES;
@@ -257,8 +302,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         // ---- scale, mask the ragged tail, online softmax per head, P^T by movmatrix
         uint32_t pb[MT][NB][2];
         uint32_t pb2[MIX ? MT : 1][NB][2];
-        const bool tail = (t + 1) * TT > a.T;       // only the last tile holds tokens past T
-        const int lim = a.T - t * TT - (lane >> 2);  // rows r of this lane are valid iff r < lim
+        const bool tail = (t + 1) * TT > tlen;       // only the last tile holds tokens past the sequence
+        const int lim = tlen - t * TT - (lane >> 2);  // rows r of this lane are valid iff r < lim
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
             float mx0 = NEG_INF, mx1 = NEG_INF;
@@ -273,6 +318,18 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         if (mt * 16 + (i >> 1) * 8 >= lim) sc[mt][nb][i] = NEG_INF;
+            }
+            if (srow != nullptr) {
+                // keep the scores of the tile's valid tokens for the attention statistics
+                const int h0 = nb * 8 + 2 * (lane & 3);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int h = h0 + (i & 1);
+                        const int r = mt * 16 + (i >> 1) * 8;
+                        if (h < g && r < lim) srow[static_cast<size_t>(h) * a.T + t * TT + (lane >> 2) + r] = sc[mt][nb][i];
+                    }
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
@@ -294,6 +351,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             mrow[nb][1] = mn1;
             lrow[nb][0] *= cr0;
             lrow[nb][1] *= cr1;
+            lxrow[nb][0] *= cr0;
+            lxrow[nb][1] *= cr1;
 #pragma unroll
             for (int dt = 0; dt < D / 16; ++dt) {
                 o[dt][nb][0] *= cr0; o[dt][nb][2] *= cr0;
@@ -303,6 +362,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             for (int mt = 0; mt < MT; ++mt) {
                 const float p0 = ex2_approx(sc[mt][nb][0] - ref0), p1 = ex2_approx(sc[mt][nb][1] - ref1);
                 const float p2 = ex2_approx(sc[mt][nb][2] - ref0), p3 = ex2_approx(sc[mt][nb][3] - ref1);
+                lxrow[nb][0] += p0 + p2;
+                lxrow[nb][1] += p1 + p3;
                 if (!MIX) {
                     const uint32_t lo = pack_bf16(p0, p1), hi = pack_bf16(p2, p3);
                     lrow[nb][0] += bf16_lo(lo) + bf16_lo(hi);
@@ -352,12 +413,13 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     __syncthreads();
     (void)t;
     float* comb_o = reinterpret_cast<float*>(smem);   // [NW][16][D]
-    float* comb_ml = comb_o + NW * 16 * D;            // [NW][32]: m[16], l[16]
-    float* fin_m = comb_ml + NW * 32;                 // [16]
+    float* comb_ml = comb_o + NW * 16 * D;            // [NW][48]: m[16], l[16], lx[16]
+    float* fin_m = comb_ml + NW * 48;                 // [16]
     float* fin_l = fin_m + 16;                        // [16]
-    float* fin_o = fin_l + 16;                        // [16][D]
+    float* fin_lx = fin_l + 16;                       // [16]
+    float* fin_o = fin_lx + 16;                       // [16][D]
     float* scratch = fin_o + 16 * D;                  // merge scratch
-    if (cur_u >= 0) store_state(comb_o + warp * 16 * D, comb_ml + warp * 32);
+    if (cur_u >= 0) store_state(comb_o + warp * 16 * D, comb_ml + warp * 48);
     if (lane == 0) {
         fin_unit[warp] = cur_u;
         sav_unit[warp] = saved_u;
@@ -365,7 +427,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     __syncthreads();
     const float* save_o = save;
     const float* save_ml = save + NW * 16 * D;
-    for (int uu = u_first; uu <= u_last && span > 0; ++uu) {
+    // every CTA whose range meets a unit takes part in its merge, also with no tokens of it
+    for (int uu = u_first; uu <= u_last && cap_span > 0; ++uu) {
         const int u = uu;
         // the warps' contributions to unit u: final states, and states saved at a unit switch;
         // one weight 2^(m_w - M) per (warp, head), so the vector combine is FMAs only
@@ -374,24 +437,27 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             const int h = threadIdx.x;
             float M = NEG_INF;
             for (int ww = 0; ww < NW; ++ww) {
-                if (fin_unit[ww] == u) M = fmaxf(M, comb_ml[ww * 32 + h]);
-                if (STRADDLE && sav_unit[ww] == u) M = fmaxf(M, save_ml[ww * 32 + h]);
+                if (fin_unit[ww] == u) M = fmaxf(M, comb_ml[ww * 48 + h]);
+                if (STRADDLE && sav_unit[ww] == u) M = fmaxf(M, save_ml[ww * 48 + h]);
             }
-            float L = 0.f;
+            float L = 0.f, LX = 0.f;
             for (int ww = 0; ww < NW; ++ww) {
-                const float mf = comb_ml[ww * 32 + h];
+                const float mf = comb_ml[ww * 48 + h];
                 const float ff = (fin_unit[ww] == u && mf != NEG_INF) ? ex2_approx(mf - M) : 0.f;
                 fac_f[ww][h] = ff;
-                L += ff * comb_ml[ww * 32 + 16 + h];
+                L += ff * comb_ml[ww * 48 + 16 + h];
+                LX += ff * comb_ml[ww * 48 + 32 + h];
                 if (STRADDLE) {
-                    const float ms = save_ml[ww * 32 + h];
+                    const float ms = save_ml[ww * 48 + h];
                     const float fs = (sav_unit[ww] == u && ms != NEG_INF) ? ex2_approx(ms - M) : 0.f;
                     fac_s[ww][h] = fs;
-                    L += fs * save_ml[ww * 32 + 16 + h];
+                    L += fs * save_ml[ww * 48 + 16 + h];
+                    LX += fs * save_ml[ww * 48 + 32 + h];
                 }
             }
             fin_m[h] = M;
             fin_l[h] = L;
+            fin_lx[h] = LX;
         }
         __syncthreads();
         for (int idx = threadIdx.x; idx < g * D; idx += blockDim.x) {
@@ -416,7 +482,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         const int c_last = static_cast<int>(((static_cast<long long>(u + 1) * a.n_t - 1) * G) / W);
         const EmitPlain emit{a, D, static_cast<size_t>(u / a.Hkv) * a.Hq + static_cast<size_t>(u % a.Hkv) * g};
         finish_unit(a, D, u, cta - c_first, c_last - c_first + 1, static_cast<long long>(u) + c_first, fin_m, fin_l,
-                    fin_o, scratch, smem + C::MERGE_STAGE_OFF,
+                    fin_lx, fin_o, scratch, smem + C::MERGE_STAGE_OFF,
                     C::BODY > C::MERGE_STAGE_OFF ? C::BODY - C::MERGE_STAGE_OFF : 0, emit);
         __syncthreads();
     }

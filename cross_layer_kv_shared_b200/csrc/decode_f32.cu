@@ -17,11 +17,15 @@ constexpr int CH = 64;
 
 template <int D, bool MIX>
 __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
-    __shared__ float sq[MAX_GROUP][D];
-    __shared__ float ss[MAX_GROUP][CH];
+    // the query rows and a chunk's scores during the stream; the split merge's scratch after it
+    constexpr int STREAM_FLOATS = MAX_GROUP * D + MAX_GROUP * CH;
+    constexpr int MERGE_FLOATS = 3 * MAX_GROUP * MAX_SPLITS;
+    __shared__ float pool[STREAM_FLOATS > MERGE_FLOATS ? STREAM_FLOATS : MERGE_FLOATS];
+    float (*sq)[D] = reinterpret_cast<float (*)[D]>(pool);
+    float (*ss)[CH] = reinterpret_cast<float (*)[CH]>(pool + MAX_GROUP * D);
+    float* scratch = pool;
     __shared__ float sm_m[MAX_GROUP], sm_l[MAX_GROUP], scorr[MAX_GROUP];
     __shared__ float fin_o[MAX_GROUP * D];
-    __shared__ float scratch[2 * MAX_GROUP * MAX_SPLITS];
     __shared__ __align__(8) uint64_t never_bar;
 
     const int split = blockIdx.x;
@@ -60,7 +64,9 @@ __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
     __syncthreads();
 
     const int t0 = split * a.tiles_per_split * CH;
-    const int t1 = min(a.T, t0 + a.tiles_per_split * CH);
+    const int t1 = min(seq_len(a, b), t0 + a.tiles_per_split * CH);
+    float* srow = a.sscore != nullptr
+                      ? a.sscore + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g) * a.T : nullptr;
     for (int c = t0; c < t1; c += CH) {
         const int n = min(CH, t1 - c);
         for (int tt = warp; tt < n; tt += NT / 32) {
@@ -77,7 +83,10 @@ __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
                 for (int i = 0; i < D / 32; ++i) part += sq[h][lane + 32 * i] * kv[i];
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-                if (lane == 0) ss[h][tt] = part * a.scale_log2;
+                if (lane == 0) {
+                    ss[h][tt] = part * a.scale_log2;
+                    if (srow != nullptr) srow[static_cast<size_t>(h) * a.T + t] = part * a.scale_log2;
+                }
             }
         }
         __syncthreads();
@@ -121,7 +130,8 @@ __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
         if (idx < g * D) fin_o[idx] = acc[i];
     }
     __syncthreads();
-    finish_split(a, D, b, j, split, sm_m, sm_l, fin_o, scratch, nullptr, 0);
+    // the weights are fp32 throughout: the P.V sum and the exact sum are the same
+    finish_split(a, D, b, j, split, sm_m, sm_l, sm_l, fin_o, scratch, nullptr, 0);
 }
 
 template <int D, bool MIX>

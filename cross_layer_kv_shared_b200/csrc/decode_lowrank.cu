@@ -61,7 +61,7 @@ struct LrCfg {
     // [K | V][TT][16] halves, rows of 32 B whose two 16-B halves swap on every 4th row
     static constexpr int CVT_BYTES = NW * 2 * TT * 32;
     static constexpr int PD = RB + RM;    // coefficient-space partial width
-    static constexpr int COMBINE_FLOATS = NW * 16 * PD + 2 * NW * 16 + 32 + 16 * PD + 16 * D + 2 * MAX_GROUP * MAX_SPLITS + 64;
+    static constexpr int COMBINE_FLOATS = NW * 16 * PD + 3 * NW * 16 + 48 + 16 * PD + 16 * D + 3 * MAX_GROUP * MAX_SPLITS + 64;
     static constexpr int QPROJ_FLOATS = 16 * PD;
     // staging: B_K [RB][D] + R_K [RM][D] (bf16), the query rows [<=16][D], then B_V + R_V
     static constexpr int STAGE_FACTORS = (RB + RM) * D * 2;
@@ -81,7 +81,7 @@ struct EmitProject {
     size_t head0;
     const uint16_t* Bv;     // [RB][D] bf16 in shared memory
     const uint16_t* Rv;     // [16][D] bf16 in shared memory
-    __device__ void operator()(const float* v, const float* l, const float* m) const {
+    __device__ void operator()(const float* v, const float* l, const float* lx, const float* m) const {
         constexpr int PDV = RB + RM;
         for (int idx = threadIdx.x; idx < a.g * D; idx += blockDim.x) {
             const int h = idx / D;
@@ -91,9 +91,9 @@ struct EmitProject {
             for (int i = 0; i < RB; ++i) acc += v[h * PDV + i] * bf16_lo(Bv[i * D + e]);
 #pragma unroll
             for (int i = 0; i < RM; ++i) acc += v[h * PDV + RB + i] * bf16_lo(Rv[i * D + e]);
-            a.out[(head0 + h) * D + e] = acc / l[h];
+            a.out[(head0 + h) * D + e] = l[h] > 0.f ? acc / l[h] : 0.f;
         }
-        if (a.lse != nullptr && threadIdx.x < a.g) a.lse[head0 + threadIdx.x] = (m[threadIdx.x] + log2f(l[threadIdx.x])) * LN2_F;
+        if (a.lse != nullptr && threadIdx.x < a.g) a.lse[head0 + threadIdx.x] = lse_of(m[threadIdx.x], lx[threadIdx.x]);
     }
 };
 
@@ -129,9 +129,11 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int g = a.g;
-    const int ntiles = (a.T + TT - 1) / TT;
     const int tile0 = split * a.tiles_per_split;
-    const int tile1 = min(tile0 + a.tiles_per_split, ntiles);
+    // the sequence's own tokens; with per-sequence lengths they are read where the first
+    // tiles are requested (before the dependent-launch wait only under kv_early)
+    int tlen = a.T;
+    int tile1 = tile0;
     const int crow = (a.pair * a.B + b) * a.Hkv + j;        // coefficient row in [P*B*Hkv]
     const int urow = b * a.Hkv + j;                         // code row within the layer's [B*Hkv]
     const size_t tokrow = static_cast<size_t>(b * a.Hkv + j) * a.T;   // s_K / s_V row start
@@ -152,8 +154,13 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     __syncthreads();   // every warp's ring barriers are initialised before any warp issues
     uint8_t* ring = smem + warp * NSW * C::STAGE_BYTES;
     uint64_t* wb = &bars[warp * NSW];
-    const int span = tile1 - tile0;
-    const int my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
+    int my_n = 0;
+    auto set_range = [&] {
+        tlen = seq_len(a, b);
+        tile1 = min(tile0 + a.tiles_per_split, (tlen + TT - 1) / TT);
+        const int span = tile1 - tile0;
+        my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
+    };
 
     auto issue = [&](int k) {
         const int t = tile0 + warp + k * NW;
@@ -178,7 +185,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
 #pragma unroll
         for (int u = 0; u < TPL; ++u) {
             const int t = t0 + lane + 32 * u;
-            if (t < a.T) {
+            if (t < tlen) {
                 pf_sk[u] = __ldg(a.s_k + tokrow + t);
                 pf_sv[u] = __ldg(a.s_v + tokrow + t);
                 pf_r[u] = __ldg(rank_row + t);
@@ -210,10 +217,18 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         __syncwarp();
         if (my_n > 0) prefetch(0);
     };
-    if (a.kv_early) request_cache();
+    if (a.kv_early) {
+        set_range();
+        request_cache();
+    }
     grid_dep_wait();
     if (threadIdx.x == 0) grid_dep_launch();
-    if (!a.kv_early) request_cache();
+    if (!a.kv_early) {
+        set_range();
+        request_cache();
+    }
+    float* srow = a.sscore != nullptr ? a.sscore + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g) * a.T
+                                      : nullptr;
     if (threadIdx.x == 0) bulk_load(stagebuf + C::STAGE_FACTORS, qsrc, g * D * 2, &fac_bar[0]);
     for (int idx = g * C::PD + threadIdx.x; idx < 16 * C::PD; idx += blockDim.x) qproj[idx] = 0.f;
     // ---- q~ = B_K q and q^ = R_K q for the g heads: one thread per output; lane l starts
@@ -288,9 +303,12 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         for (int i = 0; i < RB / 16; ++i) oc[i][nb][0] = oc[i][nb][1] = oc[i][nb][2] = oc[i][nb][3] = 0.f;
         ou[nb][0] = ou[nb][1] = ou[nb][2] = ou[nb][3] = 0.f;
     }
-    float mrow[NB][2], lrow[NB][2];
+    float mrow[NB][2], lrow[NB][2], lxrow[NB][2];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) mrow[nb][0] = mrow[nb][1] = NEG_INF, lrow[nb][0] = lrow[nb][1] = 0.f;
+    for (int nb = 0; nb < NB; ++nb) {
+        mrow[nb][0] = mrow[nb][1] = NEG_INF;
+        lrow[nb][0] = lrow[nb][1] = lxrow[nb][0] = lxrow[nb][1] = 0.f;
+    }
 
     float* tks = tok + warp * TT * 3;     // [3][TT]: s_K, s_V, rank
     int* tkr = reinterpret_cast<int*>(tks + 2 * TT);
@@ -322,6 +340,15 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             break;
         }
         const int t = tile0 + warp + k * NW;
+        if (a.lens != nullptr && (t + 1) * TT > tlen) {
+            // V coefficients past the sequence (the K side is masked by score)
+            if (RB == 32)
+                zero_tile_rows(ring + s * C::STAGE_BYTES + C::COEF_BYTES, 64, 1, 0, tlen - t * TT, TT, lane);
+            else
+                zero_tile_rows(ring + s * C::STAGE_BYTES + C::COEF_BYTES, 128, LY::HALVES, TT * 128, tlen - t * TT, TT,
+                               lane);
+            __syncwarp();
+        }
         const uint32_t ckb = smem_u32(ring + s * C::STAGE_BYTES);
         const uint32_t cvb = ckb + C::COEF_BYTES;
         const uint8_t* ukp = ring + s * C::STAGE_BYTES + C::OFF_UK;
@@ -386,8 +413,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         }
         // ---- scores, mask, online softmax per head; P^T and (P s_V)^T by movmatrix
         uint32_t pb[MT][NB][2], pvb[MT][NB][2];
-        const bool tail = (t + 1) * TT > a.T;       // only the last tile holds tokens past T
-        const int lim = a.T - t * TT;
+        const bool tail = (t + 1) * TT > tlen;       // only the last tile holds tokens past the sequence
+        const int lim = tlen - t * TT;
         float skr[MT][2];                            // s_K of this lane's two rows per m tile
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
@@ -409,6 +436,18 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                     for (int i = 0; i < 4; ++i)
                         if (mt * 16 + (lane >> 2) + (i >> 1) * 8 >= lim) sc[mt][nb][i] = NEG_INF;
             }
+            if (srow != nullptr) {
+                // keep the scores of the tile's valid tokens for the attention statistics
+                const int h0 = nb * 8 + 2 * q4;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int h = h0 + (i & 1);
+                        const int r = mt * 16 + (lane >> 2) + (i >> 1) * 8;
+                        if (h < g && r < lim) srow[static_cast<size_t>(h) * a.T + t * TT + r] = sc[mt][nb][i];
+                    }
+            }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 mx0 = fmaxf(mx0, fmaxf(sc[mt][nb][0], sc[mt][nb][2]));
@@ -427,6 +466,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             mrow[nb][1] = mn1;
             lrow[nb][0] *= cr0;
             lrow[nb][1] *= cr1;
+            lxrow[nb][0] *= cr0;
+            lxrow[nb][1] *= cr1;
 #pragma unroll
             for (int i = 0; i < RB / 16; ++i) { oc[i][nb][0] *= cr0; oc[i][nb][2] *= cr0; oc[i][nb][1] *= cr1; oc[i][nb][3] *= cr1; }
             ou[nb][0] *= cr0; ou[nb][2] *= cr0; ou[nb][1] *= cr1; ou[nb][3] *= cr1;
@@ -438,6 +479,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 const uint32_t lo = pack_bf16(p0, p1), hi = pack_bf16(p2, p3);
                 lrow[nb][0] += bf16_lo(lo) + bf16_lo(hi);
                 lrow[nb][1] += bf16_hi(lo) + bf16_hi(hi);
+                lxrow[nb][0] += p0 + p2;
+                lxrow[nb][1] += p1 + p3;
                 pb[mt][nb][0] = movmatrix_t(lo);
                 pb[mt][nb][1] = movmatrix_t(hi);
                 const float sva = tks[TT + ta], svb = tks[TT + ta + 8];
@@ -479,6 +522,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         for (int off = 4; off < 32; off <<= 1) {
             lrow[nb][0] += __shfl_xor_sync(0xffffffffu, lrow[nb][0], off);
             lrow[nb][1] += __shfl_xor_sync(0xffffffffu, lrow[nb][1], off);
+            lxrow[nb][0] += __shfl_xor_sync(0xffffffffu, lxrow[nb][0], off);
+            lxrow[nb][1] += __shfl_xor_sync(0xffffffffu, lxrow[nb][1], off);
         }
 
     // ---- merge warps in coefficient space, project once, finish the split
@@ -490,9 +535,11 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     float* comb = reinterpret_cast<float*>(smem);   // [NW][16][PD]
     float* comb_m = comb + NW * 16 * PD;
     float* comb_l = comb_m + NW * 16;
-    float* fin_m = comb_l + NW * 16;
+    float* comb_lx = comb_l + NW * 16;
+    float* fin_m = comb_lx + NW * 16;
     float* fin_l = fin_m + 16;
-    float* fin_c = fin_l + 16;                      // [16][PD]
+    float* fin_lx = fin_l + 16;
+    float* fin_c = fin_lx + 16;                     // [16][PD]
     float* fin_o = fin_c + 16 * PD;                 // [16][D]
     float* scratch = fin_o + 16 * D;
     {
@@ -516,6 +563,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 comb_m[warp * 16 + h0 + 1] = mrow[nb][1];
                 comb_l[warp * 16 + h0] = lrow[nb][0];
                 comb_l[warp * 16 + h0 + 1] = lrow[nb][1];
+                comb_lx[warp * 16 + h0] = lxrow[nb][0];
+                comb_lx[warp * 16 + h0 + 1] = lxrow[nb][1];
             }
         }
     }
@@ -526,22 +575,26 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         const int h = threadIdx.x;
         float M = NEG_INF;
         for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, comb_m[ww * 16 + h]);
-        float L = 0.f;
+        float L = 0.f, LX = 0.f;
         for (int ww = 0; ww < NW; ++ww) {
             const float m = comb_m[ww * 16 + h];
             const float f = m != NEG_INF ? ex2_approx(m - M) : 0.f;
             fac[ww][h] = f;
             L += f * comb_l[ww * 16 + h];
+            LX += f * comb_lx[ww * 16 + h];
         }
         fin_m[h] = M;
         fin_l[h] = L;
+        fin_lx[h] = LX;
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < g * PD; idx += blockDim.x) {
         const int h = idx / PD;
         float acc = 0.f;
+        // a warp without tokens left its slot unset: skip it, never 0 * x
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww) acc = fmaf(fac[ww][h], comb[(ww * 16 + h) * PD + (idx % PD)], acc);
+        for (int ww = 0; ww < NW; ++ww)
+            if (fac[ww][h] != 0.f) acc = fmaf(fac[ww][h], comb[(ww * 16 + h) * PD + (idx % PD)], acc);
         fin_c[idx] = acc;
     }
     __syncthreads();
@@ -553,7 +606,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     const int unit = b * a.Hkv + j;
     // the per-token and code-conversion buffers are free now: they stage the unit's partials
     finish_unit<(PD > D ? PD : D)>(a, PD, unit, split, a.splits, static_cast<long long>(unit) * a.splits, fin_m, fin_l,
-                                   fin_c, scratch,
+                                   fin_lx, fin_c, scratch,
                 reinterpret_cast<uint8_t*>(tok), C::TOK_BYTES + C::CVT_BYTES, emit);
 }
 

@@ -203,9 +203,41 @@ __device__ __forceinline__ uint32_t swz128(int row, int c) {
     return static_cast<uint32_t>(row * 128 + (((c ^ row) & 7) << 4));
 }
 
+// ------------------------------------------------------------------ sequence lengths
+// Tokens of sequence b: lens[b] clamped to [0, T] (a value outside records ERR_RANGE),
+// or every cached token without per-sequence lengths.
+__device__ __forceinline__ int seq_len(const DecodeArgs& a, int b) {
+    if (a.lens == nullptr) return a.T;
+    const int n = a.lens[b];
+    if (n < 0 || n > a.T) {
+        atomicOr(a.err, ERR_RANGE);
+        return n < 0 ? 0 : a.T;
+    }
+    return n;
+}
+
+// Zero rows [r0, rows) of a staged tile: `halves` blocks of `half_stride` bytes, each row
+// `row_bytes` contiguous bytes of every block (a swizzle only permutes 16-B chunks inside
+// a row). The values past a sequence's length in its last tile are whatever the cache
+// holds there, and a zero weight times a NaN is still NaN, so they are cleared before
+// the P.V product reads them. One warp; the caller syncs the warp afterwards.
+__device__ __forceinline__ void zero_tile_rows(uint8_t* base, int row_bytes, int halves, int half_stride, int r0,
+                                               int rows, int lane) {
+    const int chunks = row_bytes / 16;
+    const int n = (rows - r0) * chunks * halves;
+    for (int i = lane; i < n; i += 32) {
+        const int h = i / ((rows - r0) * chunks);
+        const int rem = i % ((rows - r0) * chunks);
+        *reinterpret_cast<uint4*>(base + h * half_stride + (r0 + rem / chunks) * row_bytes + (rem % chunks) * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
 // ------------------------------------------------------------------ split merge
-// Partial layout: [unit][split][head][D + 4] floats: o[0..D), m, l, two pad words
-// (rows stay 16-byte aligned so whole partial blocks can move by bulk copy).
+// Partial layout: [unit][split][head][D + 4] floats: o[0..D), m, l, lx, one pad word
+// (rows stay 16-byte aligned so whole partial blocks can move by bulk copy). l sums the
+// weights as the P.V products used them (rounded to the operand type), so o / l is a
+// convex combination of the values; lx sums the unrounded fp32 weights and gives the lse.
 __host__ __device__ constexpr int partial_width(int D) { return D + 4; }
 
 // 2^x by the MUFU unit (ex2.approx, flush-to-zero): one instruction; -inf gives 0.
@@ -228,28 +260,36 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Every decode CTA ends here with, in shared memory, for its g query heads:
 //   sm_m[h]  running max of the log2-domain scores,
-//   sm_l[h]  sum of 2^(s - m) weights,
+//   sm_l[h]  sum of 2^(s - m) weights as rounded for the P.V products,
+//   sm_lx[h] sum of the unrounded 2^(s - m) weights,
 //   sm_v[h][e] un-normalised accumulated vector (e < DV): the output
 //            sum_t 2^(s_t - m) V_t, or the low-rank form's coefficient-space sums.
 // With one partial per unit the CTA emits it at once. Otherwise it stores its
 // partial and the last CTA of the unit to arrive merges all partials:
-// M = max m_s, l = sum 2^(m_s - M) l_s, v = sum 2^(m_s - M) v_s, then emits
+// M = max m_s, l = sum 2^(m_s - M) l_s (lx likewise), v = sum 2^(m_s - M) v_s, then emits
 // (and resets the unit's arrival counter to zero). Arrival is one acq_rel
 // atomic per CTA. The last CTA bulk-copies the unit's partials (contiguous) into
 // `stage` (free shared memory of `stage_bytes`, 16-B aligned) in one copy when
 // they fit, in chunks otherwise (0 bytes: read them directly); one warp per head
 // reduces (m, l), then every thread combines its share of the vector.
-// `emit(v, l, m)` writes the unit's outputs from v [g][DV] (shared memory),
-// l[g] and m[g]; it is called by all threads of the CTA.
-// sm_scratch holds at least 2 * g * count floats; sm_v is reused for the merge.
+// `emit(v, l, lx, m)` writes the unit's outputs from v [g][DV] (shared memory),
+// l[g], lx[g] and m[g]; it is called by all threads of the CTA. A unit with no tokens
+// has l = 0: its outputs are 0 and its lse is -inf.
+// sm_scratch holds at least 3 * g * count floats; sm_v is reused for the merge.
+__device__ __forceinline__ float lse_of(float m, float lx) {
+    return lx > 0.f ? (m + log2f(lx)) * LN2_F : NEG_INF;
+}
+
 struct EmitPlain {
     const DecodeArgs& a;
     int D;
     size_t head0;
-    __device__ void operator()(const float* v, const float* l, const float* m) const {
-        for (int idx = threadIdx.x; idx < a.g * D; idx += blockDim.x)
-            a.out[(head0 + idx / D) * D + (idx % D)] = v[idx] / l[idx / D];
-        if (a.lse != nullptr && threadIdx.x < a.g) a.lse[head0 + threadIdx.x] = (m[threadIdx.x] + log2f(l[threadIdx.x])) * LN2_F;
+    __device__ void operator()(const float* v, const float* l, const float* lx, const float* m) const {
+        for (int idx = threadIdx.x; idx < a.g * D; idx += blockDim.x) {
+            const float lh = l[idx / D];
+            a.out[(head0 + idx / D) * D + (idx % D)] = lh > 0.f ? v[idx] / lh : 0.f;
+        }
+        if (a.lse != nullptr && threadIdx.x < a.g) a.lse[head0 + threadIdx.x] = lse_of(m[threadIdx.x], lx[threadIdx.x]);
     }
 };
 
@@ -257,13 +297,13 @@ struct EmitPlain {
 // MAX_GROUP * MAXDV / 128 merged values, as every caller runs at least 128 threads.
 template <int MAXDV = 128, typename Emit>
 __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int index, int count, long long slot0,
-                                   const float* sm_m, const float* sm_l, float* sm_v, float* sm_scratch,
-                                   uint8_t* stage, int stage_bytes, const Emit& emit) {
+                                   const float* sm_m, const float* sm_l, const float* sm_lx, float* sm_v,
+                                   float* sm_scratch, uint8_t* stage, int stage_bytes, const Emit& emit) {
     const int g = a.g;
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;
     if (count == 1) {
-        emit(sm_v, sm_l, sm_m);
+        emit(sm_v, sm_l, sm_lx, sm_m);
         return;
     }
     const int PD = partial_width(DV);
@@ -274,6 +314,7 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
     if (tid < g) {
         part[tid * PD + DV] = sm_m[tid];
         part[tid * PD + DV + 1] = sm_l[tid];
+        part[tid * PD + DV + 2] = sm_lx[tid];
     }
     __syncthreads();
     __shared__ unsigned s_is_last;
@@ -293,7 +334,8 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
     const float* base = a.ws + static_cast<size_t>(slot0) * per;
     float* fm = sm_scratch;            // [n][g]: m, then the factors 2^(m - M)
     float* fl = sm_scratch + n * g;    // [n][g]: l
-    __shared__ float hm[MAX_GROUP], hl[MAX_GROUP];
+    float* flx = fl + n * g;           // [n][g]: lx
+    __shared__ float hm[MAX_GROUP], hl[MAX_GROUP], hlx[MAX_GROUP];
     __shared__ __align__(8) uint64_t mbar;
     const int chunk = stage_bytes / (per * 4);
     float* sp_buf = reinterpret_cast<float*>(stage);
@@ -317,6 +359,7 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
             const int h = idx % g;
             fm[idx] = sp_buf[sp * per + h * PD + DV];
             fl[idx] = sp_buf[sp * per + h * PD + DV + 1];
+            flx[idx] = sp_buf[sp * per + h * PD + DV + 2];
         }
     } else {
         for (int idx = tid; idx < n * g; idx += nthr) {
@@ -324,6 +367,7 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
             const int h = idx % g;
             fm[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV);
             fl[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 1);
+            flx[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 2);
         }
     }
     __syncthreads();
@@ -332,16 +376,21 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         float M = NEG_INF;
         for (int sp = lane; sp < n; sp += 32) M = fmaxf(M, fm[sp * g + h]);
         M = warp_max(M);
-        float L = 0.f;
+        float L = 0.f, LX = 0.f;
         for (int sp = lane; sp < n; sp += 32) {
-            const float f = ex2_approx(fm[sp * g + h] - M);
+            // a split without tokens has m = -inf and weighs nothing (also when all do)
+            const float ms = fm[sp * g + h];
+            const float f = ms != NEG_INF ? ex2_approx(ms - M) : 0.f;
             fm[sp * g + h] = f;
             L += f * fl[sp * g + h];
+            LX += f * flx[sp * g + h];
         }
         L = warp_sum(L);
+        LX = warp_sum(LX);
         if (lane == 0) {
             hm[h] = M;
             hl[h] = L;
+            hlx[h] = LX;
         }
     }
     __syncthreads();
@@ -406,18 +455,18 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         if (idx < g * DV) sm_v[idx] = acc[k];
     }
     __syncthreads();
-    emit(sm_v, hl, hm);
+    emit(sm_v, hl, hlx, hm);
     if (tid == 0) a.counters[unit] = 0u;
 }
 
 // Split-grid kernels: CTA (split, j, b) holds partial `split` of `a.splits` for its unit.
 __device__ inline void finish_split(const DecodeArgs& a, int D, int b, int j, int split, const float* sm_m,
-                                    const float* sm_l, float* sm_o, float* sm_scratch, uint8_t* stage,
-                                    int stage_bytes) {
+                                    const float* sm_l, const float* sm_lx, float* sm_o, float* sm_scratch,
+                                    uint8_t* stage, int stage_bytes) {
     const int unit = b * a.Hkv + j;
     const EmitPlain emit{a, D, static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * a.g};
-    finish_unit(a, D, unit, split, a.splits, static_cast<long long>(unit) * a.splits, sm_m, sm_l, sm_o, sm_scratch,
-                stage, stage_bytes, emit);
+    finish_unit(a, D, unit, split, a.splits, static_cast<long long>(unit) * a.splits, sm_m, sm_l, sm_lx, sm_o,
+                sm_scratch, stage, stage_bytes, emit);
 }
 
 }  // namespace kvs

@@ -11,6 +11,7 @@ namespace kvs {
 
 // bits of the device status word
 constexpr unsigned ERR_TIMEOUT = 1u;
+constexpr unsigned ERR_RANGE = 2u;     // a per-sequence length outside [0, context] (clamped)
 
 // one split partial: o[d] (un-normalised, relative to m), m (log2 domain), l
 constexpr int MAX_SPLITS = 160;
@@ -25,13 +26,15 @@ struct DecodeArgs {
     const void* v;
     int src0, src1;         // slots (SINGLE/MIX)
     const float* w;         // [Hkv] mix weights of this layer (device), MIX only
-    int B, Hq, Hkv, T, g;
+    int B, Hq, Hkv, T, g;   // T: tokens each store holds (row stride of the cache)
+    const int* lens;        // [B] tokens of each sequence (device), or nullptr: all T
+    float* sscore;          // [B][Hq][T] log2-domain scaled scores for the statistics, or nullptr
     int splits;             // splits per (b, kv head)            (split-grid kernels)
     int tiles_per_split;    // token tiles per split               (split-grid kernels)
     int units;              // B * Hkv                             (balanced-grid kernels)
     int n_t;                // token tiles per unit                (balanced-grid kernels)
     float scale_log2;       // softmax scale * log2(e)
-    float* ws;              // split partials [B*Hkv][splits][g][d+2]
+    float* ws;              // split partials: [g][d + 4] each (o, m, l, lx, pad)
     unsigned* counters;     // [B*Hkv] arrival counters, zero between launches
     unsigned* err;          // device status word
     long long wait_limit;   // clock cycles a bounded wait may spin
@@ -86,6 +89,20 @@ inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, 
     cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
 }
+
+// Attention statistics of one decoded layer from its kept scores and lse.
+struct StatsArgs {
+    const float* sscore;    // [B][Hq][T] log2-domain scaled scores
+    const float* lse;       // [B][Hq] natural-log lse of the layer
+    const int* lens;        // [B] or nullptr
+    float* mass;            // [B][Hkv][T] or nullptr
+    float* score;           // [B][T] or nullptr
+    float* entropy;         // [B][Hq] or nullptr (zeroed before the launch)
+    float* peak;            // [B][Hq] or nullptr (zeroed before the launch)
+    unsigned* err;
+    int B, Hq, Hkv, T, g;
+};
+cudaError_t launch_router_stats(const StatsArgs& a, cudaStream_t st);
 
 struct PackArgs {
     const float* score; const float* u_k; const float* u_v;

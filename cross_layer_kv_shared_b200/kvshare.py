@@ -39,7 +39,8 @@ class kvshare_cache(ctypes.Structure):
                 ("s_k", ctypes.c_void_p), ("s_v", ctypes.c_void_p),
                 ("r_k", ctypes.c_void_p), ("r_v", ctypes.c_void_p),
                 ("rank", ctypes.c_void_p), ("pairs", ctypes.c_int),
-                ("batch", ctypes.c_int), ("context", ctypes.c_int)]
+                ("batch", ctypes.c_int), ("context", ctypes.c_int),
+                ("lengths", ctypes.c_void_p)]
 
 
 class KVShareError(RuntimeError):
@@ -59,6 +60,7 @@ def _load():
         "kvshare_set_map": ([P, ctypes.POINTER(kvshare_layer), P], I),
         "kvshare_decode": ([P, ctypes.POINTER(kvshare_cache), P, P, P, I, I, V], I),
         "kvshare_decode_host": ([P, ctypes.POINTER(kvshare_cache), P, P, P, I, I, V], I),
+        "kvshare_decode_stats": ([P, ctypes.POINTER(kvshare_cache), P, P, P, P, P, P, P, I, I, V], I),
         "kvshare_prefill": ([P, ctypes.POINTER(kvshare_cache), P, P, P, I, I, I, V], I),
         "kvshare_pack_residual": ([P, P, P, P, P, P, P, P, P, I, I, V], I),
         "kvshare_sync_status": ([P, V], I),
@@ -156,12 +158,13 @@ class Cache:
     r_v: object = None
     rank: object = None
     pairs: int = 0
+    lengths: object = None      # [batch] int32 device tensor of per-sequence token counts
 
     def as_c(self) -> kvshare_cache:
         p = lambda t: _ptr(t) or None  # noqa: E731
         return kvshare_cache(p(self.k), p(self.v), self.slots, p(self.coef_k), p(self.coef_v), p(self.basis_k),
                              p(self.basis_v), p(self.u_k), p(self.u_v), p(self.s_k), p(self.s_v), p(self.r_k),
-                             p(self.r_v), p(self.rank), self.pairs, self.batch, self.context)
+                             p(self.r_v), p(self.rank), self.pairs, self.batch, self.context, p(self.lengths))
 
 
 def kvshare_decode(h, cache: Cache, q, out, lse=None, l0: int = 0, l1: int = None, stream=None,
@@ -171,6 +174,17 @@ def kvshare_decode(h, cache: Cache, q, out, lse=None, l0: int = 0, l1: int = Non
                              int(l1 if l1 is not None else q.shape[0]), _stream(stream))
     if check:
         _check(st, "kvshare_decode")
+    return st
+
+
+def kvshare_decode_stats(h, cache: Cache, q, out, lse, mass=None, score=None, entropy=None, peak=None,
+                         l0: int = 0, l1: int = None, stream=None, check: bool = True) -> int:
+    c = cache.as_c()
+    st = _lib.kvshare_decode_stats(h, ctypes.byref(c), _ptr(q), _ptr(out), _ptr(lse), _ptr(mass), _ptr(score),
+                                   _ptr(entropy), _ptr(peak), int(l0), int(l1 if l1 is not None else q.shape[0]),
+                                   _stream(stream))
+    if check:
+        _check(st, "kvshare_decode_stats")
     return st
 
 

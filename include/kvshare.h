@@ -23,7 +23,8 @@
  *                    by Sharing Across Layers and Adapting Per Token", Core
  *                    Mechanism and Framework Shift).
  *
- * Decode: the query attends to all `context` cached tokens. Prefill: query row i
+ * Decode: the query attends to the cached tokens of its sequence (all `context`
+ * of them, or its own length, see kvshare_cache.lengths). Prefill: query row i
  * attends to tokens 0..i (causal, no earlier context).
  *
  * Conventions for every entry point
@@ -104,7 +105,14 @@ typedef struct {
     const uint8_t* rank;   /* [L][batch][T] per-token residual rank, <= Rm       */
     int pairs;
     int batch;             /* 1 .. max_batch                                     */
-    int context;           /* 1 .. max_context                                   */
+    int context;           /* 1 .. max_context: tokens every store holds (T)      */
+    const int* lengths;    /* [batch] int32 DEVICE array or NULL: sequence b's own
+                              token count n_b in [0, T]; decode attends to tokens
+                              0 .. n_b - 1 only, and a sequence with n_b = 0 gets
+                              out 0 and lse -inf. The values are read on the device:
+                              one outside [0, T] is clamped and makes the next
+                              kvshare_sync_status return KVS_EINVAL. NULL: every
+                              sequence has T tokens. Prefill takes NULL only. */
 } kvshare_cache;
 
 /* Create a context on the current CUDA device. Allocates the split workspace
@@ -137,6 +145,29 @@ kvshare_status kvshare_set_map(kvshare_t ctx, const kvshare_layer* map, const fl
  * the context's workspace; results agree to fp32 rounding whatever the split. */
 kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const void* q,
                               float* out, float* lse, int l0, int l1, void* stream);
+
+/* kvshare_decode plus the attention statistics the online rank router reads
+ * ("DepthWeave-KV: Smarter KV Cache Compression by Sharing Across Layers and
+ * Adapting Per Token", Core Mechanism, second component: attention statistics,
+ * entropy and peak, read online per token and step). With p_{h,t} the softmax
+ * weight of query head h on cached token t (exactly what kvshare_decode attends
+ * with), for each layer of [l0, l1):
+ *   mass    [L][batch][Hkv][T] fp32: sum of p_{h,t} over the g query heads of kv
+ *           head j (sums to g over t; 0 past a sequence's length)
+ *   score   [L][batch][T] fp32 router score of token t: x / (1 + x) with
+ *           x = (n_b * sum_j mass[j][t]) / Hq, evaluated in fp32 in that order
+ *           (sum over j from 0 up, each operation correctly rounded); a token at
+ *           the uniform share 1/n_b scores 0.5. kvshare_pack_residual maps it to a
+ *           rank: 8 from 7/3 times the uniform share, 16 from 9 times.
+ *   entropy [L][batch][Hq] fp32: -sum_t p ln p (nats) per query head
+ *   peak    [L][batch][Hq] fp32: max_t p per query head
+ * Any of the four may be NULL; lse is required. Entropy is summed with atomics, so
+ * its last bits can differ from run to run. The first call with an output allocates
+ * a score buffer of max_batch x Hq x max_context floats in the context (KVS_ENOMEM
+ * if that fails); each layer adds one statistics kernel after its decode kernel. */
+kvshare_status kvshare_decode_stats(kvshare_t ctx, const kvshare_cache* cache, const void* q, float* out,
+                                    float* lse, float* mass, float* score, float* entropy, float* peak,
+                                    int l0, int l1, void* stream);
 
 /* kvshare_decode with HOST buffers: copies q for layers [l0, l1) from
  * `q_host` into a device staging buffer the context owns, decodes, and copies
@@ -186,7 +217,8 @@ kvshare_status kvshare_pack_residual(kvshare_t ctx, const float* score, const fl
                                      void* stream);
 
 /* Synchronise `stream`, then read and clear the device status word.
- * Returns KVS_OK, KVS_ETIMEOUT (a bounded device wait ran out) or KVS_ECUDA. */
+ * Returns KVS_OK, KVS_ETIMEOUT (a bounded device wait ran out), KVS_EINVAL (a
+ * per-sequence length outside [0, context] was clamped) or KVS_ECUDA. */
 kvshare_status kvshare_sync_status(kvshare_t ctx, void* stream);
 
 /* Split-KV override for decode: 0 = automatic (default), n > 0 = n splits per

@@ -64,6 +64,30 @@ def lowrank_unit(cfg_name, l, j):
     return o, lse, r, codes_k, codes_v, sck, scv
 
 
+def lowrank_stats_unit(cfg_name, l, j):
+    """Attention statistics of layer l, kv head j at batch 0 of a named low-rank workload
+    (codes and scales from the host packer): (mass [T], entropy [g], peak [g])."""
+    from oracle import kvshare_ref as ref
+    from oracle import quant_ref as qr
+    from oracle import router_ref as rr
+    from synth.configs import BY_NAME
+    cfg = BY_NAME[cfg_name]
+    p = l // 2
+    g = cfg.group
+    r = qr.route_rank(cfg.make("score", (l, 0)))
+    kv = []
+    for s in ("k", "v"):
+        codes, sc = qr.quantize(cfg.make("u_" + s, (l, 0, j)), r)
+        kv.append(ref.kv_lowrank(ref.bf16_bits_to_f64(cfg.make("coef_" + s, (p, 0, j))),
+                                 ref.bf16_bits_to_f64(cfg.make("basis_" + s, (p, j))),
+                                 ref.f16_bits_to_f64(sc), codes.astype(np.float64),
+                                 ref.bf16_bits_to_f64(cfg.make("r_" + s, (l, j))), r))
+    q = ref.bf16_bits_to_f64(cfg.make("q", (l, 0))[j * g:(j + 1) * g])
+    _, _, pw = ref.attend(q, kv[0], kv[1], 1 / np.sqrt(cfg.head_dim))
+    ent, peak = rr.attention_stats(pw)
+    return rr.kv_mass(pw, g)[0], ent, peak
+
+
 # ---------------------------------------------------------------- causal prefill
 def prefill_unit(cfg_name, l, b, h, rows):
     """(o [n][d], lse [n]) of prefill layer l, batch b, q head h at the given rows."""
