@@ -14,6 +14,9 @@ Modules
 ``router_ref``   attention statistics of a decode step (per-head entropy and
                  peak, per-kv-head attention mass each cached token receives)
                  and the fp32 router score that feeds the rank rule.
+``encode_ref``   the write side of the low-rank form for one new token: shared
+                 coefficients (bf16) from the pair's basis, each layer's residual
+                 coordinates, in a stated fp32 order; a calibration basis fit.
 ``quant_ref``    the write side of the low-rank form: per-token rank routing and
                  symmetric int8 quantisation with an fp16 per-token scale,
                  evaluated in fp32 with correctly rounded IEEE operations.
@@ -21,4 +24,4 @@ Modules
 Every function is pinned by tests under ``tests/`` against closed forms,
 invariants, a library routine (torch SDPA in fp64) or high-precision brute force.
 """
-from . import kvshare_ref, quant_ref, router_ref  # noqa: F401
+from . import encode_ref, kvshare_ref, quant_ref, router_ref  # noqa: F401
