@@ -760,6 +760,72 @@ kvshare_status kvshare_pack_residual(kvshare_t ctx, const float* score, const fl
     return KVS_OK;
 }
 
+kvshare_status kvshare_append_lowrank(kvshare_t ctx, const kvshare_cache* cache, const void* k_new, const void* v_new,
+                                      const float* score, const int* pos, void* stream) {
+    if (ctx == nullptr || !ctx->map_set) return KVS_EINVAL;
+    kvshare_status s = validate_cache_common(ctx, cache);
+    if (s != KVS_OK) return s;
+    const kvshare_config& cf = ctx->cfg;
+    if (cf.dtype != KVS_BF16) return KVS_EUNSUPPORTED;
+    if (cache->pairs < 1 || cache->pairs > APPEND_MAX_PAIRS) return cache->pairs < 1 ? KVS_EINVAL : KVS_EUNSUPPORTED;
+    AppendArgs a;
+    std::memset(&a, 0, sizeof(a));
+    for (int i = 0; i < 2 * APPEND_MAX_PAIRS; ++i) a.pair_layers[i] = -1;
+    bool any = false;
+    for (int l = 0; l < cf.num_layers; ++l) {
+        const kvshare_layer& e = ctx->map[l];
+        if (e.kind != KVS_SRC_LOWRANK) continue;
+        if (e.src0 < 0 || e.src0 >= cache->pairs) return KVS_EINVAL;
+        int* pl = &a.pair_layers[2 * e.src0];
+        if (pl[0] < 0) {
+            pl[0] = pl[1] = l;
+        } else if (pl[1] == pl[0]) {
+            pl[1] = l;
+        } else {
+            return KVS_EUNSUPPORTED;   // a basis shared by more than two layers
+        }
+        any = true;
+    }
+    if (!any) return KVS_EINVAL;
+    const void* ins[] = {k_new, v_new};
+    for (const void* p : ins)
+        if (!dev_ok(p)) return KVS_EINVAL;
+    const void* small[] = {score, pos};
+    for (const void* p : small)
+        if (p == nullptr || !is_device_ptr(p) || (reinterpret_cast<uintptr_t>(p) & 3u)) return KVS_EINVAL;
+    const void* cs[] = {cache->coef_k, cache->coef_v, cache->basis_k, cache->basis_v, cache->u_k, cache->u_v,
+                        cache->s_k, cache->s_v, cache->r_k, cache->r_v, cache->rank};
+    for (const void* p : cs)
+        if (!dev_ok(p)) return KVS_EINVAL;
+    if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
+    a.k_new = static_cast<const uint16_t*>(k_new);
+    a.v_new = static_cast<const uint16_t*>(v_new);
+    a.score = score;
+    a.pos = pos;
+    a.basis_k = static_cast<const uint16_t*>(cache->basis_k);
+    a.basis_v = static_cast<const uint16_t*>(cache->basis_v);
+    a.r_k = static_cast<const uint16_t*>(cache->r_k);
+    a.r_v = static_cast<const uint16_t*>(cache->r_v);
+    // the cache arrays the decode reads are the ones the append writes
+    a.coef_k = static_cast<uint16_t*>(const_cast<void*>(cache->coef_k));
+    a.coef_v = static_cast<uint16_t*>(const_cast<void*>(cache->coef_v));
+    a.u_k = const_cast<int8_t*>(cache->u_k);
+    a.u_v = const_cast<int8_t*>(cache->u_v);
+    a.s_k = const_cast<uint16_t*>(cache->s_k);
+    a.s_v = const_cast<uint16_t*>(cache->s_v);
+    a.rank = const_cast<uint8_t*>(cache->rank);
+    a.err = ctx->err;
+    a.P = cache->pairs;
+    a.B = cache->batch;
+    a.Hkv = cf.num_kv_heads;
+    a.T = cache->context;
+    a.d = cf.head_dim;
+    a.Rb = cf.basis_rank;
+    if (launch_append_lowrank(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return KVS_ECUDA;
+    ++ctx->launches;
+    return KVS_OK;
+}
+
 kvshare_status kvshare_sync_status(kvshare_t ctx, void* stream) {
     if (ctx == nullptr) return KVS_EINVAL;
     if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;

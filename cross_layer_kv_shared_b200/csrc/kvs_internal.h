@@ -104,6 +104,24 @@ struct StatsArgs {
 };
 cudaError_t launch_router_stats(const StatsArgs& a, cudaStream_t st);
 
+// Append of one new token to a low-rank cache (every basis pair, sequence and kv head).
+constexpr int APPEND_MAX_PAIRS = 64;
+struct AppendArgs {
+    const uint16_t* k_new; const uint16_t* v_new;   // [L][B][Hkv][d] bf16: the token in every layer
+    const float* score;                             // [L][B] router score of the token per layer
+    const int* pos;                                 // [B] token index written in each sequence
+    const uint16_t* basis_k; const uint16_t* basis_v;   // [P][Hkv][Rb][d]
+    const uint16_t* r_k; const uint16_t* r_v;           // [L][Hkv][16][d]
+    uint16_t* coef_k; uint16_t* coef_v;                 // [P][B][Hkv][T][Rb]
+    int8_t* u_k; int8_t* u_v;                           // [L][B][Hkv][T][16]
+    uint16_t* s_k; uint16_t* s_v;                       // [L][B][Hkv][T]
+    uint8_t* rank;                                      // [L][B][T]
+    unsigned* err;
+    int P, B, Hkv, T, d, Rb;
+    int pair_layers[2 * APPEND_MAX_PAIRS];              // the two layers of each pair (-1: unused)
+};
+cudaError_t launch_append_lowrank(const AppendArgs& a, cudaStream_t st);
+
 struct PackArgs {
     const float* score; const float* u_k; const float* u_v;
     uint8_t* rank; int8_t* u_k8; int8_t* u_v8; uint16_t* s_k; uint16_t* s_v;

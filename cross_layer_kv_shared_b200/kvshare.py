@@ -63,6 +63,7 @@ def _load():
         "kvshare_decode_stats": ([P, ctypes.POINTER(kvshare_cache), P, P, P, P, P, P, P, I, I, V], I),
         "kvshare_prefill": ([P, ctypes.POINTER(kvshare_cache), P, P, P, I, I, I, V], I),
         "kvshare_pack_residual": ([P, P, P, P, P, P, P, P, P, I, I, V], I),
+        "kvshare_append_lowrank": ([P, ctypes.POINTER(kvshare_cache), P, P, P, P, V], I),
         "kvshare_sync_status": ([P, V], I),
         "kvshare_set_splits": ([P, I], I),
         "kvshare_set_kv_overlap": ([P, I], I),
@@ -215,6 +216,15 @@ def kvshare_pack_residual(h, score, u_k, u_v, rank, u_k8, u_v8, s_k, s_v, batch:
                                     _ptr(s_k), _ptr(s_v), int(batch), int(context), _stream(stream))
     if check:
         _check(st, "kvshare_pack_residual")
+    return st
+
+
+def kvshare_append_lowrank(h, cache: Cache, k_new, v_new, score, pos, stream=None, check: bool = True) -> int:
+    c = cache.as_c()
+    st = _lib.kvshare_append_lowrank(h, ctypes.byref(c), _ptr(k_new), _ptr(v_new), _ptr(score), _ptr(pos),
+                                     _stream(stream))
+    if check:
+        _check(st, "kvshare_append_lowrank")
     return st
 
 

@@ -216,6 +216,31 @@ kvshare_status kvshare_pack_residual(kvshare_t ctx, const float* score, const fl
                                      uint16_t* s_k, uint16_t* s_v, int batch, int context,
                                      void* stream);
 
+/* Append one new token to the form-(c) arrays of `cache`, in place (the read-only
+ * fields of kvshare_cache are written here: coef_k/v, u_k/v, s_k/v, rank). A layer
+ * pair shares a low-rank basis and each layer keeps a light quantised residual
+ * ("DepthWeave-KV: Smarter KV Cache Compression by Sharing Across Layers and
+ * Adapting Per Token", Core Mechanism, first component and diagram). For every
+ * basis pair p of the layer table (its one or two LOWRANK layers la, lb), sequence
+ * b and kv head j, at token index t = pos[b], for K and for V:
+ *   m = (k_la + k_lb) * 0.5, c = B_p m, coef[p][b][j][t] = bf16_rne(c)
+ *   e_a = k_a - B_p^T coef,  u_a = R_a e_a  (16 values) for a = la, lb
+ *   rank[a][b][t] = 0 / 8 / 16 for score[a][b] below 0.7f / below 0.9f / above;
+ *   codes and scale of u_a at that rank as in kvshare_pack_residual.
+ * Every dot product is fp32 from index 0 up with each product and sum correctly
+ * rounded (no fused multiply-add), so coefficients and codes are bit-reproducible.
+ *   k_new, v_new: [L][batch][Hkv][d] bf16 DEVICE: the token's key and value in
+ *                 every layer (rows of non-LOWRANK layers are not read)
+ *   score:        [L][batch] fp32 DEVICE router score of the token per layer
+ *   pos:          [batch] int32 DEVICE token index to write; an index outside
+ *                 [0, context) writes nothing for that sequence and makes the next
+ *                 kvshare_sync_status return KVS_EINVAL.
+ * The caller then raises the sequences' lengths. A basis pair read by more than two
+ * layers, or more than 64 pairs: KVS_EUNSUPPORTED. A decode that follows an append
+ * on the same stream must run with kvshare_set_kv_overlap off. */
+kvshare_status kvshare_append_lowrank(kvshare_t ctx, const kvshare_cache* cache, const void* k_new,
+                                      const void* v_new, const float* score, const int* pos, void* stream);
+
 /* Synchronise `stream`, then read and clear the device status word.
  * Returns KVS_OK, KVS_ETIMEOUT (a bounded device wait ran out), KVS_EINVAL (a
  * per-sequence length outside [0, context] was clamped) or KVS_ECUDA. */
