@@ -97,6 +97,8 @@ struct kvshare_ctx {
     std::unordered_map<MapKey, CUtensorMap, MapKeyHash> maps;
     // kept scores of one layer for the attention statistics [max_batch][Hq][max_context]
     float* sscore = nullptr;
+    // projected queries of one low-rank prefill layer [max_batch][Hq][max_context][64] bf16
+    uint16_t* qp = nullptr;
     // staging for kvshare_decode_host
     void* q_stage = nullptr;
     float* out_stage = nullptr;
@@ -115,10 +117,13 @@ size_t elem_size(kvshare_dtype t) { return t == KVS_F32 ? 4 : 2; }
 
 kvshare_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVS_OK : KVS_ECUDA; }
 
-// 3-D tiled map over [rows][T][inner] elements, box {box0, tt, 1}.
+// 3-D tiled map over [rows][T][inner] elements, box {box0, tt, 1}; rows are `pitch`
+// tokens apart (0: T), so a map may end before the store does.
 bool get_map(kvshare_ctx* c, const void* base, CUtensorMapDataType dt, int esize, int inner, int T, int rows,
-             int box0, int tt, CUtensorMapSwizzle sw, CUtensorMap* out) {
-    MapKey key{base, (uint64_t)inner, (uint64_t)T, (uint64_t)rows, (uint32_t)box0, (uint32_t)tt, (int)dt, (int)sw};
+             int box0, int tt, CUtensorMapSwizzle sw, CUtensorMap* out, int pitch = 0) {
+    if (pitch == 0) pitch = T;
+    MapKey key{base, (uint64_t)inner, (uint64_t)T | (static_cast<uint64_t>(pitch) << 32), (uint64_t)rows,
+               (uint32_t)box0, (uint32_t)tt, (int)dt, (int)sw};
     auto it = c->maps.find(key);
     if (it != c->maps.end()) {
         *out = it->second;
@@ -128,7 +133,7 @@ bool get_map(kvshare_ctx* c, const void* base, CUtensorMapDataType dt, int esize
     if (fn == nullptr) return false;
     CUtensorMap m;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)T, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)inner * esize, (cuuint64_t)T * inner * esize};
+    cuuint64_t strides[2] = {(cuuint64_t)inner * esize, (cuuint64_t)pitch * inner * esize};
     cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)tt, 1u};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     CUresult r = fn(&m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
@@ -411,6 +416,63 @@ kvshare_status validate_decode(kvshare_ctx* c, const kvshare_cache* k, const voi
     return KVS_OK;
 }
 
+// One low-rank layer of a prefill: the query projection pre-pass, then the tcgen05 kernel.
+// The K/V operand maps end at seqlen, so rows past the sequence arrive as zeros.
+kvshare_status prefill_lowrank_layer(kvshare_ctx* ctx, const kvshare_cache* cache, const void* q, void* out,
+                                     float* lse, int l, int seqlen, cudaStream_t st) {
+    const kvshare_config& cf = ctx->cfg;
+    const kvshare_layer& e = ctx->map[l];
+    const int D = cf.head_dim, B = cache->batch, Hq = cf.num_q_heads, Hkv = cf.num_kv_heads, T = cache->context;
+    const size_t per_layer = static_cast<size_t>(B) * Hq * seqlen;
+    const size_t BHT = static_cast<size_t>(B) * Hkv * T;
+    PrefillLrArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = static_cast<const uint16_t*>(q) + static_cast<size_t>(l) * per_layer * D;
+    a.qp = ctx->qp;
+    a.lse = lse ? lse + static_cast<size_t>(l) * per_layer : nullptr;
+    a.basis_k = static_cast<const uint16_t*>(cache->basis_k) + static_cast<size_t>(e.src0) * Hkv * 32 * D;
+    a.basis_v = static_cast<const uint16_t*>(cache->basis_v) + static_cast<size_t>(e.src0) * Hkv * 32 * D;
+    a.r_k = static_cast<const uint16_t*>(cache->r_k) + static_cast<size_t>(l) * Hkv * 16 * D;
+    a.r_v = static_cast<const uint16_t*>(cache->r_v) + static_cast<size_t>(l) * Hkv * 16 * D;
+    a.s_k = cache->s_k + static_cast<size_t>(l) * BHT;
+    a.s_v = cache->s_v + static_cast<size_t>(l) * BHT;
+    a.rank = cache->rank + static_cast<size_t>(l) * B * T;
+    a.pair = e.src0;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.S = seqlen;
+    a.T = T;
+    a.g = Hq / Hkv;
+    a.d = D;
+    a.scale_log2 = ctx->scale * 1.4426950408889634f;
+    a.err = ctx->err;
+    a.wait_limit = ctx->wait_limit;
+    const int8_t* uk = cache->u_k + static_cast<size_t>(l) * BHT * 16;
+    const int8_t* uv = cache->u_v + static_cast<size_t>(l) * BHT * 16;
+    void* o = static_cast<uint16_t*>(out) + static_cast<size_t>(l) * per_layer * D;
+    const int crows = cache->pairs * B * Hkv;
+    CUtensorMap maps[6];
+    if (!get_map(ctx, ctx->qp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, LR_QW, seqlen, B * Hq, 64, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B, &maps[0]) ||
+        !get_map(ctx, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, seqlen, B * Hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B,
+                 &maps[1]) ||
+        !get_map(ctx, cache->coef_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, seqlen, crows, 32, 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE, &maps[2], T) ||
+        !get_map(ctx, cache->coef_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, seqlen, crows, 32, 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE, &maps[3], T) ||
+        !get_map(ctx, uk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, seqlen, B * Hkv, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE,
+                 &maps[4], T) ||
+        !get_map(ctx, uv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, seqlen, B * Hkv, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE,
+                 &maps[5], T))
+        return KVS_ECUDA;
+    if (launch_lr_qproj(a, st) != cudaSuccess) return KVS_ECUDA;
+    ++ctx->launches;
+    if (launch_prefill_lowrank(D, maps, a, st) != cudaSuccess) return KVS_ECUDA;
+    ++ctx->launches;
+    return KVS_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -482,6 +544,7 @@ kvshare_status kvshare_destroy(kvshare_t ctx) {
     cudaFree(ctx->err);
     cudaFree(ctx->w_dev);
     cudaFree(ctx->sscore);
+    cudaFree(ctx->qp);
     cudaFree(ctx->q_stage);
     cudaFree(ctx->out_stage);
     cudaFree(ctx->lse_stage);
@@ -676,8 +739,9 @@ kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const 
     if (!dev_ok(q) || !dev_ok(out) || (lse != nullptr && (!is_device_ptr(lse) || (reinterpret_cast<uintptr_t>(lse) & 3u))))
         return KVS_EINVAL;
     bool need_kv = false, need_lr = false;
+    if (cf.dtype != KVS_BF16) return KVS_EUNSUPPORTED;
     for (int l = l0; l < l1; ++l)
-        if (ctx->map[l].kind == KVS_SRC_LOWRANK) return KVS_EUNSUPPORTED;
+        if (ctx->map[l].kind == KVS_SRC_LOWRANK && cf.basis_rank != 32) return KVS_EUNSUPPORTED;
     for (int l = l0; l < l1; ++l) {
         s = check_layer_sources(ctx, cache, l, &need_kv, &need_lr);
         if (s != KVS_OK) return s;
@@ -685,14 +749,32 @@ kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const 
                                                   prefill_source_ready(ctx, ctx->map[l].src1, l)))
             return KVS_EINVAL;
     }
-    if (need_lr || cf.dtype != KVS_BF16) return KVS_EUNSUPPORTED;
     if (need_kv && (cache->slots < 1 || !dev_ok(cache->k) || !dev_ok(cache->v))) return KVS_EINVAL;
+    if (need_lr) {
+        const void* ps[] = {cache->coef_k, cache->coef_v, cache->basis_k, cache->basis_v, cache->u_k, cache->u_v,
+                            cache->s_k, cache->s_v, cache->r_k, cache->r_v, cache->rank};
+        for (const void* p : ps)
+            if (!dev_ok(p)) return KVS_EINVAL;
+    }
     if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
+    if (need_lr && ctx->qp == nullptr) {
+        const size_t n = static_cast<size_t>(cf.max_batch) * cf.num_q_heads * cf.max_context * LR_QW;
+        if (cudaMalloc(&ctx->qp, n * sizeof(uint16_t)) != cudaSuccess) {
+            cudaGetLastError();
+            ctx->qp = nullptr;
+            return KVS_ENOMEM;
+        }
+    }
     const int D = cf.head_dim, B = cache->batch, Hq = cf.num_q_heads, Hkv = cf.num_kv_heads, T = cache->context;
     const size_t per_layer = static_cast<size_t>(B) * Hq * seqlen;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     for (int l = l0; l < l1; ++l) {
         const kvshare_layer& e = ctx->map[l];
+        if (e.kind == KVS_SRC_LOWRANK) {
+            s = prefill_lowrank_layer(ctx, cache, q, out, lse, l, seqlen, st);
+            if (s != KVS_OK) return s;
+            continue;
+        }
         const bool mix = e.kind == KVS_SRC_MIX;
         PrefillArgs a;
         std::memset(&a, 0, sizeof(a));
@@ -719,10 +801,10 @@ kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const 
                      CU_TENSOR_MAP_SWIZZLE_128B, &tq) ||
             !get_map(ctx, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, seqlen, B * Hq, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B, &to) ||
-            !get_map(ctx, cache->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, rows, 64, bn,
-                     CU_TENSOR_MAP_SWIZZLE_128B, &tk) ||
-            !get_map(ctx, cache->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, T, rows, 64, bn,
-                     CU_TENSOR_MAP_SWIZZLE_128B, &tv))
+            !get_map(ctx, cache->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, seqlen, rows, 64, bn,
+                     CU_TENSOR_MAP_SWIZZLE_128B, &tk, T) ||
+            !get_map(ctx, cache->v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, seqlen, rows, 64, bn,
+                     CU_TENSOR_MAP_SWIZZLE_128B, &tv, T))
             return KVS_ECUDA;
         if (launch_prefill(D, mix, tq, tk, tv, to, a, st) != cudaSuccess) return KVS_ECUDA;
         ++ctx->launches;

@@ -141,6 +141,29 @@ struct PrefillArgs {
     long long wait_limit;
 };
 
+// Low-rank causal prefill of one layer (absorbed form, basis rank 32).
+constexpr int LR_QW = 64;   // width of a projected query row: B_K q (32) | R_K q (16) | 0 (16)
+struct PrefillLrArgs {
+    const uint16_t* q;          // layer's [B][Hq][S][d] bf16
+    uint16_t* qp;               // [B][Hq][S][LR_QW] bf16 projected queries (written by the pre-pass)
+    float* lse;                 // layer's [B][Hq][S] or nullptr
+    const uint16_t* basis_k;    // pair's [Hkv][32][d]
+    const uint16_t* basis_v;
+    const uint16_t* r_k;        // layer's [Hkv][16][d]
+    const uint16_t* r_v;
+    const uint16_t* s_k;        // layer's [B][Hkv][T] fp16
+    const uint16_t* s_v;
+    const uint8_t* rank;        // layer's [B][T]
+    int pair;                   // basis pair (row block of the coefficient maps)
+    int B, Hq, Hkv, S, T, g, d;
+    float scale_log2;
+    unsigned* err;
+    long long wait_limit;
+};
+cudaError_t launch_lr_qproj(const PrefillLrArgs& a, cudaStream_t st);
+// maps: Q' [B*Hq][S][64], O [B*Hq][S][d], C_K, C_V [P*B*Hkv][T][32], U_K, U_V [B*Hkv][T][16] (the layer's)
+cudaError_t launch_prefill_lowrank(int d, const CUtensorMap* maps, const PrefillLrArgs& a, cudaStream_t st);
+
 // kernel launchers (return cudaGetLastError() of the launch)
 struct TileShape { int tt; int nsw; int smem; };
 TileShape decode_bf16_shape(int d, bool mix);

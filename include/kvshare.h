@@ -186,9 +186,17 @@ kvshare_status kvshare_decode_stats(kvshare_t ctx, const kvshare_cache* cache, c
 kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, const void* q_host,
                                    float* out_host, float* lse_host, int l0, int l1, void* stream);
 
-/* Causal prefill of `seqlen` tokens for layers [l0, l1) (bf16 only; SINGLE and
- * MIX layers, LOWRANK gives KVS_EUNSUPPORTED). A MIX layer's K/V operands are
- * mixed from its two source slots inside the kernel and never written to HBM.
+/* Causal prefill of `seqlen` tokens for layers [l0, l1) (bf16 only). A MIX
+ * layer's K/V operands are mixed from its two source slots inside the kernel and
+ * never written to HBM. A LOWRANK layer (basis_rank 32 only, else
+ * KVS_EUNSUPPORTED) runs in the absorbed form ("DepthWeave-KV: Token-Adaptive
+ * Cross-Layer Residual Factorization for Long-Context KV Cache Compression",
+ * Detailed Explanation: basis lookup, dequantisation and attention projection in
+ * one pass): a pre-pass projects every query row to [B_K q | R_K q] (bf16, into a
+ * buffer of max_batch x Hq x max_context x 64 bf16 the context allocates on first
+ * use, KVS_ENOMEM if it cannot), the kernel attends over [C | s U] operands built
+ * per tile in shared memory and projects the result once through [B_V; R_V]; the
+ * rebuilt K/V never exist. Maps may mix all three kinds.
  * In a forward pass a slot is filled by its owner, the first layer of the map that
  * reads it as a SINGLE source, so a MIX layer's two sources must each be read as
  * SINGLE by some layer shallower than it; otherwise KVS_EINVAL ("DepthGraft:
@@ -198,7 +206,8 @@ kvshare_status kvshare_decode_host(kvshare_t ctx, const kvshare_cache* cache, co
  *   q:   [L][batch][Hq][seqlen][d] bf16
  *   out: [L][batch][Hq][seqlen][d] bf16
  *   lse: [L][batch][Hq][seqlen] fp32 or NULL
- * K/V rows 0..seqlen-1 of each store are used (seqlen <= context). */
+ * K/V rows 0..seqlen-1 of each store are used (seqlen <= context); cache.lengths
+ * must be NULL (KVS_EUNSUPPORTED otherwise). */
 kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const void* q,
                                void* out, float* lse, int l0, int l1, int seqlen, void* stream);
 

@@ -134,13 +134,16 @@ def prefill_ctx(K, layer_map, L=3, Hq=4, Hkv=2, d=64, T=32, w=None):
     return h, q, o, cache, w
 
 
-def test_prefill_lowrank_layer_is_unsupported(K):
+def test_prefill_lowrank_layer_needs_the_lowrank_arrays(K):
+    # a low-rank layer is prefilled in the absorbed form; without its cache arrays the
+    # call is rejected before any launch
     h, q, o, cache, w = prefill_ctx(K, None)
     try:
         K.kvshare_set_map(h, [(SINGLE, 0, 0), (SINGLE, 1, 0), (LOWRANK, 0, 0)], None)
         n0 = K.kvshare_launch_count(h)
+        cache.pairs = 1
         st = K.kvshare_prefill(h, cache, q, o, None, 0, 3, seqlen=32, check=False)
-        assert st == K.KVS_EUNSUPPORTED
+        assert st == K.KVS_EINVAL
         assert K.kvshare_launch_count(h) == n0
     finally:
         K.kvshare_destroy(h)
