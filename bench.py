@@ -344,6 +344,8 @@ def gpu_arm(args, cfg_name, secondary=False):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in e2e]))
 
+    extra = lowrank_extras(args, r, cfg, K, torch) if cfg.lowrank else {}
+
     read_bytes = sum(r.layer_bytes)
     res = {
         "cfg": cfg, "step_ms": step_ms, "per_layer_ms": per_layer, "launches": launches,
@@ -352,7 +354,7 @@ def gpu_arm(args, cfg_name, secondary=False):
         "h2d": q_host.numel() * q_host.element_size(),
         "d2h": out_host.numel() * 4 + lse_host.numel() * 4,
         "read_bytes": read_bytes, "pack_ms": r.pack_ms,
-        "pack_bytes": getattr(r, "pack_bytes", None),
+        "pack_bytes": getattr(r, "pack_bytes", None), "extra": extra,
     }
     r.close()
     del r
@@ -360,9 +362,100 @@ def gpu_arm(args, cfg_name, secondary=False):
     return res
 
 
+def lowrank_extras(args, r, cfg, K, torch):
+    """The low-rank workload's other per-step paths: the decode step with the router's
+    attention statistics (one statistics kernel after every layer), and the append of one
+    new token to every layer's cache (coefficients, residual codes, scales, ranks)."""
+    L, B, Hq, Hkv, T, d = cfg.layers, cfg.batch, cfg.q_heads, cfg.kv_heads, cfg.context, cfg.head_dim
+    mass = torch.empty((L, B, Hkv, T), device="cuda")
+    score = torch.empty((L, B, T), device="cuda")
+    ent = torch.empty((L, B, Hq), device="cuda")
+    peak = torch.empty((L, B, Hq), device="cuda")
+    order = cold_order(cfg)
+    for l in order:   # eager pass first: the score buffer is allocated and the kernels set up
+        K.kvshare_decode_stats(r.h, r.cache, r.dev["q"], r.out, r.lse, mass, score, ent, peak, l, l + 1, r.stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        cap = torch.cuda.current_stream()
+        for l in order:
+            K.kvshare_decode_stats(r.h, r.cache, r.dev["q"], r.out, r.lse, mass, score, ent, peak, l, l + 1, cap)
+    ev = []
+    for i in range(3 + max(5, args.steps // 2)):
+        r.flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(r.stream)
+        graph.replay()
+        e1.record(r.stream)
+        if i >= 3:
+            ev.append((e0, e1))
+    torch.cuda.synchronize()
+    stats_ms = statistics.median([a.elapsed_time(b) for a, b in ev])
+    del graph
+    # append: the new token of every layer written at the last position of the store
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    k_new = torch.randn((L, B, Hkv, d), device="cuda", generator=gen).to(torch.bfloat16)
+    v_new = torch.randn((L, B, Hkv, d), device="cuda", generator=gen).to(torch.bfloat16)
+    sc_new = torch.rand((L, B), device="cuda", generator=gen)
+    pos = torch.full((B,), T - 1, dtype=torch.int32, device="cuda")
+    app = []
+    for i in range(13):
+        r.flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(r.stream)
+        K.kvshare_append_lowrank(r.h, r.cache, k_new, v_new, sc_new, pos, r.stream)
+        e1.record(r.stream)
+        if i >= 3:
+            app.append((e0, e1))
+    torch.cuda.synchronize()
+    st = K.kvshare_sync_status(r.h)
+    assert st == K.KVS_OK, K.kvshare_status_string(st)
+    append_us = statistics.median([a.elapsed_time(b) for a, b in app]) * 1e3
+    return {"stats_ms_per_step": stats_ms, "append_us_per_token": append_us}
+
+
+def ragged_arm(args, cfg_name="cla2_1p1b"):
+    """The 1.1B CLA2 decode step with per-sequence lengths drawn uniformly from 1..T (seeded):
+    bytes read = each layer's source K and V over every sequence's own tokens."""
+    import torch
+    import synth.gpu as sgpu
+    from cross_layer_kv_shared_b200 import kvshare as K
+    cfg = BY_NAME[cfg_name]
+    r = DecodeRunner(cfg, K, torch, sgpu)
+    rng = np.random.default_rng(cfg.seed)
+    lens = rng.integers(1, cfg.context + 1, size=cfg.batch).astype(np.int32)
+    r.cache.lengths = torch.from_numpy(lens).cuda()
+    r.capture_step()
+    ev = []
+    for i in range(3 + max(5, args.steps)):
+        r.flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(r.stream)
+        r.step_graph()
+        e1.record(r.stream)
+        if i >= 3:
+            ev.append((e0, e1))
+    torch.cuda.synchronize()
+    st = K.kvshare_sync_status(r.h)
+    assert st == K.KVS_OK, K.kvshare_status_string(st)
+    ms = statistics.mean([a.elapsed_time(b) for a, b in ev])
+    es = 4 if cfg.dtype == "f32" else 2
+    read = sum((2 if cfg.layer_map[l][0] == MIX else 1) * 2 * cfg.kv_heads * cfg.head_dim * es * int(lens.sum())
+               for l in range(cfg.layers))
+    r.close()
+    del r
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "tok_s": cfg.batch / (ms * 1e-3), "kv_gbs": read / (ms * 1e-3) / 1e9,
+            "algorithmic_bytes_per_step": read, "mean_length": float(lens.mean()),
+            "lengths": "uniform on 1..%d, seeded" % cfg.context}
+
+
 def prefill_flops(cfg):
-    """Causal prefill FLOPs credited per step: 2 * B * Hq * d * S^2 per layer (QK^T + PV, causal half)."""
-    return 2.0 * cfg.batch * cfg.q_heads * cfg.head_dim * cfg.context ** 2 * cfg.layers
+    """Causal prefill FLOPs credited per step: 2 * B * Hq * w * S^2 per layer (QK^T + PV,
+    causal half), with w = d, or for a low-rank layer the absorbed operand width
+    Rb + 16 = 48 (the MMAs run padded to 64; the padding is not credited)."""
+    w = cfg.basis_rank + cfg.max_resid_rank if cfg.lowrank else cfg.head_dim
+    return 2.0 * cfg.batch * cfg.q_heads * w * cfg.context ** 2 * cfg.layers
 
 
 def prefill_arm(args, cfg_name="depthgraft_prefill"):
@@ -374,11 +467,23 @@ def prefill_arm(args, cfg_name="depthgraft_prefill"):
     cfg = BY_NAME[cfg_name]
     dev = {n: sgpu.make_device(cfg, n) for n in cfg.recipe()}
     _, h = K.kvshare_create(cfg.layers, cfg.q_heads, cfg.kv_heads, cfg.head_dim, K.KVS_BF16, cfg.batch, cfg.context)
-    K.kvshare_set_map(h, cfg.layer_map, cfg.make("w"))
+    K.kvshare_set_map(h, cfg.layer_map, None if cfg.lowrank else cfg.make("w"))
     S = cfg.context
     out = torch.empty((cfg.layers, cfg.batch, cfg.q_heads, S, cfg.head_dim), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((cfg.layers, cfg.batch, cfg.q_heads, S), device="cuda")
-    cache = K.Cache(batch=cfg.batch, context=S, k=dev["k"], v=dev["v"], slots=cfg.slots)
+    if cfg.lowrank:
+        L, B, Hkv = cfg.layers, cfg.batch, cfg.kv_heads
+        rank = torch.empty((L, B, S), dtype=torch.uint8, device="cuda")
+        ck = torch.empty((L, B, Hkv, S, 16), dtype=torch.int8, device="cuda")
+        cv = torch.empty_like(ck)
+        sk = torch.empty((L, B, Hkv, S), dtype=torch.int16, device="cuda")
+        sv = torch.empty_like(sk)
+        K.kvshare_pack_residual(h, dev["score"], dev["u_k"], dev["u_v"], rank, ck, cv, sk, sv, B, S)
+        cache = K.Cache(batch=B, context=S, coef_k=dev["coef_k"], coef_v=dev["coef_v"], basis_k=dev["basis_k"],
+                        basis_v=dev["basis_v"], u_k=ck, u_v=cv, s_k=sk, s_v=sv, r_k=dev["r_k"], r_v=dev["r_v"],
+                        rank=rank, pairs=cfg.pairs)
+    else:
+        cache = K.Cache(batch=cfg.batch, context=S, k=dev["k"], v=dev["v"], slots=cfg.slots)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         K.kvshare_prefill(h, cache, dev["q"], out, lse, stream=stream)
@@ -402,8 +507,8 @@ def prefill_arm(args, cfg_name="depthgraft_prefill"):
         per_layer[l] += e0.elapsed_time(e1)
     per_layer /= args.steps
     step_ms = max_over_ranks(float(per_layer.sum()))
-    single = [l for l in range(cfg.layers) if cfg.layer_map[l][0] == 0]
-    mixed = [l for l in range(cfg.layers) if cfg.layer_map[l][0] == 1]
+    single = [l for l in range(cfg.layers) if cfg.layer_map[l][0] != MIX]
+    mixed = [l for l in range(cfg.layers) if cfg.layer_map[l][0] == MIX]
     K.kvshare_destroy(h)
     del dev, out, lse
     torch.cuda.empty_cache()
@@ -597,7 +702,19 @@ def main():
             if r2["pack_ms"] is not None:
                 sec[name]["pack_residual_ms"] = r2["pack_ms"]
                 sec[name]["pack_residual_gbs"] = r2["pack_bytes"] / (r2["pack_ms"] * 1e-3) / 1e9
+            if r2["extra"]:
+                sec[name]["with_router_stats_ms_per_step"] = r2["extra"]["stats_ms_per_step"]
+                sec[name]["append_us_per_token"] = r2["extra"]["append_us_per_token"]
+        rg = ragged_arm(argparse.Namespace(steps=max(5, args.steps // 2), warmup=3))
+        sec["cla2_1p1b_ragged_lengths"] = dict(rg, hbm_frac=rg["kv_gbs"] / hbm_peak)
     if not args.no_secondary and not args.no_prefill:
+        pl = prefill_arm(argparse.Namespace(steps=max(3, args.steps // 3), warmup=3), "depthweave_prefill")
+        sec["depthweave_prefill"] = {
+            "tflops_absorbed": pl["tflops"], "ms_per_step": pl["step_ms"],
+            "tok_s": pl["tokens"] * world / (pl["step_ms"] * 1e-3),
+            "tensor_frac_of_burst_padded": pl["tflops"] * 64 / 48 / bf16_peak,
+            "equivalent_d128_tflops": pl["tflops"] * 128 / 48,
+            "flops_per_step": prefill_flops(pl["cfg"]), "gpu_launches": pl["launches"], "clocks": pl["clocks"]}
         pr = prefill_arm(argparse.Namespace(steps=max(3, args.steps // 3), warmup=3))
         sec["depthgraft_prefill"] = {
             "tflops": pr["tflops"], "ms_per_step": pr["step_ms"], "tok_s": pr["tokens"] * world / (pr["step_ms"] * 1e-3),

@@ -1,6 +1,6 @@
 """Workload presets and their seeded tensors.
 
-Five presets follow the workloads the pages describe, at the sizes the build is
+Six presets follow the workloads the pages describe, at the sizes the build is
 measured on:
 
 * ``tiny_cla2_f32``   - CLA2 (adjacent-layer sharing, sharing factor 2), fp32, tiny.
@@ -10,6 +10,7 @@ measured on:
   16+j reads the stride-aligned pair (j, 8+j). DepthGraft page, "Abstract".
 * ``depthweave_decode`` - 16 layer pairs sharing a rank-32 basis, per-layer int8
   low-rank residual with per-token rank. DepthWeave-KV page, "Core Mechanism".
+* ``depthweave_prefill`` - the same model's causal prefill of 4096 tokens.
 
 Everything here is data: shapes, layer tables and the (seed, tensor id, scale)
 recipe of every input. No attention, mixing or quantisation arithmetic.
@@ -164,5 +165,10 @@ DEPTHWEAVE_DECODE = Config("depthweave_decode", "decode", layers=32, q_heads=32,
                            head_dim=128, batch=1, context=65536, dtype="bf16",
                            layer_map=depthweave_map(32), pairs=16, seed=SEED0 + 4)
 
-PRESETS = [TINY_CLA2, CLA2_1P1B, DEPTHGRAFT_DECODE, DEPTHGRAFT_PREFILL, DEPTHWEAVE_DECODE]
+# causal prefill of the DepthWeave model's first 4096 tokens (its head layout, 16 layer pairs)
+DEPTHWEAVE_PREFILL = Config("depthweave_prefill", "prefill", layers=32, q_heads=32, kv_heads=8,
+                            head_dim=128, batch=1, context=4096, dtype="bf16",
+                            layer_map=depthweave_map(32), pairs=16, seed=SEED0 + 5)
+
+PRESETS = [TINY_CLA2, CLA2_1P1B, DEPTHGRAFT_DECODE, DEPTHGRAFT_PREFILL, DEPTHWEAVE_DECODE, DEPTHWEAVE_PREFILL]
 BY_NAME = {c.name: c for c in PRESETS}

@@ -88,7 +88,7 @@ def test_offsets_continue_the_stream():
 
 
 def test_presets_match_the_workloads():
-    c0, c1, c2, c3, c4 = PRESETS
+    c0, c1, c2, c3, c4, c5 = PRESETS
     assert (c0.layers, c0.q_heads, c0.kv_heads, c0.head_dim, c0.batch, c0.context, c0.dtype) == \
         (4, 4, 2, 64, 1, 128, "f32")
     assert [m[1] for m in c0.layer_map] == [0, 0, 1, 1]
@@ -99,4 +99,5 @@ def test_presets_match_the_workloads():
     assert c3.layer_map == c2.layer_map and c3.mode == "prefill" and c3.context == 4096
     assert (c4.layers, c4.pairs, c4.q_heads, c4.kv_heads, c4.context) == (32, 16, 32, 8, 65536)
     assert BY_NAME["depthweave_decode"] is c4
-    assert len({c.seed for c in PRESETS}) == 5
+    assert c5.layer_map == c4.layer_map and c5.mode == "prefill" and (c5.q_heads, c5.kv_heads) == (32, 8)
+    assert len({c.seed for c in PRESETS}) == 6
