@@ -131,35 +131,6 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             }
         }
     };
-    // The warp's tiles past its ring are requested into L2 a window ahead (lane 0), so
-    // the memory system keeps streaming while a launch's fixed-cost phases run.
-    constexpr int W_L2 = l2_window_tiles(NW, C::STAGE_BYTES);
-    int pu = u_w0, pt = t_w0, n_pf = 0;   // next tile to request into L2, tiles passed so far
-    auto prefetch_next = [&] {
-        if (n_pf >= my_n) return;
-        const int u = pu, t = pt;
-        advance(pu, pt);
-        ++n_pf;
-        if (STRADDLE && a.lens != nullptr && t >= unit_tiles(u)) return;
-        const int row0 = a.src0 * BH + u;
-        const int row1 = MIX ? a.src1 * BH + u : 0;
-#pragma unroll
-        for (int h = 0; h < C::HALVES; ++h) {
-            tma_prefetch_3d(&tmK, h * 64, t * TT, row0);
-            tma_prefetch_3d(&tmV, h * 64, t * TT, row0);
-            if (MIX) {
-                tma_prefetch_3d(&tmK, h * 64, t * TT, row1);
-                tma_prefetch_3d(&tmV, h * 64, t * TT, row1);
-            }
-        }
-    };
-    auto start_prefetch = [&] {       // skip the ring's tiles, then fill the window
-        for (int i = 0; i < NSW && n_pf < my_n; ++i) {
-            advance(pu, pt);
-            ++n_pf;
-        }
-        for (int i = 0; i < W_L2; ++i) prefetch_next();
-    };
     // Under a dependent launch everything up to grid_dep_wait overlaps the previous
     // kernel's tail. Inputs, workspace and counters are touched only after it; with
     // kv_early the caller has promised that no kernel ahead on the stream writes the
@@ -168,7 +139,6 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         set_range();
         if (lane == 0) {
             for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
-            start_prefetch();
         }
         __syncwarp();
     }
@@ -178,7 +148,6 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         set_range();
         if (lane == 0) {
             for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
-            start_prefetch();
         }
         __syncwarp();
     }
@@ -290,7 +259,6 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             // a tile past the sequence: its stage completed empty; hand it on
             __syncwarp();
             if (lane == 0 && k + NSW < my_n) issue(k + NSW);
-            if (lane == 0) prefetch_next();
             __syncwarp();
             continue;
         }
@@ -438,7 +406,6 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             fence_proxy_async();
             issue(k + NSW);
         }
-        if (lane == 0) prefetch_next();
         __syncwarp();
     }
 

@@ -175,18 +175,6 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         tma_load_3d(st + C::OFF_UK, &tmUK, 0, t * TT, urow, &wb[s]);
         tma_load_3d(st + C::OFF_UV, &tmUV, 0, t * TT, urow, &wb[s]);
     };
-    // the warp's tiles past its ring are requested into L2 a window ahead (lane 0)
-    constexpr int W_L2 = l2_window_tiles(NW, 2 * C::COEF_BYTES + 2 * C::U_BYTES);
-    auto prefetch_l2 = [&](int k) {
-        const int t = tile0 + warp + k * NW;
-#pragma unroll
-        for (int h = 0; h < LY::HALVES; ++h) {
-            tma_prefetch_3d(&tmCK, h * 64, t * TT, crow);
-            tma_prefetch_3d(&tmCV, h * 64, t * TT, crow);
-        }
-        tma_prefetch_3d(&tmUK, 0, t * TT, urow);
-        tma_prefetch_3d(&tmUV, 0, t * TT, urow);
-    };
     // per-token scales and ranks of a tile, loaded by the lanes (tokens lane, lane+32, ...)
     constexpr int TPL = TT / 32;
     // raw 16-bit scales and 8-bit ranks: converted only when published, a tile later, so
@@ -225,7 +213,6 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         }
         if (lane == 0) {
             for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
-            for (int k = NSW; k < min(NSW + W_L2, my_n); ++k) prefetch_l2(k);
         }
         __syncwarp();
         if (my_n > 0) prefetch(0);
@@ -528,7 +515,6 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             fence_proxy_async();
             issue(k + NSW);
         }
-        if (lane == 0 && k + NSW + W_L2 < my_n) prefetch_l2(k + NSW + W_L2);
     }
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)

@@ -93,22 +93,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
-// Prefetch a 3-D tile of a tensor map into L2 (no shared memory, no completion): the
-// later TMA load of the same box then finds its lines in L2.
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
-}
-
-// Tiles a warp keeps requested into L2 ahead of its shared-memory ring: about 320 KB per
-// CTA, so that the whole GPU holds under 48 MB of prefetched lines (well inside the
-// 126 MB L2, with room for the tiles in use) whatever the workload.
-__host__ __device__ constexpr int l2_window_tiles(int nwarps, int tile_bytes) {
-    return (320 * 1024) / (nwarps * tile_bytes) > 0 ? (320 * 1024) / (nwarps * tile_bytes) : 1;
-}
-
 // 3-D tiled bulk tensor store shared -> global (rows outside the tensor are not written).
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
