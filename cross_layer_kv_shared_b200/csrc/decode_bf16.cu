@@ -311,7 +311,9 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    sc[mt][nb][i] = (MIX ? (w * sc[mt][nb][i] + w1 * sc2[mt][nb][i]) : sc[mt][nb][i]) * a.scale_log2;
+                    // explicitly rounded, so every compiled copy of this loop gives the same bits
+                    sc[mt][nb][i] = __fmul_rn(MIX ? fmaf(w, sc[mt][nb][i], w1 * sc2[mt][nb][i]) : sc[mt][nb][i],
+                                              a.scale_log2);
             if (tail) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)

@@ -269,10 +269,9 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     __syncthreads();
     if (a.stall && threadIdx.x == 0) mbar_wait_bounded(&bars[NW * NSW], 0, a.stall_limit, a.err);
 
-    // B fragments of q~^T (RB rows, bf16 hi + lo) and q^^T (16 rows, f16: the residual term
-    // is scaled by s_K, far below the basis term, so f16's 11 bits suffice there);
-    // column = head nb*8 + lane/4
-    uint32_t qch[RB / 16][NB][2], qcl[RB / 16][NB][2], quh[NB][2];
+    // B fragments of q~^T (RB rows, bf16 hi + lo) and q^^T (16 rows, f16 hi + lo): each
+    // projection keeps about 16 (bf16) or 22 (f16) bits; column = head nb*8 + lane/4
+    uint32_t qch[RB / 16][NB][2], qcl[RB / 16][NB][2], quh[NB][2], qul[NB][2];
     {
         const int cq = 2 * (lane & 3);
 #pragma unroll
@@ -289,8 +288,15 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 frag(ks * 16 + cq, qch[ks][nb][0], qcl[ks][nb][0]);
                 frag(ks * 16 + 8 + cq, qch[ks][nb][1], qcl[ks][nb][1]);
             }
-            quh[nb][0] = pack_f16(qproj[h * C::PD + RB + cq], qproj[h * C::PD + RB + cq + 1]);
-            quh[nb][1] = pack_f16(qproj[h * C::PD + RB + 8 + cq], qproj[h * C::PD + RB + 8 + cq + 1]);
+            auto frag16 = [&](int col, uint32_t& hi, uint32_t& lo) {
+                const float x0 = qproj[h * C::PD + col];
+                const float x1 = qproj[h * C::PD + col + 1];
+                hi = pack_f16(x0, x1);
+                const __half2 hv = *reinterpret_cast<const __half2*>(&hi);
+                lo = pack_f16(x0 - __low2float(hv), x1 - __high2float(hv));
+            };
+            frag16(RB + cq, quh[nb][0], qul[nb][0]);
+            frag16(RB + 8 + cq, quh[nb][1], qul[nb][1]);
         }
     }
 
@@ -409,7 +415,10 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             uint32_t af[4];
             ldsm_x4(smem_u32(cvk) + cvt_off(row, mi >> 1), af[0], af[1], af[2], af[3]);
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) mma_f16(su[mt][nb], af, quh[nb][0], quh[nb][1]);
+            for (int nb = 0; nb < NB; ++nb) {
+                mma_f16(su[mt][nb], af, quh[nb][0], quh[nb][1]);
+                mma_f16(su[mt][nb], af, qul[nb][0], qul[nb][1]);
+            }
         }
         // ---- scores, mask, online softmax per head; P^T and (P s_V)^T by movmatrix
         uint32_t pb[MT][NB][2], pvb[MT][NB][2];
@@ -428,7 +437,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    sc[mt][nb][i] = (sc[mt][nb][i] + skr[mt][i >> 1] * su[mt][nb][i]) * a.scale_log2;
+                    sc[mt][nb][i] = __fmul_rn(fmaf(skr[mt][i >> 1], su[mt][nb][i], sc[mt][nb][i]), a.scale_log2);
             if (tail) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)

@@ -77,6 +77,8 @@ def check_against_oracle(cfg, inp, lens, out, lse):
     get = lambda name, index: ref.to_f64(inp[name][index], cfg.dtype)  # noqa: E731
     want, want_lse = ref.decode(cfg.layer_map, ref.to_f64(inp["q"], cfg.dtype), get, w=inp["w"], lengths=lens)
     tol = 1e-4 if cfg.dtype == "f32" else TOL
+    err = np.max(np.abs(np.nan_to_num(out, nan=1e9) - np.nan_to_num(want, nan=0.0)), axis=(2, 3))
+    print(f"{cfg.name}: max|d| per (layer, sequence) with lengths {list(lens)}:\n{err}")
     empty = lens == 0
     assert np.all(out[:, empty] == 0.0) and np.all(lse[:, empty] == -np.inf)
     full = ~empty
@@ -101,6 +103,15 @@ def test_ragged_lengths_match_the_oracle(K, cfg):
         for grid in (7, 3 * cfg.batch * cfg.kv_heads + 1):
             out3, lse3 = run_kv(K, cfg, inp, lens, grid=grid)
             check_against_oracle(cfg, inp, lens, out3, lse3)
+
+
+@pytest.mark.parametrize("cfg", CASES[1:], ids=lambda c: c.name)
+def test_ragged_lengths_on_a_clean_cache(K, cfg):
+    # the same lengths with ordinary values past them: only the lengths decide
+    inp = cfg.make_all()
+    lens = lengths_for(cfg.batch, cfg.context, cfg.seed)
+    out, lse = run_kv(K, cfg, inp, lens)
+    check_against_oracle(cfg, inp, lens, out, lse)
 
 
 def test_all_lengths_full_equals_no_lengths(K):
