@@ -316,6 +316,9 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         part[tid * PD + DV + 1] = sm_l[tid];
         part[tid * PD + DV + 2] = sm_lx[tid];
     }
+    // the last CTA reads the partials with a bulk copy (the async proxy): every writer
+    // orders its own generic stores before that proxy before the arrival releases them
+    asm volatile("fence.proxy.async.global;" ::: "memory");
     __syncthreads();
     __shared__ unsigned s_is_last;
     if (tid == 0) {
