@@ -59,9 +59,10 @@ def oracle_prefill(cfg, inp, S, layers=None, batches=None, heads=None, rows=None
 SMALL = [
     pcfg("pf_single_d128", 2, [(SINGLE, 0, 0), (SINGLE, 1, 0)], 2, 4, 2, 128, 1, 300),
     pcfg("pf_mix_d128", 3, [(SINGLE, 0, 0), (SINGLE, 1, 0), (MIX, 0, 1)], 2, 4, 2, 128, 2, 200),
-    pcfg("pf_d64", 2, [(SINGLE, 1, 0), (MIX, 1, 0)], 2, 8, 2, 64, 1, 257),
-    pcfg("pf_s1", 1, [(MIX, 0, 1)], 2, 2, 1, 128, 1, 1),
-    pcfg("pf_s128_ctx_longer", 2, [(SINGLE, 0, 0), (MIX, 1, 0)], 2, 4, 4, 128, 1, 128, T=160),
+    # a two-source target reads slots that shallower layers fill (own) in the same pass
+    pcfg("pf_d64", 3, [(SINGLE, 1, 0), (SINGLE, 0, 0), (MIX, 1, 0)], 2, 8, 2, 64, 1, 257),
+    pcfg("pf_s1", 3, [(SINGLE, 0, 0), (SINGLE, 1, 0), (MIX, 0, 1)], 2, 2, 1, 128, 1, 1),
+    pcfg("pf_s128_ctx_longer", 3, [(SINGLE, 0, 0), (SINGLE, 1, 0), (MIX, 1, 0)], 2, 4, 4, 128, 1, 128, T=160),
 ]
 
 
