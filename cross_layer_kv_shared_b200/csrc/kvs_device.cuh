@@ -355,22 +355,27 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         }
         __syncthreads();
     }
+    // This CTA's own partial is taken from its shared memory, never read back from
+    // global: its stores may not yet be what a bulk copy of the slot returns, and a
+    // stale slot (an earlier launch's partial) would silently take its place.
     if (one_copy) {
         mbar_wait_bounded(&mbar, 0, a.wait_limit, a.err);
         for (int idx = tid; idx < n * g; idx += nthr) {
             const int sp = idx / g;
             const int h = idx % g;
-            fm[idx] = sp_buf[sp * per + h * PD + DV];
-            fl[idx] = sp_buf[sp * per + h * PD + DV + 1];
-            flx[idx] = sp_buf[sp * per + h * PD + DV + 2];
+            const bool own = sp == index;
+            fm[idx] = own ? sm_m[h] : sp_buf[sp * per + h * PD + DV];
+            fl[idx] = own ? sm_l[h] : sp_buf[sp * per + h * PD + DV + 1];
+            flx[idx] = own ? sm_lx[h] : sp_buf[sp * per + h * PD + DV + 2];
         }
     } else {
         for (int idx = tid; idx < n * g; idx += nthr) {
             const int sp = idx / g;
             const int h = idx % g;
-            fm[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV);
-            fl[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 1);
-            flx[idx] = __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 2);
+            const bool own = sp == index;
+            fm[idx] = own ? sm_m[h] : __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV);
+            fl[idx] = own ? sm_l[h] : __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 1);
+            flx[idx] = own ? sm_lx[h] : __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 2);
         }
     }
     __syncthreads();
@@ -409,7 +414,7 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
                 const int h = idx / DV;
                 const int e = idx % DV;
                 float v = 0.f;
-                for (int c = 0; c < n; ++c) v += fm[c * g + h] * sp_buf[c * per + h * PD + e];
+                for (int c = 0; c < n; ++c) v += fm[c * g + h] * (c == index ? sm_v[h * DV + e] : sp_buf[c * per + h * PD + e]);
                 acc[k] = v;
             }
         }
@@ -431,7 +436,8 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
                     const int h = idx / DV;
                     const int e = idx % DV;
                     float v = acc[k];
-                    for (int c = 0; c < cnt; ++c) v += fm[(s0 + c) * g + h] * sp_buf[c * per + h * PD + e];
+                    for (int c = 0; c < cnt; ++c)
+                        v += fm[(s0 + c) * g + h] * (s0 + c == index ? sm_v[h * DV + e] : sp_buf[c * per + h * PD + e]);
                     acc[k] = v;
                 }
             }
@@ -446,7 +452,8 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
                 const int e = idx % DV;
                 float v = 0.f;
 #pragma unroll 8
-                for (int sp = 0; sp < n; ++sp) v += fm[sp * g + h] * __ldcg(base + static_cast<size_t>(sp) * per + h * PD + e);
+                for (int sp = 0; sp < n; ++sp)
+                    v += fm[sp * g + h] * (sp == index ? sm_v[h * DV + e] : __ldcg(base + static_cast<size_t>(sp) * per + h * PD + e));
                 acc[k] = v;
             }
         }
