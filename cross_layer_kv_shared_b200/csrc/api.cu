@@ -99,6 +99,9 @@ struct kvshare_ctx {
     float* sscore = nullptr;
     // projected queries of one low-rank prefill layer [max_batch][Hq][max_context][64] bf16
     uint16_t* qp = nullptr;
+    // statistics kernel: per-block entropy/peak partials and per-sequence arrival counters
+    float* stats_part = nullptr;
+    unsigned* stats_counters = nullptr;
     // staging for kvshare_decode_host
     void* q_stage = nullptr;
     float* out_stage = nullptr;
@@ -366,17 +369,14 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
             sa.score = stats->score ? stats->score + lbt * T : nullptr;
             sa.entropy = stats->entropy ? stats->entropy + lbt * Hq : nullptr;
             sa.peak = stats->peak ? stats->peak + lbt * Hq : nullptr;
+            sa.part = c->stats_part;
+            sa.counters = c->stats_counters;
             sa.err = c->err;
             sa.B = B;
             sa.Hq = Hq;
             sa.Hkv = Hkv;
             sa.T = T;
             sa.g = g;
-            // entropy and peak accumulate: start each layer's rows at zero
-            if (sa.entropy && cudaMemsetAsync(sa.entropy, 0, static_cast<size_t>(B) * Hq * sizeof(float), st) != cudaSuccess)
-                return KVS_ECUDA;
-            if (sa.peak && cudaMemsetAsync(sa.peak, 0, static_cast<size_t>(B) * Hq * sizeof(float), st) != cudaSuccess)
-                return KVS_ECUDA;
             if (launch_router_stats(sa, st) != cudaSuccess) return KVS_ECUDA;
             ++c->launches;
         }
@@ -545,6 +545,8 @@ kvshare_status kvshare_destroy(kvshare_t ctx) {
     cudaFree(ctx->w_dev);
     cudaFree(ctx->sscore);
     cudaFree(ctx->qp);
+    cudaFree(ctx->stats_part);
+    cudaFree(ctx->stats_counters);
     cudaFree(ctx->q_stage);
     cudaFree(ctx->out_stage);
     cudaFree(ctx->lse_stage);
@@ -623,10 +625,20 @@ kvshare_status kvshare_decode_stats(kvshare_t ctx, const kvshare_cache* cache, c
                              static_cast<cudaStream_t>(stream));
     if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
     if (ctx->sscore == nullptr) {
-        const size_t n = static_cast<size_t>(ctx->cfg.max_batch) * ctx->cfg.num_q_heads * ctx->cfg.max_context;
-        if (cudaMalloc(&ctx->sscore, n * sizeof(float)) != cudaSuccess) {
+        const kvshare_config& cf = ctx->cfg;
+        const size_t n = static_cast<size_t>(cf.max_batch) * cf.num_q_heads * cf.max_context;
+        const size_t np = static_cast<size_t>(cf.max_batch) * router_stats_blocks(cf.max_context) * cf.num_q_heads * 2;
+        if (cudaMalloc(&ctx->sscore, n * sizeof(float)) != cudaSuccess ||
+            cudaMalloc(&ctx->stats_part, np * sizeof(float)) != cudaSuccess ||
+            cudaMalloc(&ctx->stats_counters, cf.max_batch * sizeof(unsigned)) != cudaSuccess ||
+            cudaMemset(ctx->stats_counters, 0, cf.max_batch * sizeof(unsigned)) != cudaSuccess) {
             cudaGetLastError();
+            cudaFree(ctx->sscore);
+            cudaFree(ctx->stats_part);
+            cudaFree(ctx->stats_counters);
             ctx->sscore = nullptr;
+            ctx->stats_part = nullptr;
+            ctx->stats_counters = nullptr;
             return KVS_ENOMEM;
         }
     }

@@ -442,19 +442,31 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                 if (fin_unit[ww] == u) M = fmaxf(M, comb_ml[ww * 48 + h]);
                 if (STRADDLE && sav_unit[ww] == u) M = fmaxf(M, save_ml[ww * 48 + h]);
             }
+            // a warp without a state for u left its slots as they were (ring data, or an
+            // earlier kernel's shared memory, NaN included): never read them, not even as 0 * x
             float L = 0.f, LX = 0.f;
             for (int ww = 0; ww < NW; ++ww) {
-                const float mf = comb_ml[ww * 48 + h];
-                const float ff = (fin_unit[ww] == u && mf != NEG_INF) ? ex2_approx(mf - M) : 0.f;
+                float ff = 0.f;
+                if (fin_unit[ww] == u) {
+                    const float mf = comb_ml[ww * 48 + h];
+                    if (mf != NEG_INF) {
+                        ff = ex2_approx(mf - M);
+                        L = fmaf(ff, comb_ml[ww * 48 + 16 + h], L);
+                        LX = fmaf(ff, comb_ml[ww * 48 + 32 + h], LX);
+                    }
+                }
                 fac_f[ww][h] = ff;
-                L += ff * comb_ml[ww * 48 + 16 + h];
-                LX += ff * comb_ml[ww * 48 + 32 + h];
                 if (STRADDLE) {
-                    const float ms = save_ml[ww * 48 + h];
-                    const float fs = (sav_unit[ww] == u && ms != NEG_INF) ? ex2_approx(ms - M) : 0.f;
+                    float fs = 0.f;
+                    if (sav_unit[ww] == u) {
+                        const float ms = save_ml[ww * 48 + h];
+                        if (ms != NEG_INF) {
+                            fs = ex2_approx(ms - M);
+                            L = fmaf(fs, save_ml[ww * 48 + 16 + h], L);
+                            LX = fmaf(fs, save_ml[ww * 48 + 32 + h], LX);
+                        }
+                    }
                     fac_s[ww][h] = fs;
-                    L += fs * save_ml[ww * 48 + 16 + h];
-                    LX += fs * save_ml[ww * 48 + 32 + h];
                 }
             }
             fin_m[h] = M;

@@ -97,11 +97,14 @@ struct StatsArgs {
     const int* lens;        // [B] or nullptr
     float* mass;            // [B][Hkv][T] or nullptr
     float* score;           // [B][T] or nullptr
-    float* entropy;         // [B][Hq] or nullptr (zeroed before the launch)
-    float* peak;            // [B][Hq] or nullptr (zeroed before the launch)
+    float* entropy;         // [B][Hq] or nullptr
+    float* peak;            // [B][Hq] or nullptr
+    float* part;            // [B][blocks][Hq][2] per-block entropy and peak partials
+    unsigned* counters;     // [B] arrival counters, zero between launches
     unsigned* err;
     int B, Hq, Hkv, T, g;
 };
+int router_stats_blocks(int T);
 cudaError_t launch_router_stats(const StatsArgs& a, cudaStream_t st);
 
 // Append of one new token to a low-rank cache (every basis pair, sequence and kv head).

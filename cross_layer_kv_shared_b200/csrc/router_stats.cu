@@ -6,24 +6,27 @@
 // second component; Key Concepts, Token-Conditional Depth Routing). The decode
 // kernels keep every valid token's log2-domain scaled score s_{h,t} for the layer;
 // with the layer's lse (exact weight sums) each weight is p_{h,t} = 2^(s - lse/ln 2).
-// One thread per (sequence, token) then writes
+// Each thread takes TPT tokens of one sequence (HB heads' scores loaded at a time) and writes
 //   mass[j][t]  = sum over the g heads of kv head j of p_{h,t}
 //   score[t]    = x / (1 + x),  x = (T_b * sum_j mass[j][t]) / Hq     (fp32, in this order)
-// and adds each head's entropy terms p (lse2 - s) ln 2 and peak candidates p into
-// the per-head outputs (warp reductions, one atomic per warp and head). Tokens past
-// the sequence get mass 0 and score 0.
+// Tokens past the sequence get mass 0 and score 0. Per head, each block reduces its
+// entropy terms p (lse2 - s) ln 2 and its largest p in shared memory and stores one
+// partial; the last block of the sequence to finish (an arrival counter) adds the
+// partials in block order, so entropy and peak are deterministic.
 #include "kvs_device.cuh"
 
 namespace kvs {
 namespace {
 
 constexpr int NT = 256;
+constexpr int TPT = 1;                        // tokens per thread
+constexpr int HB = 16;                        // heads whose scores are loaded together
+constexpr int HC = 64;                        // heads reduced per pass through shared memory
 constexpr float LOG2E_F = 1.4426950408889634f;
 
 __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
     const int b = blockIdx.y;
-    const int t = blockIdx.x * NT + threadIdx.x;
-    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int n = a.T;
     if (a.lens != nullptr) {
         n = a.lens[b];
@@ -32,46 +35,116 @@ __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
             n = n < 0 ? 0 : a.T;
         }
     }
-    const bool in_store = t < a.T;
-    const bool valid = t < n;
-    const bool want_ent = a.entropy != nullptr, want_peak = a.peak != nullptr;
-    float total = 0.f;
-    for (int j = 0; j < a.Hkv; ++j) {
-        float mj = 0.f;
-        for (int hh = 0; hh < a.g; ++hh) {
-            const int h = j * a.g + hh;
-            const size_t bh = static_cast<size_t>(b) * a.Hq + h;
-            const float lse2 = a.lse[bh] * LOG2E_F;
-            float p = 0.f, e = 0.f;
-            if (valid) {
-                const float s = a.sscore[bh * a.T + t];
-                p = exp2f(s - lse2);
-                e = p * (lse2 - s);
-            }
-            mj += p;
-            if (want_ent) {
-                const float es = warp_sum(e);
-                if (lane == 0 && es != 0.f) atomicAdd(a.entropy + bh, es * LN2_F);
-            }
-            if (want_peak) {
-                const float pm = warp_max(p);
-                if (lane == 0 && pm > 0.f) atomicMax(reinterpret_cast<int*>(a.peak + bh), __float_as_int(pm));
+    const bool want_red = a.entropy != nullptr || a.peak != nullptr;
+    __shared__ float red_e[NT / 32][HC], red_p[NT / 32][HC];
+    __shared__ float lse2_s[HC];
+    float macc[TPT], total[TPT];
+#pragma unroll
+    for (int k = 0; k < TPT; ++k) macc[k] = total[k] = 0.f;
+    const int t0 = blockIdx.x * NT * TPT + threadIdx.x;   // this thread's tokens: t0 + k * NT
+    const float* srow0 = a.sscore + static_cast<size_t>(b) * a.Hq * a.T;
+    for (int h0 = 0; h0 < a.Hq; h0 += HC) {
+        const int hn = min(HC, a.Hq - h0);
+        if (threadIdx.x < hn) lse2_s[threadIdx.x] = a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] * LOG2E_F;
+        __syncthreads();
+        for (int hb = 0; hb < hn; hb += HB) {
+            // the scores of HB heads first, all loads in flight together
+            float sv[HB][TPT];
+#pragma unroll
+            for (int q = 0; q < HB; ++q)
+#pragma unroll
+                for (int k = 0; k < TPT; ++k) {
+                    const int t = t0 + k * NT;
+                    sv[q][k] = (hb + q < hn && t < n) ? __ldcs(srow0 + static_cast<size_t>(h0 + hb + q) * a.T + t) : 0.f;
+                }
+#pragma unroll
+            for (int q = 0; q < HB; ++q) {
+                const int hh = hb + q;
+                if (hh >= hn) break;
+                const int h = h0 + hh;
+                const float l2 = lse2_s[hh];
+                float es = 0.f, pm = 0.f;
+#pragma unroll
+                for (int k = 0; k < TPT; ++k) {
+                    const int t = t0 + k * NT;
+                    float p = 0.f;
+                    if (t < n) {
+                        p = exp2f(sv[q][k] - l2);
+                        es += p * (l2 - sv[q][k]);
+                        pm = fmaxf(pm, p);
+                    }
+                    macc[k] = h % a.g == 0 ? p : macc[k] + p;   // kv head j = h / g, heads in order
+                }
+                if (h % a.g == a.g - 1) {                     // group complete: its mass, then the total
+                    const int j = h / a.g;
+#pragma unroll
+                    for (int k = 0; k < TPT; ++k) {
+                        const int t = t0 + k * NT;
+                        if (a.mass != nullptr && t < a.T) a.mass[(static_cast<size_t>(b) * a.Hkv + j) * a.T + t] = macc[k];
+                        total[k] = j == 0 ? macc[k] : __fadd_rn(total[k], macc[k]);
+                    }
+                }
+                if (want_red) {
+                    es = warp_sum(es);
+                    pm = warp_max(pm);
+                    if (lane == 0) {
+                        red_e[warp][hh] = es;
+                        red_p[warp][hh] = pm;
+                    }
+                }
             }
         }
-        if (a.mass != nullptr && in_store) a.mass[(static_cast<size_t>(b) * a.Hkv + j) * a.T + t] = mj;
-        total = j == 0 ? mj : __fadd_rn(total, mj);
+        __syncthreads();
+        if (want_red && threadIdx.x < hn) {
+            float e = 0.f, p = 0.f;
+            for (int w = 0; w < NT / 32; ++w) {
+                e += red_e[w][threadIdx.x];
+                p = fmaxf(p, red_p[w][threadIdx.x]);
+            }
+            float* part = a.part + ((static_cast<size_t>(b) * gridDim.x + blockIdx.x) * a.Hq + h0 + threadIdx.x) * 2;
+            part[0] = e;
+            part[1] = p;
+        }
+        __syncthreads();
     }
-    if (a.score != nullptr && in_store) {
-        float x = __fmul_rn(static_cast<float>(n), total);
-        x = __fdiv_rn(x, static_cast<float>(a.Hq));
-        a.score[static_cast<size_t>(b) * a.T + t] = __fdiv_rn(x, __fadd_rn(1.f, x));
+    if (a.score != nullptr) {
+#pragma unroll
+        for (int k = 0; k < TPT; ++k) {
+            const int t = t0 + k * NT;
+            if (t >= a.T) continue;
+            float x = __fmul_rn(static_cast<float>(n), total[k]);
+            x = __fdiv_rn(x, static_cast<float>(a.Hq));
+            a.score[static_cast<size_t>(b) * a.T + t] = __fdiv_rn(x, __fadd_rn(1.f, x));
+        }
     }
+    if (!want_red) return;
+    // the last block of the sequence adds the per-block partials in block order
+    __threadfence();
+    __shared__ unsigned last;
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(a.counters + b, 1u) == gridDim.x - 1 ? 1u : 0u;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    for (int h = threadIdx.x; h < a.Hq; h += NT) {
+        float e = 0.f, p = 0.f;
+        for (unsigned blk = 0; blk < gridDim.x; ++blk) {
+            const float* part = a.part + ((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h) * 2;
+            e += __ldcg(part);
+            p = fmaxf(p, __ldcg(part + 1));
+        }
+        if (a.entropy != nullptr) a.entropy[static_cast<size_t>(b) * a.Hq + h] = e * LN2_F;
+        if (a.peak != nullptr) a.peak[static_cast<size_t>(b) * a.Hq + h] = p;
+    }
+    if (threadIdx.x == 0) a.counters[b] = 0u;
 }
 
 }  // namespace
 
+int router_stats_blocks(int T) { return (T + NT * TPT - 1) / (NT * TPT); }
+
 cudaError_t launch_router_stats(const StatsArgs& a, cudaStream_t st) {
-    dim3 grid((a.T + NT - 1) / NT, a.B);
+    dim3 grid(router_stats_blocks(a.T), a.B);
     router_stats_kernel<<<grid, NT, 0, st>>>(a);
     return cudaGetLastError();
 }

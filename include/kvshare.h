@@ -161,10 +161,10 @@ kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const v
  *           rank: 8 from 7/3 times the uniform share, 16 from 9 times.
  *   entropy [L][batch][Hq] fp32: -sum_t p ln p (nats) per query head
  *   peak    [L][batch][Hq] fp32: max_t p per query head
- * Any of the four may be NULL; lse is required. Entropy is summed with atomics, so
- * its last bits can differ from run to run. The first call with an output allocates
- * a score buffer of max_batch x Hq x max_context floats in the context (KVS_ENOMEM
- * if that fails); each layer adds one statistics kernel after its decode kernel. */
+ * Any of the four may be NULL; lse is required. The first call with an output
+ * allocates a score buffer of max_batch x Hq x max_context floats and a small
+ * reduction buffer in the context (KVS_ENOMEM if that fails); each layer adds one
+ * statistics kernel after its decode kernel. Results are the same bits run to run. */
 kvshare_status kvshare_decode_stats(kvshare_t ctx, const kvshare_cache* cache, const void* q, float* out,
                                     float* lse, float* mass, float* score, float* entropy, float* peak,
                                     int l0, int l1, void* stream);
@@ -279,6 +279,7 @@ kvshare_status kvshare_set_kv_overlap(kvshare_t ctx, int on);
  * order decides which shared sources are still in L2 when a layer reads them.
  * KVS_EINVAL if an entry is out of range or repeated. */
 kvshare_status kvshare_set_layer_order(kvshare_t ctx, const int* order);
+
 
 /* Test hook: force the bf16 decode grid to `ctas` CTAs (0 = automatic). The
  * units' token tiles are cut into that many equal ranges, so a CTA may cover
