@@ -13,13 +13,17 @@
 //   codes, scale of u_a at the rank the router gives the token in layer a
 // Every dot product runs in fp32 from index 0 up, each product and each sum
 // correctly rounded (no fused multiply-add), so the bf16 coefficients and the
-// integer codes are reproducible bit for bit. One CTA per (pair, sequence, kv head).
+// integer codes are reproducible bit for bit. One CTA per (pair, sequence, kv head);
+// it first copies the pair's basis and both layers' residual factors into shared
+// memory (one coalesced pass), then walks them there.
 #include "kvs_quant.cuh"
 
 namespace kvs {
 namespace {
 
 constexpr int NT = 128;
+constexpr int LDB = 128 + 2;   // padded bf16 rows: a walk along a row (thread per row) and down a
+                               // column (thread per column) both fall on distinct banks
 
 __device__ __forceinline__ float bf(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
 
@@ -37,12 +41,43 @@ __global__ void __launch_bounds__(NT) append_lowrank_kernel(const AppendArgs a) 
         return;
     }
     const int D = a.d, RB = a.Rb;
+    extern __shared__ uint16_t sfac[];                    // [RB basis rows | nl x 16 factor rows][LDB]
     __shared__ float kk[2][128], m[128], cst[128], e[2][128], us[2][QUANT_RM];
     const size_t BHkv = static_cast<size_t>(a.B) * a.Hkv;
     const size_t bj = static_cast<size_t>(b) * a.Hkv + j;
+    const int rows = RB + nl * QUANT_RM;
     for (int side = 0; side < 2; ++side) {                 // K, then V
         const uint16_t* nw = side == 0 ? a.k_new : a.v_new;
         const uint16_t* basis = (side == 0 ? a.basis_k : a.basis_v) + (static_cast<size_t>(p) * a.Hkv + j) * RB * D;
+        const uint16_t* Rf = side == 0 ? a.r_k : a.r_v;
+        // the pair's basis and both layers' residual factors, in one coalesced pass
+        // (loads in groups of eight per thread before any store: one round trip a group)
+        constexpr int G = 8;
+        for (int i0 = tid; i0 < rows * (D / 8); i0 += G * NT) {
+            uint4 v[G];
+#pragma unroll
+            for (int k = 0; k < G; ++k) {
+                const int idx = i0 + k * NT;
+                if (idx >= rows * (D / 8)) break;
+                const int r = idx / (D / 8), c8 = idx % (D / 8);
+                const uint16_t* src;
+                if (r < RB) {
+                    src = basis + static_cast<size_t>(r) * D;
+                } else {
+                    const int ai = (r - RB) / QUANT_RM, s = (r - RB) % QUANT_RM;
+                    src = Rf + ((static_cast<size_t>(ai == 0 ? la : lb) * a.Hkv + j) * QUANT_RM + s) * D;
+                }
+                v[k] = *reinterpret_cast<const uint4*>(src + c8 * 8);
+            }
+#pragma unroll
+            for (int k = 0; k < G; ++k) {
+                const int idx = i0 + k * NT;
+                if (idx >= rows * (D / 8)) break;
+                const int r = idx / (D / 8), c8 = idx % (D / 8);
+                uint32_t* dst = reinterpret_cast<uint32_t*>(sfac + r * LDB + c8 * 8);
+                dst[0] = v[k].x; dst[1] = v[k].y; dst[2] = v[k].z; dst[3] = v[k].w;
+            }
+        }
         if (tid < D) {
             const float x0 = bf(nw[(la * BHkv + bj) * D + tid]);
             const float x1 = bf(nw[(lb * BHkv + bj) * D + tid]);
@@ -52,7 +87,7 @@ __global__ void __launch_bounds__(NT) append_lowrank_kernel(const AppendArgs a) 
         }
         __syncthreads();
         if (tid < RB) {
-            const uint16_t* row = basis + static_cast<size_t>(tid) * D;
+            const uint16_t* row = sfac + tid * LDB;
             float c = __fmul_rn(bf(row[0]), m[0]);
             for (int i = 1; i < D; ++i) c = __fadd_rn(c, __fmul_rn(bf(row[i]), m[i]));
             const __nv_bfloat16 cb = __float2bfloat16_rn(c);
@@ -62,19 +97,18 @@ __global__ void __launch_bounds__(NT) append_lowrank_kernel(const AppendArgs a) 
         }
         __syncthreads();
         if (tid < D) {
-            float r = __fmul_rn(cst[0], bf(basis[tid]));
-            for (int i = 1; i < RB; ++i) r = __fadd_rn(r, __fmul_rn(cst[i], bf(basis[static_cast<size_t>(i) * D + tid])));
+            float r = __fmul_rn(cst[0], bf(sfac[tid]));
+            for (int i = 1; i < RB; ++i) r = __fadd_rn(r, __fmul_rn(cst[i], bf(sfac[i * LDB + tid])));
             e[0][tid] = __fsub_rn(kk[0][tid], r);
             e[1][tid] = __fsub_rn(kk[1][tid], r);
         }
         __syncthreads();
         if (tid < nl * QUANT_RM) {
-            const int ai = tid / QUANT_RM, s = tid % QUANT_RM;
-            const int l = ai == 0 ? la : lb;
-            const uint16_t* R = (side == 0 ? a.r_k : a.r_v) + ((static_cast<size_t>(l) * a.Hkv + j) * QUANT_RM + s) * D;
+            const int ai = tid / QUANT_RM;
+            const uint16_t* R = sfac + (RB + tid) * LDB;
             float u = __fmul_rn(bf(R[0]), e[ai][0]);
             for (int i = 1; i < D; ++i) u = __fadd_rn(u, __fmul_rn(bf(R[i]), e[ai][i]));
-            us[ai][s] = u;
+            us[ai][tid % QUANT_RM] = u;
         }
         __syncthreads();
         if (tid < nl) {
@@ -100,7 +134,9 @@ __global__ void __launch_bounds__(NT) append_lowrank_kernel(const AppendArgs a) 
 
 cudaError_t launch_append_lowrank(const AppendArgs& a, cudaStream_t st) {
     dim3 grid(a.P, a.B, a.Hkv);
-    append_lowrank_kernel<<<grid, NT, 0, st>>>(a);
+    // at most (128 + 32) rows of LDB bf16 (41.6 KB), with the static arrays under 48 KB
+    const size_t smem = static_cast<size_t>(a.Rb + 2 * QUANT_RM) * LDB * sizeof(uint16_t);
+    append_lowrank_kernel<<<grid, NT, smem, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -40,7 +40,7 @@ struct LrPfCfg {
     static constexpr int NS = 3;                       // ring A: [K' | V'] stages (built by the converters)
     static constexpr int STAGE_A = 2 * OP_TILE;
     // ring B: raw tiles [C_K | C_V | U_K | U_V], filled by TMA, freed by the converters
-    static constexpr int NSB = 2;
+    static constexpr int NSB = 4;
     static constexpr int C_BYTES = BN * RB * 2;        // [64][32] bf16, unswizzled 64-byte rows
     static constexpr int U_BYTES = BN * RM;            // [64][16] int8
     static constexpr int STAGE_B = 2 * C_BYTES + 2 * U_BYTES;
@@ -71,8 +71,8 @@ struct LrPfCfg {
 struct LrSync {
     uint64_t q_full;
     uint64_t w_full;
-    uint64_t raw_full[2];
-    uint64_t raw_empty[2];
+    uint64_t raw_full[4];
+    uint64_t raw_empty[4];
     uint64_t op_ready[3];
     uint64_t op_empty[3];
     uint64_t s_full[NQ];
@@ -313,17 +313,31 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const int hf = t & 1;
         const size_t tok_row = (static_cast<size_t>(b) * a.Hkv + jkv) * a.T;
         const uint16_t* s_src = m == 0 ? a.s_k : a.s_v;
-        for (int j = 0; j < n_kv; ++j) {
+        // the token's scale bits and rank, loaded PF tiles ahead of their use (plain loads;
+        // the loop below is unrolled by PF so that no register with a load in flight moves)
+        constexpr int PF = 3;
+        uint32_t pf_s[PF], pf_r[PF];
+        auto meta = [&](int jj, uint32_t& sb, uint32_t& rb) {
+            const int tok = jj * BN + r;
+            sb = 0u;
+            rb = 0u;
+            if (hf == 1 && jj < n_kv && tok < a.S) {     // rows past the sequence stay zero
+                sb = s_src[tok_row + tok];
+                rb = a.rank[static_cast<size_t>(b) * a.T + tok];
+            }
+        };
+#pragma unroll
+        for (int q = 0; q < PF; ++q) meta(q, pf_s[q], pf_r[q]);
+        for (int j0 = 0; j0 < n_kv; j0 += PF) {
+#pragma unroll
+          for (int q = 0; q < PF; ++q) {
+            const int j = j0 + q;
+            if (j >= n_kv) break;
             const int s = j % NS;
             const int sb = j % NSB;
-            const int tok = j * BN + r;
-            // the token's scale and rank (plain loads, in flight while the tile lands)
-            float scale = 0.f;
-            int rk = 0;
-            if (hf == 1 && tok < a.S) {     // rows past the sequence stay zero
-                scale = __half2float(__ushort_as_half(s_src[tok_row + tok]));
-                rk = a.rank[static_cast<size_t>(b) * a.T + tok];
-            }
+            const float scale = __half2float(__ushort_as_half(static_cast<unsigned short>(pf_s[q])));
+            const int rk = static_cast<int>(pf_r[q]);
+            meta(j + PF, pf_s[q], pf_r[q]);
             wait_lr(sy, &sy.raw_full[sb], (j / NSB) & 1, a.wait_limit, a.err);
             if (j >= NS) wait_lr(sy, &sy.op_empty[s], ((j / NS) - 1) & 1, a.wait_limit, a.err);
             const uint8_t* raw = sB + sb * C::STAGE_B;
@@ -354,6 +368,7 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             fence_proxy_async();
             mbar_arrive(&sy.op_ready[s]);
             mbar_arrive(&sy.raw_empty[sb]);
+          }
         }
     } else {
         tc::reg_dec<C::REG_CTRL>();
@@ -456,44 +471,74 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 }
 
 // ---------------------------------------------------------------- query projection pre-pass
-// q'[b][h][s] = [B_K q | R_K q | 0] as bf16, each value one fp32 dot product over d.
-// Block: one (sequence, head) and 64 query rows; thread = (row group, output column).
-constexpr int QP_ROWS = 64;
-constexpr int QP_THREADS = 192;
+// q'[b][h][s] = [B_K q | R_K q | 0] as bf16: per (sequence, head) a [rows x d] by [d x 48]
+// product on the tensor cores (mma.sync m16n8k16, bf16 operands, fp32 accumulation),
+// rounded once to bf16. Block: one (sequence, head) and 128 query rows, 16 rows per warp.
+constexpr int QP_ROWS = 128;
+constexpr int QP_WARPS = QP_ROWS / 16;
 
 template <int D>
-__global__ void __launch_bounds__(QP_THREADS) lr_qproj_kernel(const PrefillLrArgs a) {
-    __shared__ __align__(16) uint16_t Wt[D][RB + RM];        // transposed [B_K; R_K]
-    __shared__ __align__(16) uint16_t qs[QP_ROWS][D];
+__global__ void __launch_bounds__(QP_WARPS * 32) lr_qproj_kernel(const PrefillLrArgs a) {
+    constexpr int LD = D + 8;     // padded rows: the 8 rows of an ldmatrix fall on distinct banks
+    __shared__ __align__(16) uint16_t W[RB + RM][LD];     // [B_K; R_K], row n = output column n
+    __shared__ __align__(16) uint16_t qs[QP_ROWS][LD];
     const int h = blockIdx.x, b = blockIdx.y, r0 = blockIdx.z * QP_ROWS;
     const int j = h / a.g;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint16_t* Bk = a.basis_k + static_cast<size_t>(j) * RB * D;
     const uint16_t* Rk = a.r_k + static_cast<size_t>(j) * RM * D;
-    for (int idx = tid; idx < (RB + RM) * D; idx += QP_THREADS) {
-        const int c = idx / D, i = idx % D;
-        Wt[i][c] = c < RB ? Bk[c * D + i] : Rk[(c - RB) * D + i];
+    for (int idx = tid; idx < (RB + RM) * D / 8; idx += blockDim.x) {
+        const int c = idx / (D / 8), i8 = idx % (D / 8);
+        const uint16_t* src = c < RB ? Bk + c * D : Rk + (c - RB) * D;
+        *reinterpret_cast<uint4*>(&W[c][i8 * 8]) = *reinterpret_cast<const uint4*>(src + i8 * 8);
     }
     const size_t bh = static_cast<size_t>(b) * a.Hq + h;
     const int nrows = min(QP_ROWS, a.S - r0);
-    for (int idx = tid; idx < QP_ROWS * D / 8; idx += QP_THREADS) {
+    for (int idx = tid; idx < QP_ROWS * D / 8; idx += blockDim.x) {
         const int rr = idx / (D / 8), c8 = idx % (D / 8);
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (rr < nrows) v = *reinterpret_cast<const uint4*>(a.q + (bh * a.S + r0 + rr) * D + c8 * 8);
         *reinterpret_cast<uint4*>(&qs[rr][c8 * 8]) = v;
     }
     __syncthreads();
-    const int c = tid % (RB + RM);
-    const int rg = tid / (RB + RM);
-    for (int rr = rg; rr < nrows; rr += QP_THREADS / (RB + RM)) {
-        float acc = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < D; ++i)
-            acc = fmaf(__uint_as_float(static_cast<uint32_t>(qs[rr][i]) << 16),
-                       __uint_as_float(static_cast<uint32_t>(Wt[i][c]) << 16), acc);
+    const int wr = warp * 16;
+    if (wr >= nrows) return;
+    constexpr int NT = (RB + RM) / 8;     // n8 tiles of output columns
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        // A: (rows 0-7 | 8-15) x (k 0-7 | 8-15) of the warp's 16 rows
+        uint32_t af[4];
+        ldsm_x4(smem_u32(&qs[wr + (mi & 1) * 8 + ri][ks * 16 + (mi >> 1) * 8]), af[0], af[1], af[2], af[3]);
+#pragma unroll
+        for (int n = 0; n < NT; n += 2) {
+            // B of two n-tiles: W rows are the output columns, contiguous in k
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(smem_u32(&W[(n + (mi >> 1)) * 8 + ri][ks * 16 + (mi & 1) * 8]), b0, b1, b2, b3);
+            mma_bf16(acc[n], af, b0, b1);
+            mma_bf16(acc[n + 1], af, b2, b3);
+        }
+    }
+    // accumulator rows lane/4 and lane/4 + 8, columns 2 (lane % 4) and + 1 of each n-tile
+    const int rw = lane >> 2, cq = 2 * (lane & 3);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int rr = wr + rw + half * 8;
+        if (rr >= nrows) continue;
         uint16_t* dst = a.qp + (bh * a.S + r0 + rr) * QW;
-        dst[c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
-        if (c < QW - RB - RM) dst[RB + RM + c] = 0;
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+            *reinterpret_cast<uint32_t*>(dst + n * 8 + cq) = pack_bf16(acc[n][2 * half], acc[n][2 * half + 1]);
+    }
+    // the padding columns 48..63 of the warp's rows are zero
+    {
+        const int rr = wr + (lane >> 1);
+        if (rr < nrows)
+            *reinterpret_cast<uint4*>(a.qp + (bh * a.S + r0 + rr) * QW + RB + RM + (lane & 1) * 8) =
+                make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
@@ -521,9 +566,9 @@ cudaError_t launch_lr_one(const CUtensorMap* maps, const PrefillLrArgs& a, cudaS
 cudaError_t launch_lr_qproj(const PrefillLrArgs& a, cudaStream_t st) {
     dim3 grid(a.Hq, a.B, (a.S + QP_ROWS - 1) / QP_ROWS);
     if (a.d == 64)
-        lr_qproj_kernel<64><<<grid, QP_THREADS, 0, st>>>(a);
+        lr_qproj_kernel<64><<<grid, QP_WARPS * 32, 0, st>>>(a);
     else
-        lr_qproj_kernel<128><<<grid, QP_THREADS, 0, st>>>(a);
+        lr_qproj_kernel<128><<<grid, QP_WARPS * 32, 0, st>>>(a);
     return cudaGetLastError();
 }
 

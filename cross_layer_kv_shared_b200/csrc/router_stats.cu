@@ -12,7 +12,8 @@
 // Tokens past the sequence get mass 0 and score 0. Per head, each block reduces its
 // entropy terms p (lse2 - s) ln 2 and its largest p in shared memory and stores one
 // partial; the last block of the sequence to finish (an arrival counter) adds the
-// partials in block order, so entropy and peak are deterministic.
+// partials in a fixed order (per thread, then a fixed tree), so entropy and peak are
+// deterministic.
 #include "kvs_device.cuh"
 
 namespace kvs {
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
         }
     }
     if (!want_red) return;
-    // the last block of the sequence adds the per-block partials in block order
+    // the last block of the sequence to arrive adds the per-block partials
     __threadfence();
     __shared__ unsigned last;
     __syncthreads();
@@ -126,15 +127,46 @@ __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
     __syncthreads();
     if (!last) return;
     __threadfence();
-    for (int h = threadIdx.x; h < a.Hq; h += NT) {
-        float e = 0.f, p = 0.f;
-        for (unsigned blk = 0; blk < gridDim.x; ++blk) {
-            const float* part = a.part + ((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h) * 2;
-            e += __ldcg(part);
-            p = fmaxf(p, __ldcg(part + 1));
+    // thread i adds the partials of blocks i, i + NT, ... in order; a fixed tree over the
+    // threads (shuffles, then the warps in order) finishes each head
+    for (int h0 = 0; h0 < a.Hq; h0 += HC) {
+        const int hn = min(HC, a.Hq - h0);
+        for (int hb = 0; hb < hn; hb += HB) {
+            float ve[HB], vp[HB];
+#pragma unroll
+            for (int q = 0; q < HB; ++q) ve[q] = vp[q] = 0.f;
+            for (unsigned blk = threadIdx.x; blk < gridDim.x; blk += NT) {
+                const float* part = a.part + ((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h0 + hb) * 2;
+#pragma unroll
+                for (int q = 0; q < HB; ++q)
+                    if (hb + q < hn) {
+                        ve[q] += __ldcg(part + 2 * q);
+                        vp[q] = fmaxf(vp[q], __ldcg(part + 2 * q + 1));
+                    }
+            }
+#pragma unroll
+            for (int q = 0; q < HB; ++q) {
+                if (hb + q >= hn) break;
+                const float e = warp_sum(ve[q]);
+                const float p = warp_max(vp[q]);
+                if (lane == 0) {
+                    red_e[warp][hb + q] = e;
+                    red_p[warp][hb + q] = p;
+                }
+            }
         }
-        if (a.entropy != nullptr) a.entropy[static_cast<size_t>(b) * a.Hq + h] = e * LN2_F;
-        if (a.peak != nullptr) a.peak[static_cast<size_t>(b) * a.Hq + h] = p;
+        __syncthreads();
+        if (threadIdx.x < hn) {
+            float e = 0.f, p = 0.f;
+            for (int w = 0; w < NT / 32; ++w) {
+                e += red_e[w][threadIdx.x];
+                p = fmaxf(p, red_p[w][threadIdx.x]);
+            }
+            const size_t o = static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x;
+            if (a.entropy != nullptr) a.entropy[o] = e * LN2_F;
+            if (a.peak != nullptr) a.peak[o] = p;
+        }
+        __syncthreads();
     }
     if (threadIdx.x == 0) a.counters[b] = 0u;
 }
