@@ -647,24 +647,25 @@ int occupancy_of() {
     return n > 0 ? n : 1;
 }
 
-// token tile, stages per warp and warps per CTA by basis rank (the full-rank basis only serves tests)
-// (defaults: the fastest of a measured sweep on the 64K-token, Rb = 32 workload:
-// 16 warps with one 32-token stage each beat deeper rings on fewer warps, two stages
-// on 16 warps, and 18 to 20 warps)
+// token tile, stages per warp and warps per CTA by basis rank (the 64 and full-rank
+// bases only serve tests). Rb = 32 defaults: the fastest of a measured sweep on the
+// 64K-token workload (µs per layer in the replayed step): 12 warps with two 32-token
+// stages each 25.7; 16 warps x 1 stage 27.5; 8 x 2 and 8 x 3 27.0; 8 warps x one
+// 64-token stage 28.5 (and earlier: 18 to 20 warps x 1 stage slower than 16).
 #ifndef KVS_LR_TT
 #define KVS_LR_TT 32
 #endif
 #ifndef KVS_LR_NSW
-#define KVS_LR_NSW 1
+#define KVS_LR_NSW 2
 #endif
 #ifndef KVS_LR_NW
-#define KVS_LR_NW 16
+#define KVS_LR_NW 12
 #endif
 template <int RB>
 struct LrShape {
-    static constexpr int TT = RB == 128 ? 32 : KVS_LR_TT;
-    static constexpr int NSW = RB == 128 ? 1 : KVS_LR_NSW;
-    static constexpr int NW = RB == 128 ? 4 : KVS_LR_NW;
+    static constexpr int TT = RB == 32 ? KVS_LR_TT : 32;
+    static constexpr int NSW = RB == 32 ? KVS_LR_NSW : 1;
+    static constexpr int NW = RB == 32 ? KVS_LR_NW : (RB == 128 ? 4 : 16);
 };
 
 template <int D, int RB>
@@ -677,7 +678,7 @@ cudaError_t run(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
 
 }  // namespace
 
-int decode_lowrank_tile(int rb) { return rb == 128 ? LrShape<128>::TT : LrShape<32>::TT; }
+int decode_lowrank_tile(int rb) { return rb == 32 ? LrShape<32>::TT : (rb == 64 ? LrShape<64>::TT : LrShape<128>::TT); }
 
 int decode_lowrank_occupancy(int d, int rb) {
     if (d == 64) return rb == 32 ? occ<64, 32>() : occ<64, 64>();
