@@ -592,12 +592,22 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(cfg, seconds=12.0):
+def cpu_baseline(cfg, seconds=12.0, seconds_1core=4.0):
     per_unit, units, threads = oracle_sample(cfg, seconds)
     step_s = per_unit * cfg.layers * cfg.batch
-    return {"value": cfg.batch / step_s, "unit": "tok/s", "cores": threads, "kind": "oracle",
-            "sample": f"{units} (layer, batch) units of {cfg.name}, fp64 numpy, extrapolated to "
-                      f"{cfg.layers} layers x {cfg.batch} batch"}
+    out = {"value": cfg.batch / step_s, "unit": "tok/s", "cores": threads, "kind": "oracle",
+           "sample": f"{units} (layer, batch) units of {cfg.name}, fp64 numpy, extrapolated to "
+                     f"{cfg.layers} layers x {cfg.batch} batch"}
+    # the same oracle on one host core (BLAS threads limited to 1)
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            per1, units1, _ = oracle_sample(cfg, seconds_1core, rng_seed=1)
+        out["value_1core"] = cfg.batch / (per1 * cfg.layers * cfg.batch)
+        out["sample_1core"] = f"{units1} units, BLAS limited to 1 thread"
+    except ImportError:
+        out["value_1core"] = None
+    return out
 
 
 def data_desc(cfg):
@@ -653,7 +663,8 @@ def main():
     ap.add_argument("--only", choices=["prefill"], default=None,
                     help="profiling aid: run only the causal prefill workload and print its numbers")
     ap.add_argument("--batch", type=int, default=0,
-                    help="profiling aid (with --only prefill): batch of the prefill workload")
+                    help="profiling aid: batch of the prefill workload (with --only prefill) or of the "
+                         "--config decode workload (a smaller case of the same kernels)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -685,6 +696,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     hbm_peak, bf16_peak, bf16_sust, peak_src = load_peaks()
+    if args.batch > 0:
+        name = f"{args.config}_b{args.batch}"
+        BY_NAME[name] = BY_NAME[args.config].replace(name=name, batch=args.batch)
+        args.config = name
     main_res = gpu_arm(args, args.config)
     cfg = main_res["cfg"]
     sec = {}

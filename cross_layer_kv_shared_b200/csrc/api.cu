@@ -305,16 +305,13 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
             a.r_k = static_cast<const uint16_t*>(k->r_k) + static_cast<size_t>(l) * Hkv * 16 * D;
             a.r_v = static_cast<const uint16_t*>(k->r_v) + static_cast<size_t>(l) * Hkv * 16 * D;
             a.rank = k->rank + static_cast<size_t>(l) * B * T;
-            CUtensorMap maps[4];
+            // coefficient tiles by TMA; the group-packed residual codes by sized bulk copies
+            CUtensorMap maps[2];
             const int crows = k->pairs * B * Hkv;
             const int box0 = Rb < 64 ? Rb : 64;
             const CUtensorMapSwizzle sw = Rb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
             if (!get_map(c, k->coef_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Rb, T, crows, box0, tt, sw, &maps[0]) ||
-                !get_map(c, k->coef_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Rb, T, crows, box0, tt, sw, &maps[1]) ||
-                !get_map(c, a.u_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, T, B * Hkv, 16, tt,
-                         CU_TENSOR_MAP_SWIZZLE_NONE, &maps[2]) ||
-                !get_map(c, a.u_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, T, B * Hkv, 16, tt,
-                         CU_TENSOR_MAP_SWIZZLE_NONE, &maps[3]))
+                !get_map(c, k->coef_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Rb, T, crows, box0, tt, sw, &maps[1]))
                 return KVS_ECUDA;
             err = launch_decode_lowrank(D, Rb, a, maps, st);
         } else {

@@ -121,8 +121,13 @@ __global__ void __launch_bounds__(NT) append_lowrank_kernel(const AppendArgs a) 
             uint16_t sc;
             quantize16(x, r, packed, sc);
             const size_t row = (static_cast<size_t>(l) * BHkv + bj) * a.T + t;
+            // group-packed codes: after those of the group's earlier tokens
+            const int t0 = t - t % CODE_GROUP;
+            const uint8_t* rk = a.rank + (static_cast<size_t>(l) * a.B + b) * a.T;
+            int o = 0;
+            for (int tt = t0; tt < t; ++tt) o += code_len(rk[tt]);
             int8_t* codes = side == 0 ? a.u_k : a.u_v;
-            *reinterpret_cast<uint4*>(codes + row * QUANT_RM) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            store_codes(codes + (row - (t - t0)) * QUANT_RM + o, packed, code_len(r));
             (side == 0 ? a.s_k : a.s_v)[row] = sc;
             if (side == 0 && j == 0) a.rank[(static_cast<size_t>(l) * a.B + b) * a.T + t] = r;
         }

@@ -311,9 +311,9 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    // explicitly rounded, so every compiled copy of this loop gives the same bits
-                    sc[mt][nb][i] = __fmul_rn(MIX ? fmaf(w, sc[mt][nb][i], w1 * sc2[mt][nb][i]) : sc[mt][nb][i],
-                                              a.scale_log2);
+                    // raw (unscaled) scores: every operation written out, so every compiled
+                    // copy of this loop gives the same bits
+                    if (MIX) sc[mt][nb][i] = fmaf(w, sc[mt][nb][i], __fmul_rn(w1, sc2[mt][nb][i]));
             if (tail) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
@@ -330,7 +330,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                     for (int i = 0; i < 4; ++i) {
                         const int h = h0 + (i & 1);
                         const int r = mt * 16 + (i >> 1) * 8;
-                        if (h < g && r < lim) srow[static_cast<size_t>(h) * a.T + t * TT + (lane >> 2) + r] = sc[mt][nb][i];
+                        if (h < g && r < lim) srow[static_cast<size_t>(h) * a.T + t * TT + (lane >> 2) + r] = __fmul_rn(sc[mt][nb][i], a.scale_log2);
                     }
             }
 #pragma unroll
@@ -343,6 +343,10 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                 mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
             }
+            // the row max in the scaled (log2) domain: scaling by a positive factor and
+            // rounding are monotonic, so this is the max of the scaled scores
+            mx0 = __fmul_rn(mx0, a.scale_log2);
+            mx1 = __fmul_rn(mx1, a.scale_log2);
             const float mn0 = fmaxf(mrow[nb][0], mx0);
             const float mn1 = fmaxf(mrow[nb][1], mx1);
             const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
@@ -362,8 +366,10 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const float p0 = ex2_approx(sc[mt][nb][0] - ref0), p1 = ex2_approx(sc[mt][nb][1] - ref1);
-                const float p2 = ex2_approx(sc[mt][nb][2] - ref0), p3 = ex2_approx(sc[mt][nb][3] - ref1);
+                const float p0 = ex2_approx(fmaf(sc[mt][nb][0], a.scale_log2, -ref0));
+                const float p1 = ex2_approx(fmaf(sc[mt][nb][1], a.scale_log2, -ref1));
+                const float p2 = ex2_approx(fmaf(sc[mt][nb][2], a.scale_log2, -ref0));
+                const float p3 = ex2_approx(fmaf(sc[mt][nb][3], a.scale_log2, -ref1));
                 lxrow[nb][0] += p0 + p2;
                 lxrow[nb][1] += p1 + p3;
                 if (!MIX) {

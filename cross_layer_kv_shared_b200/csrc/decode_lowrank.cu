@@ -21,12 +21,13 @@
 //   - int8 codes convert exactly to f16 operands, masked by the token's rank;
 //   - c^ and u^ accumulate in fp32 MMA accumulators; split partials stay in this
 //     coefficient space and the CTA that merges a unit projects it once.
-#include "kvs_device.cuh"
+#include "kvs_quant.cuh"
 
 namespace kvs {
 namespace {
 
 constexpr int RM = 16;
+
 
 template <int RB>
 struct CoefLayout {
@@ -51,7 +52,9 @@ struct LrCfg {
     static constexpr int ALIGN128(int x) { return (x + 127) / 128 * 128; }
     static constexpr int OFF_UK = 2 * COEF_BYTES;
     static constexpr int OFF_UV = OFF_UK + ALIGN128(U_BYTES);
-    static constexpr int STAGE_BYTES = ((OFF_UV + U_BYTES + 1023) / 1024) * 1024;   // keeps swizzled tiles aligned
+    // keeps swizzled tiles aligned (the word-wise code reads may run up to 20 bytes past a
+    // stage's V codes: into the next stage, or the buffers that follow the ring)
+    static constexpr int STAGE_BYTES = ((OFF_UV + U_BYTES + 1023) / 1024) * 1024;
     static_assert(COEF_BYTES % 128 == 0 && OFF_UK % 128 == 0 && OFF_UV % 128 == 0,
                   "TMA destinations must be 128-byte aligned");
     static constexpr int RING_BYTES = NW * NSW * STAGE_BYTES;
@@ -107,7 +110,6 @@ __device__ __forceinline__ uint32_t i8pair_bf16(uint32_t w16, bool keep0, bool k
 template <int D, int RB, int TT, int NSW, int NW, int NH>
 __global__ void __launch_bounds__(NW * 32, 1)
 decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_constant__ CUtensorMap tmCV,
-                      const __grid_constant__ CUtensorMap tmUK, const __grid_constant__ CUtensorMap tmUV,
                       const DecodeArgs a) {
     using C = LrCfg<D, RB, TT, NSW, NW>;
     using LY = typename C::L;
@@ -144,8 +146,6 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     if (threadIdx.x == 0) {
         prefetch_tmap(&tmCK);
         prefetch_tmap(&tmCV);
-        prefetch_tmap(&tmUK);
-        prefetch_tmap(&tmUV);
         for (int i = 0; i < NW * NSW + 1; ++i) mbar_init(&bars[i], 1);
         mbar_init(&fac_bar[0], 1);
         mbar_init(&fac_bar[1], 1);
@@ -162,21 +162,55 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         my_n = span > warp ? (span - warp + NW - 1) / NW : 0;
     };
 
-    auto issue = [&](int k) {
+    // A tile's stage: its coefficients by TMA first (lane 0), then, once the tile's ranks
+    // are known, the used bytes of its code groups by bulk copy; the second step arrives.
+    auto issue_coef = [&](int k) {
         const int t = tile0 + warp + k * NW;
         const int s = k % NSW;
         uint8_t* st = ring + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&wb[s], 2 * C::COEF_BYTES + 2 * C::U_BYTES);
+        mbar_expect_tx(&wb[s], 2 * C::COEF_BYTES);
 #pragma unroll
         for (int h = 0; h < LY::HALVES; ++h) {
             tma_load_3d(st + h * TT * 128, &tmCK, h * 64, t * TT, crow, &wb[s]);
             tma_load_3d(st + C::COEF_BYTES + h * TT * 128, &tmCV, h * 64, t * TT, crow, &wb[s]);
         }
-        tma_load_3d(st + C::OFF_UK, &tmUK, 0, t * TT, urow, &wb[s]);
-        tma_load_3d(st + C::OFF_UV, &tmUV, 0, t * TT, urow, &wb[s]);
     };
-    // per-token scales and ranks of a tile, loaded by the lanes (tokens lane, lane+32, ...)
+    // per-token scales and ranks of a tile, loaded by the lanes (tokens lane, lane+32, ...);
+    // lane u-th token of the tile's code group u
     constexpr int TPL = TT / 32;
+    static_assert(TT % CODE_GROUP == 0 && CODE_GROUP == 32, "code groups of 32 tokens, one per lane set");
+    // whole warp: the tile's code-group sizes (pad16 of the summed code lengths) from
+    // its ranks, then lane 0 requests them
+    auto issue_codes = [&](int k, const unsigned (&rr)[TPL]) {
+        const int t = tile0 + warp + k * NW;
+        const int s = k % NSW;
+        unsigned gb[TPL], total = 0;
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            gb[u] = (__reduce_add_sync(0xffffffffu, static_cast<unsigned>(code_len(rr[u]))) + 15u) & ~15u;
+            total += gb[u];
+        }
+        if (lane == 0) {
+            uint8_t* st = ring + s * C::STAGE_BYTES;
+            mbar_arrive_expect_tx(&wb[s], 2 * total);
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) {
+                if (gb[u] == 0) continue;
+                const size_t g0 = (static_cast<size_t>(urow) * a.T + static_cast<size_t>(t) * TT + u * 32) * RM;
+                bulk_load(st + C::OFF_UK + u * 32 * RM, a.u_k + g0, gb[u], &wb[s]);
+                bulk_load(st + C::OFF_UV + u * 32 * RM, a.u_v + g0, gb[u], &wb[s]);
+            }
+        }
+    };
+    // ranks of the tokens of tile k this lane stands for (0 past the sequence)
+    auto ranks_of = [&](int k, unsigned (&rr)[TPL]) {
+        const int t0 = (tile0 + warp + k * NW) * TT;
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            const int tt = t0 + lane + 32 * u;
+            rr[u] = tt < tlen ? static_cast<unsigned>(__ldg(rank_row + tt)) : 0u;
+        }
+    };
     // raw 16-bit scales and 8-bit ranks: converted only when published, a tile later, so
     // nothing waits on these loads until then
     unsigned pf_sk[TPL], pf_sv[TPL], pf_r[TPL];
@@ -211,9 +245,17 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             bulk_load(vfac + RB * D * 2, static_cast<const uint16_t*>(a.r_v) + static_cast<size_t>(j) * RM * D,
                       RM * D * 2, &fac_bar[1]);
         }
+        const int first = min(NSW, my_n);
         if (lane == 0) {
-            for (int k = 0; k < min(NSW, my_n); ++k) issue(k);
+            for (int k = 0; k < first; ++k) issue_coef(k);
         }
+        unsigned r0[NSW][TPL];
+#pragma unroll
+        for (int k = 0; k < NSW; ++k)
+            if (k < first) ranks_of(k, r0[k]);
+#pragma unroll
+        for (int k = 0; k < NSW; ++k)
+            if (k < first) issue_codes(k, r0[k]);
         __syncwarp();
         if (my_n > 0) prefetch(0);
     };
@@ -337,7 +379,26 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             tks[TT + lane + 32 * u] = __half2float(__ushort_as_half(static_cast<unsigned short>(pf_sv[u])));
             tkr[lane + 32 * u] = static_cast<int>(pf_r[u]);
         }
+        // where each token's codes start in its group: the exclusive scan of the group's
+        // code lengths (lane = token), while the tile is still landing
+        int code_off[TPL];
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            const int kl = code_len(pf_r[u]);
+            int o = kl;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, o, d);
+                if (lane >= d) o += n;
+            }
+            code_off[u] = o - kl;
+        }
         if (k + 1 < my_n) prefetch(k + 1);
+        // ranks of the tile requested at the end of this one (loaded here, a register
+        // that no later iteration carries: a load still in flight across the loop's
+        // back edge made the whole step 2.2 us per layer slower)
+        unsigned nr[TPL];
+        if (k + NSW < my_n) ranks_of(k + NSW, nr);
         __syncwarp();
         const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&wb[s], (k / NSW) & 1, a.wait_limit, a.err));
         if (!ok) {
@@ -364,8 +425,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         for (int u = 0; u < TPL; ++u) {
             const int tr = lane + 32 * u;
             const int r = tkr[tr];
-            const uint4 wk = *reinterpret_cast<const uint4*>(ukp + tr * RM);
-            const uint4 wv = *reinterpret_cast<const uint4*>(uvp + tr * RM);
+            const uint4 wk = codes_at(ukp + u * 32 * RM + code_off[u]);
+            const uint4 wv = codes_at(uvp + u * 32 * RM + code_off[u]);
             uint32_t m0, m1, m2, m3;
             rank_keep4(r, m0, m1, m2, m3);
             uint4 k0, k1, v0, v1;
@@ -437,7 +498,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    sc[mt][nb][i] = __fmul_rn(fmaf(skr[mt][i >> 1], su[mt][nb][i], sc[mt][nb][i]), a.scale_log2);
+                    sc[mt][nb][i] = fmaf(skr[mt][i >> 1], su[mt][nb][i], sc[mt][nb][i]);   // raw score
             if (tail) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
@@ -454,7 +515,7 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                     for (int i = 0; i < 4; ++i) {
                         const int h = h0 + (i & 1);
                         const int r = mt * 16 + (lane >> 2) + (i >> 1) * 8;
-                        if (h < g && r < lim) srow[static_cast<size_t>(h) * a.T + t * TT + r] = sc[mt][nb][i];
+                        if (h < g && r < lim) srow[static_cast<size_t>(h) * a.T + t * TT + r] = __fmul_rn(sc[mt][nb][i], a.scale_log2);
                     }
             }
 #pragma unroll
@@ -467,6 +528,10 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
             }
+            // the row max in the scaled (log2) domain: scaling by a positive factor and
+            // rounding are monotonic, so this is the max of the scaled scores
+            mx0 = __fmul_rn(mx0, a.scale_log2);
+            mx1 = __fmul_rn(mx1, a.scale_log2);
             const float mn0 = fmaxf(mrow[nb][0], mx0), mn1 = fmaxf(mrow[nb][1], mx1);
             const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
             const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
@@ -483,8 +548,10 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const int ta = mt * 16 + (lane >> 2);
-                const float p0 = ex2_approx(sc[mt][nb][0] - ref0), p1 = ex2_approx(sc[mt][nb][1] - ref1);
-                const float p2 = ex2_approx(sc[mt][nb][2] - ref0), p3 = ex2_approx(sc[mt][nb][3] - ref1);
+                const float p0 = ex2_approx(fmaf(sc[mt][nb][0], a.scale_log2, -ref0));
+                const float p1 = ex2_approx(fmaf(sc[mt][nb][1], a.scale_log2, -ref1));
+                const float p2 = ex2_approx(fmaf(sc[mt][nb][2], a.scale_log2, -ref0));
+                const float p3 = ex2_approx(fmaf(sc[mt][nb][3], a.scale_log2, -ref1));
                 const uint32_t lo = pack_bf16(p0, p1), hi = pack_bf16(p2, p3);
                 lrow[nb][0] += bf16_lo(lo) + bf16_lo(hi);
                 lrow[nb][1] += bf16_hi(lo) + bf16_hi(hi);
@@ -520,9 +587,12 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             for (int nb = 0; nb < NB; ++nb) mma_f16(ou[nb], af, pvb[mt][nb][0], pvb[mt][nb][1]);
         }
         __syncwarp();
-        if (lane == 0 && k + NSW < my_n) {
-            fence_proxy_async();
-            issue(k + NSW);
+        if (k + NSW < my_n) {
+            if (lane == 0) {
+                fence_proxy_async();
+                issue_coef(k + NSW);
+            }
+            issue_codes(k + NSW, nr);
         }
     }
 #pragma unroll
@@ -629,7 +699,7 @@ cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t
     });
     if (e != cudaSuccess) return e;
     dim3 grid(a.splits, a.Hkv, a.B);
-    return launch_kernel(kern, grid, dim3(NW * 32), C::SMEM, st, a.pdl != 0, maps[0], maps[1], maps[2], maps[3], a);
+    return launch_kernel(kern, grid, dim3(NW * 32), C::SMEM, st, a.pdl != 0, maps[0], maps[1], a);
 }
 
 template <int D, int RB, int TT, int NSW, int NW>
@@ -655,6 +725,7 @@ int occupancy_of() {
 #ifndef KVS_LR_TT
 #define KVS_LR_TT 32
 #endif
+
 #ifndef KVS_LR_NSW
 #define KVS_LR_NSW 2
 #endif

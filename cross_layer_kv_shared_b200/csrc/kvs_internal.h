@@ -179,7 +179,7 @@ cudaError_t launch_decode_f32(bool mix, int d, const DecodeArgs& a, cudaStream_t
 
 int decode_lowrank_tile(int rb);
 int decode_lowrank_occupancy(int d, int rb);
-// maps: coef_k, coef_v (whole [P*B*Hkv][T][Rb]) and u_k, u_v (the layer's [B*Hkv][T][16])
+// maps: coef_k, coef_v (whole [P*B*Hkv][T][Rb]); the group-packed codes come through a.u_k, a.u_v
 cudaError_t launch_decode_lowrank(int d, int rb, const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st);
 
 cudaError_t launch_pack_residual(const PackArgs& a, cudaStream_t st);

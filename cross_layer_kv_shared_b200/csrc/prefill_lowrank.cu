@@ -21,6 +21,7 @@
 // the last warpgroup has the TMA producer and the MMA issuer. Every wait is bounded.
 #include <type_traits>
 
+#include "kvs_quant.cuh"
 #include "tc_sm100.cuh"
 
 namespace kvs {
@@ -116,6 +117,7 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     uint8_t* sW = smem + C::OFF_W;               // [B_V; R_V] [48][D] bf16
     uint8_t* sOut = smem + C::OFF_OUT;           // [NQ][D / 64][128][64] swizzled
     __shared__ __align__(8) LrSync sy;
+    __shared__ int conv_len[2][BN];              // code lengths of a tile's tokens (converters)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -338,6 +340,13 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             const float scale = __half2float(__ushort_as_half(static_cast<unsigned short>(pf_s[q])));
             const int rk = static_cast<int>(pf_r[q]);
             meta(j + PF, pf_s[q], pf_r[q]);
+            // where the token's codes start in its 32-token code group: after the codes of
+            // the group's earlier tokens (the converters exchange the tile's code lengths)
+            if (hf == 1 && m == 0) conv_len[j & 1][r] = code_len(static_cast<unsigned>(rk));
+            named_sync(3, C::CONV);
+            int o = 0;
+            if (hf == 1)
+                for (int i = r & ~31; i < r; ++i) o += conv_len[j & 1][i];
             wait_lr(sy, &sy.raw_full[sb], (j / NSB) & 1, a.wait_limit, a.err);
             if (j >= NS) wait_lr(sy, &sy.op_empty[s], ((j / NS) - 1) & 1, a.wait_limit, a.err);
             const uint8_t* raw = sB + sb * C::STAGE_B;
@@ -349,7 +358,7 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(op + swz128(r, c)) = src[c];
             } else {
                 // chunks 4-5: s * u for the first r_t codes (exact product, one bf16 rounding); 6-7: zero
-                const uint4 w = *reinterpret_cast<const uint4*>(raw + 2 * C::C_BYTES + m * C::U_BYTES + r * RM);
+                const uint4 w = codes_at(raw + 2 * C::C_BYTES + m * C::U_BYTES + (r & ~31) * RM + o);
                 const uint32_t words[4] = {w.x, w.y, w.z, w.w};
                 uint32_t pk[8];
 #pragma unroll

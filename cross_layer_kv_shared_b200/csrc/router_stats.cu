@@ -6,23 +6,22 @@
 // second component; Key Concepts, Token-Conditional Depth Routing). The decode
 // kernels keep every valid token's log2-domain scaled score s_{h,t} for the layer;
 // with the layer's lse (exact weight sums) each weight is p_{h,t} = 2^(s - lse/ln 2).
-// Each thread takes TPT tokens of one sequence (HB heads' scores loaded at a time) and writes
+// Each thread takes TPT tokens of one sequence (all of a pass's head scores loaded at once) and writes
 //   mass[j][t]  = sum over the g heads of kv head j of p_{h,t}
 //   score[t]    = x / (1 + x),  x = (T_b * sum_j mass[j][t]) / Hq     (fp32, in this order)
 // Tokens past the sequence get mass 0 and score 0. Per head, each block reduces its
 // entropy terms p (lse2 - s) ln 2 and its largest p in shared memory and stores one
 // partial; the last block of the sequence to finish (an arrival counter) adds the
-// partials in a fixed order (per thread, then a fixed tree), so entropy and peak are
-// deterministic.
+// partials in a fixed order (per lane over blocks, then the warps in order), so
+// entropy and peak are deterministic.
 #include "kvs_device.cuh"
 
 namespace kvs {
 namespace {
 
-constexpr int NT = 256;
+constexpr int NT = 128;
 constexpr int TPT = 1;                        // tokens per thread
-constexpr int HB = 16;                        // heads whose scores are loaded together
-constexpr int HC = 64;                        // heads reduced per pass through shared memory
+constexpr int HC = 32;                        // heads per pass: all their scores loaded at once
 constexpr float LOG2E_F = 1.4426950408889634f;
 
 __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
@@ -44,54 +43,63 @@ __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
     for (int k = 0; k < TPT; ++k) macc[k] = total[k] = 0.f;
     const int t0 = blockIdx.x * NT * TPT + threadIdx.x;   // this thread's tokens: t0 + k * NT
     const float* srow0 = a.sscore + static_cast<size_t>(b) * a.Hq * a.T;
+    int hg = 0, j = 0;                                   // head h = j g + hg, heads in order
     for (int h0 = 0; h0 < a.Hq; h0 += HC) {
         const int hn = min(HC, a.Hq - h0);
         if (threadIdx.x < hn) lse2_s[threadIdx.x] = a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] * LOG2E_F;
         __syncthreads();
-        for (int hb = 0; hb < hn; hb += HB) {
-            // the scores of HB heads first, all loads in flight together
-            float sv[HB][TPT];
+        // every score of the pass first, all loads in flight together
+        float sv[HC][TPT];
 #pragma unroll
-            for (int q = 0; q < HB; ++q)
+        for (int q = 0; q < HC; ++q)
+#pragma unroll
+            for (int k = 0; k < TPT; ++k) {
+                const int t = t0 + k * NT;
+                sv[q][k] = (q < hn && t < n) ? __ldcs(srow0 + static_cast<size_t>(h0 + q) * a.T + t) : 0.f;
+            }
+        // this thread's entropy terms and largest weight per head; reduced over the block
+        // after the pass, so the reductions of different heads overlap
+        float es[HC], pm[HC];
+#pragma unroll
+        for (int q = 0; q < HC; ++q) {
+            es[q] = pm[q] = 0.f;
+            if (q >= hn) continue;
+            const float l2 = lse2_s[q];
+#pragma unroll
+            for (int k = 0; k < TPT; ++k) {
+                const int t = t0 + k * NT;
+                float p = 0.f;
+                if (t < n) {
+                    p = exp2f(sv[q][k] - l2);
+                    es[q] += p * (l2 - sv[q][k]);
+                    pm[q] = fmaxf(pm[q], p);
+                }
+                macc[k] = hg == 0 ? p : macc[k] + p;
+            }
+            if (hg == a.g - 1) {                         // group complete: its mass, then the total
 #pragma unroll
                 for (int k = 0; k < TPT; ++k) {
                     const int t = t0 + k * NT;
-                    sv[q][k] = (hb + q < hn && t < n) ? __ldcs(srow0 + static_cast<size_t>(h0 + hb + q) * a.T + t) : 0.f;
+                    if (a.mass != nullptr && t < a.T) a.mass[(static_cast<size_t>(b) * a.Hkv + j) * a.T + t] = macc[k];
+                    total[k] = j == 0 ? macc[k] : __fadd_rn(total[k], macc[k]);
                 }
+                hg = 0;
+                ++j;
+            } else {
+                ++hg;
+            }
+        }
+        if (want_red) {
 #pragma unroll
-            for (int q = 0; q < HB; ++q) {
-                const int hh = hb + q;
-                if (hh >= hn) break;
-                const int h = h0 + hh;
-                const float l2 = lse2_s[hh];
-                float es = 0.f, pm = 0.f;
+            for (int q = 0; q < HC; ++q) {
+                es[q] = warp_sum(es[q]);
+                pm[q] = warp_max(pm[q]);
+            }
+            if (lane == 0) {
 #pragma unroll
-                for (int k = 0; k < TPT; ++k) {
-                    const int t = t0 + k * NT;
-                    float p = 0.f;
-                    if (t < n) {
-                        p = exp2f(sv[q][k] - l2);
-                        es += p * (l2 - sv[q][k]);
-                        pm = fmaxf(pm, p);
-                    }
-                    macc[k] = h % a.g == 0 ? p : macc[k] + p;   // kv head j = h / g, heads in order
-                }
-                if (h % a.g == a.g - 1) {                     // group complete: its mass, then the total
-                    const int j = h / a.g;
-#pragma unroll
-                    for (int k = 0; k < TPT; ++k) {
-                        const int t = t0 + k * NT;
-                        if (a.mass != nullptr && t < a.T) a.mass[(static_cast<size_t>(b) * a.Hkv + j) * a.T + t] = macc[k];
-                        total[k] = j == 0 ? macc[k] : __fadd_rn(total[k], macc[k]);
-                    }
-                }
-                if (want_red) {
-                    es = warp_sum(es);
-                    pm = warp_max(pm);
-                    if (lane == 0) {
-                        red_e[warp][hh] = es;
-                        red_p[warp][hh] = pm;
-                    }
+                for (int q = 0; q < HC; ++q) {
+                    red_e[warp][q] = es[q];
+                    red_p[warp][q] = pm[q];
                 }
             }
         }
@@ -127,44 +135,32 @@ __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
     __syncthreads();
     if (!last) return;
     __threadfence();
-    // thread i adds the partials of blocks i, i + NT, ... in order; a fixed tree over the
-    // threads (shuffles, then the warps in order) finishes each head
-    for (int h0 = 0; h0 < a.Hq; h0 += HC) {
-        const int hn = min(HC, a.Hq - h0);
-        for (int hb = 0; hb < hn; hb += HB) {
-            float ve[HB], vp[HB];
-#pragma unroll
-            for (int q = 0; q < HB; ++q) ve[q] = vp[q] = 0.f;
-            for (unsigned blk = threadIdx.x; blk < gridDim.x; blk += NT) {
-                const float* part = a.part + ((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h0 + hb) * 2;
-#pragma unroll
-                for (int q = 0; q < HB; ++q)
-                    if (hb + q < hn) {
-                        ve[q] += __ldcg(part + 2 * q);
-                        vp[q] = fmaxf(vp[q], __ldcg(part + 2 * q + 1));
-                    }
-            }
-#pragma unroll
-            for (int q = 0; q < HB; ++q) {
-                if (hb + q >= hn) break;
-                const float e = warp_sum(ve[q]);
-                const float p = warp_max(vp[q]);
-                if (lane == 0) {
-                    red_e[warp][hb + q] = e;
-                    red_p[warp][hb + q] = p;
-                }
+    // lane = head (32 at a time), warp w adds blocks w, w + 8, ... in order (coalesced
+    // rows of the partials); then the warps' sums in order: a fixed order throughout
+    for (int h0 = 0; h0 < a.Hq; h0 += 32) {
+        const int h = h0 + lane;
+        float e = 0.f, p = 0.f;
+        if (h < a.Hq) {
+#pragma unroll 8
+            for (unsigned blk = warp; blk < gridDim.x; blk += NT / 32) {
+                const float2 v = __ldcg(reinterpret_cast<const float2*>(
+                    a.part + ((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h) * 2));
+                e += v.x;
+                p = fmaxf(p, v.y);
             }
         }
+        red_e[warp][lane] = e;
+        red_p[warp][lane] = p;
         __syncthreads();
-        if (threadIdx.x < hn) {
-            float e = 0.f, p = 0.f;
+        if (threadIdx.x < 32 && h0 + threadIdx.x < a.Hq) {
+            float se = 0.f, sp = 0.f;
             for (int w = 0; w < NT / 32; ++w) {
-                e += red_e[w][threadIdx.x];
-                p = fmaxf(p, red_p[w][threadIdx.x]);
+                se += red_e[w][threadIdx.x];
+                sp = fmaxf(sp, red_p[w][threadIdx.x]);
             }
             const size_t o = static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x;
-            if (a.entropy != nullptr) a.entropy[o] = e * LN2_F;
-            if (a.peak != nullptr) a.peak[o] = p;
+            if (a.entropy != nullptr) a.entropy[o] = se * LN2_F;
+            if (a.peak != nullptr) a.peak[o] = sp;
         }
         __syncthreads();
     }

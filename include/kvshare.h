@@ -96,7 +96,18 @@ typedef struct {
     const void* coef_v;
     const void* basis_k;   /* [pairs][Hkv][Rb][d] bf16                           */
     const void* basis_v;
-    const int8_t* u_k;     /* [L][batch][Hkv][T][Rm] int8 residual codes         */
+    const int8_t* u_k;     /* [L][batch][Hkv][T x 16] int8 residual codes, group-
+                              packed: each (layer, sequence, kv head) row of T x 16
+                              bytes holds its tokens in groups of 32 (group g: tokens
+                              32g .. 32g+31, the last possibly shorter), group g owning
+                              bytes [512 g, 512 g + 16 n_g); within a group the tokens'
+                              code slots follow one another in token order, token t's
+                              slot k_t = 8 ceil(min(rank_t, 16) / 8) bytes (0, 8 or 16)
+                              holding its first min(rank_t, 16) codes, then zeros. The
+                              other bytes of a group are unused and never read: readers
+                              fetch the first pad16(sum of k) bytes of each group, so a
+                              rank-0 token costs no code traffic. kvshare_pack_residual
+                              and kvshare_append_lowrank write this layout. */
     const int8_t* u_v;
     const uint16_t* s_k;   /* [L][batch][Hkv][T] fp16 per-token residual scale   */
     const uint16_t* s_v;
@@ -215,11 +226,13 @@ kvshare_status kvshare_prefill(kvshare_t ctx, const kvshare_cache* cache, const 
  *   score [L][batch][T] fp32 router score -> rank [L][batch][T]:
  *         0 if score < 0.7f, 8 if score < 0.9f, else 16
  *   u_k, u_v [L][batch][Hkv][T][16] fp32 residual rows ->
- *   u_k8, u_v8 [L][batch][Hkv][T][16] int8 codes and s_k, s_v [L][batch][Hkv][T]
- *         fp16 scales: amax = max_{i<r}|u_i|, scale = fp16_rne(min(amax/127f, 65504)),
- *         code_i = clamp(rint(u_i / scale), -127, 127) for i < r, else 0;
+ *   u_k8, u_v8 [L][batch][Hkv][T x 16] int8 codes, group-packed (see
+ *         kvshare_cache.u_k: token t's codes 0 .. r_t - 1 only), and s_k, s_v
+ *         [L][batch][Hkv][T] fp16 scales: amax = max_{i<r}|u_i|,
+ *         scale = fp16_rne(min(amax/127f, 65504)),
+ *         code_i = clamp(rint(u_i / scale), -127, 127) for i < r;
  *         a zero scale gives zero codes. fp32 IEEE arithmetic, bit-exact.
- * Inputs must be finite. */
+ * Inputs must be finite. The unused bytes of each code group are not written. */
 kvshare_status kvshare_pack_residual(kvshare_t ctx, const float* score, const float* u_k,
                                      const float* u_v, uint8_t* rank, int8_t* u_k8, int8_t* u_v8,
                                      uint16_t* s_k, uint16_t* s_v, int batch, int context,
@@ -243,7 +256,11 @@ kvshare_status kvshare_pack_residual(kvshare_t ctx, const float* score, const fl
  *   score:        [L][batch] fp32 DEVICE router score of the token per layer
  *   pos:          [batch] int32 DEVICE token index to write; an index outside
  *                 [0, context) writes nothing for that sequence and makes the next
- *                 kvshare_sync_status return KVS_EINVAL.
+ *                 kvshare_sync_status return KVS_EINVAL. The token's codes go after
+ *                 those of its code group's earlier tokens (group-packed layout, by
+ *                 their stored ranks), so later tokens of the same 32-token group
+ *                 must not have been written yet (appends run in token order; the
+ *                 last token may be rewritten).
  * The caller then raises the sequences' lengths. A basis pair read by more than two
  * layers, or more than 64 pairs: KVS_EUNSUPPORTED. A decode that follows an append
  * on the same stream must run with kvshare_set_kv_overlap off. */

@@ -14,6 +14,7 @@ import oracle.kvshare_ref as ref
 import oracle.quant_ref as qr
 from synth.configs import Config, depthweave_map
 
+import code_layout as cl
 from gpu_helpers import assert_close, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -32,12 +33,14 @@ def layers_of_pair(cfg, p):
 
 
 def host_state(d, packed):
+    """The device state on the host; the group-packed codes as dense [..., T, 16] by the stored ranks."""
     rank, ck, cv, sk, sv = packed
+    r = rank.cpu().numpy().copy()
     return {"coef_k": d["coef_k"].cpu().numpy().view(np.uint16).copy(),
             "coef_v": d["coef_v"].cpu().numpy().view(np.uint16).copy(),
-            "u_k": ck.cpu().numpy().copy(), "u_v": cv.cpu().numpy().copy(),
+            "u_k": cl.unpack(ck.cpu().numpy(), r), "u_v": cl.unpack(cv.cpu().numpy(), r),
             "s_k": sk.cpu().numpy().view(np.uint16).copy(), "s_v": sv.cpu().numpy().view(np.uint16).copy(),
-            "rank": rank.cpu().numpy().copy()}
+            "rank": r}
 
 
 def oracle_append(cfg, state, inp, k_new, v_new, score, pos):
@@ -106,12 +109,20 @@ def test_append_is_bit_exact_and_decodes(K, shape):
             want = oracle_append(cfg, state, inp, k_new, v_new, score, pos)
             got = host_state(d, packed)
             for name in want:
-                assert np.array_equal(got[name], want[name]), (step, name)
+                if name in ("u_k", "u_v"):
+                    # codes of the tokens up to the append (later tokens of a code group
+                    # move with the appended token's length: past the sequence, undefined)
+                    for b in range(cfg.batch):
+                        n = int(pos[b]) + 1
+                        assert np.array_equal(got[name][:, b, :, :n], want[name][:, b, :, :n]), (step, name, b)
+                else:
+                    assert np.array_equal(got[name], want[name]), (step, name)
             state = want
+            last = pos
             pos = np.minimum(pos + 1, cfg.context - 1)
-        # decode over each sequence's tokens up to the last append
-        lens = pos + 1
-        lens[1] = cfg.context
+        # decode over each sequence's tokens up to the last append (a token after it in
+        # the same code group moved with the appended token's code length)
+        lens = last + 1
         out = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim, device="cuda")
         lse = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, device="cuda")
         cache.lengths = torch.from_numpy(lens.astype(np.int32)).cuda()

@@ -7,6 +7,7 @@ import oracle.quant_ref as qr
 import synth.gpu as sgpu
 from synth.configs import DEPTHWEAVE_DECODE, LOWRANK, SINGLE, Config, depthweave_map
 
+import code_layout as cl
 from gpu_helpers import assert_scaled, assert_close, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -67,7 +68,8 @@ def run_small(K, cfg, inp=None, kv_overlap=False, splits=0):
         assert K.kvshare_sync_status(h) == K.KVS_OK
     finally:
         K.kvshare_destroy(h)
-    packed = tuple(x.cpu().numpy() for x in (rank, ck, cv, sk, sv))
+    rank, ck, cv, sk, sv = (x.cpu().numpy() for x in (rank, ck, cv, sk, sv))
+    packed = (rank, cl.unpack(ck, rank), cl.unpack(cv, rank), sk, sv)   # codes as dense [..., T, 16]
     return out.cpu().numpy(), lse.cpu().numpy(), packed, inp
 
 
@@ -124,8 +126,10 @@ def test_pack_edge_rows(K):
     finally:
         K.kvshare_destroy(h)
     want = qr.pack_residual(score, u, u[:, :, ::-1].copy())
-    for got, exp in zip(packed, want):
-        assert np.array_equal(got.cpu().numpy().view(exp.dtype), exp)
+    got = [x.cpu().numpy() for x in packed]
+    got[1], got[2] = cl.unpack(got[1], got[0]), cl.unpack(got[2], got[0])   # group-packed codes as dense
+    for g_, exp in zip(got, want):
+        assert np.array_equal(g_.view(exp.dtype), exp)
 
 
 def test_full_rank_identity_basis_equals_single_source(K):
@@ -238,8 +242,8 @@ def test_full_size_sampled(K):
     worst = scale = 0.0
     for (l, j), (o, s_, r, codes_k, codes_v, sck, scv) in zip(units, res):
         assert np.array_equal(rank_d[l, 0], r)
-        assert np.array_equal(ck_d[l, 0, j], codes_k)
-        assert np.array_equal(cv_d[l, 0, j], codes_v)
+        assert np.array_equal(cl.unpack_row(ck_d[l, 0, j], rank_d[l, 0]), codes_k)
+        assert np.array_equal(cl.unpack_row(cv_d[l, 0, j], rank_d[l, 0]), codes_v)
         assert np.array_equal(sk_d[l, 0, j], sck)
         assert np.array_equal(sv_d[l, 0, j], scv)
         worst = max(worst, assert_close(out[l, 0, j * g:(j + 1) * g], o, TOL, f"l{l} j{j}")[0])
