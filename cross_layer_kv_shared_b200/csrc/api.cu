@@ -99,9 +99,8 @@ struct kvshare_ctx {
     float* sscore = nullptr;
     // projected queries of one low-rank prefill layer [max_batch][Hq][max_context][64] bf16
     uint16_t* qp = nullptr;
-    // statistics kernel: per-block entropy/peak partials and per-sequence arrival counters
+    // statistics kernel: per-block entropy/peak partials
     float* stats_part = nullptr;
-    unsigned* stats_counters = nullptr;
     // staging for kvshare_decode_host
     void* q_stage = nullptr;
     float* out_stage = nullptr;
@@ -367,15 +366,15 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
             sa.entropy = stats->entropy ? stats->entropy + lbt * Hq : nullptr;
             sa.peak = stats->peak ? stats->peak + lbt * Hq : nullptr;
             sa.part = c->stats_part;
-            sa.counters = c->stats_counters;
             sa.err = c->err;
             sa.B = B;
             sa.Hq = Hq;
             sa.Hkv = Hkv;
             sa.T = T;
             sa.g = g;
-            if (launch_router_stats(sa, st) != cudaSuccess) return KVS_ECUDA;
-            ++c->launches;
+            const int n = launch_router_stats(sa, st);
+            if (n < 0) return KVS_ECUDA;
+            c->launches += n;
         }
     }
     return KVS_OK;
@@ -543,7 +542,6 @@ kvshare_status kvshare_destroy(kvshare_t ctx) {
     cudaFree(ctx->sscore);
     cudaFree(ctx->qp);
     cudaFree(ctx->stats_part);
-    cudaFree(ctx->stats_counters);
     cudaFree(ctx->q_stage);
     cudaFree(ctx->out_stage);
     cudaFree(ctx->lse_stage);
@@ -626,16 +624,12 @@ kvshare_status kvshare_decode_stats(kvshare_t ctx, const kvshare_cache* cache, c
         const size_t n = static_cast<size_t>(cf.max_batch) * cf.num_q_heads * cf.max_context;
         const size_t np = static_cast<size_t>(cf.max_batch) * router_stats_blocks(cf.max_context) * cf.num_q_heads * 2;
         if (cudaMalloc(&ctx->sscore, n * sizeof(float)) != cudaSuccess ||
-            cudaMalloc(&ctx->stats_part, np * sizeof(float)) != cudaSuccess ||
-            cudaMalloc(&ctx->stats_counters, cf.max_batch * sizeof(unsigned)) != cudaSuccess ||
-            cudaMemset(ctx->stats_counters, 0, cf.max_batch * sizeof(unsigned)) != cudaSuccess) {
+            cudaMalloc(&ctx->stats_part, np * sizeof(float)) != cudaSuccess) {
             cudaGetLastError();
             cudaFree(ctx->sscore);
             cudaFree(ctx->stats_part);
-            cudaFree(ctx->stats_counters);
             ctx->sscore = nullptr;
             ctx->stats_part = nullptr;
-            ctx->stats_counters = nullptr;
             return KVS_ENOMEM;
         }
     }

@@ -100,12 +100,13 @@ struct StatsArgs {
     float* entropy;         // [B][Hq] or nullptr
     float* peak;            // [B][Hq] or nullptr
     float* part;            // [B][blocks][Hq][2] per-block entropy and peak partials
-    unsigned* counters;     // [B] arrival counters, zero between launches
     unsigned* err;
     int B, Hq, Hkv, T, g;
 };
 int router_stats_blocks(int T);
-cudaError_t launch_router_stats(const StatsArgs& a, cudaStream_t st);
+// launches the statistics kernel and, when entropy or peak is asked for, the kernel that
+// finishes them; returns the number of launches, or -1 on a launch error
+int launch_router_stats(const StatsArgs& a, cudaStream_t st);
 
 // Append of one new token to a low-rank cache (every basis pair, sequence and kv head).
 constexpr int APPEND_MAX_PAIRS = 64;

@@ -64,7 +64,7 @@ struct LrPfCfg {
     static constexpr int LAUNCH_REGS = 96;
     static constexpr int REG_SOFTMAX = 152;
     static constexpr int REG_CONV = 56;
-    static constexpr int REG_CTRL = 48;
+    static constexpr int REG_CTRL = 64;
     static constexpr int REG_SUM = 2 * 128 * REG_SOFTMAX + CONV * REG_CONV + 128 * REG_CTRL;
     static_assert(REG_SUM <= THREADS * LAUNCH_REGS, "register split exceeds the launch allocation");
 };
@@ -427,27 +427,24 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             if (lane == 0) {
                 constexpr uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
                 constexpr uint32_t idO = tc::idesc_bf16(BM, QW, false, true);
-                const uint32_t q_addr = smem_u32(sQ);
+                // descriptors: one base per operand tile, then the start-address field
+                // (address >> 4, in the low bits) advanced by a constant per K step
                 auto issue_s = [&](int i, int j) {          // S_i = Q'_i K'_j^T
-                    const uint32_t k_addr = smem_u32(sA + (j % NS) * C::STAGE_A);
+                    const uint64_t qd = tc::smem_desc(smem_u32(sQ + i * C::Q_BYTES), 16, 1024, tc::LAYOUT_SW128);
+                    const uint64_t kd = tc::smem_desc(smem_u32(sA + (j % NS) * C::STAGE_A), 16, 1024, tc::LAYOUT_SW128);
 #pragma unroll
-                    for (int kk = 0; kk < QW / 16; ++kk) {
-                        const uint32_t off = kk * 32;
-                        const uint64_t ad = tc::smem_desc(q_addr + i * C::Q_BYTES + off, 16, 1024, tc::LAYOUT_SW128);
-                        const uint64_t bd = tc::smem_desc(k_addr + off, 16, 1024, tc::LAYOUT_SW128);
-                        tc::mma_ss(tS(i), ad, bd, idS, kk > 0 ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < QW / 16; ++kk)
+                        tc::mma_ss(tS(i), qd + ((kk * 32) >> 4), kd + ((kk * 32) >> 4), idS, kk > 0 ? 1u : 0u);
                     tc::commit(&sy.s_full[i]);
                 };
                 auto issue_pv = [&](int i, int j) {         // O'_i += P_i V'_j, P_i from TMEM
                     wait_lr(sy, &sy.p_full[i], j & 1, a.wait_limit, a.err);
                     tc::fence_after();
-                    const uint32_t v_addr = smem_u32(sA + (j % NS) * C::STAGE_A + C::OP_TILE);
+                    const uint64_t vd = tc::smem_desc(smem_u32(sA + (j % NS) * C::STAGE_A + C::OP_TILE), BN * 128, 1024,
+                                                      tc::LAYOUT_SW128);
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        const uint64_t bd = tc::smem_desc(v_addr + kk * 16 * 128, BN * 128, 1024, tc::LAYOUT_SW128);
-                        tc::mma_ts(tO(i), tS(i) + kk * 8, bd, idO, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        tc::mma_ts(tO(i), tS(i) + kk * 8, vd + ((kk * 16 * 128) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
                 };
                 auto wait_op = [&](int j) {
                     wait_lr(sy, &sy.op_ready[j % NS], (j / NS) & 1, a.wait_limit, a.err);

@@ -63,9 +63,9 @@ struct PfCfg {
     // per-thread registers after the split (setmaxnreg): the softmax threads hold a whole
     // S row; the sum over the block must not exceed what the block was launched with
     static constexpr int LAUNCH_REGS = MIX ? 96 : 168;
-    static constexpr int REG_SOFTMAX = MIX ? 152 : 224;
+    static constexpr int REG_SOFTMAX = MIX ? 152 : 216;
     static constexpr int REG_MIXER = 56;
-    static constexpr int REG_CTRL = MIX ? 48 : 56;
+    static constexpr int REG_CTRL = 64;
     static constexpr int REG_SUM = 2 * 128 * REG_SOFTMAX + (MIX ? MIXERS * REG_MIXER : 0) + 128 * REG_CTRL;
     static_assert(REG_SUM <= THREADS * LAUNCH_REGS, "register split exceeds the launch allocation");
     static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
@@ -435,15 +435,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (lane == 0) {
                 constexpr uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
                 constexpr uint32_t idO = tc::idesc_bf16(BM, D, false, true);
-                const uint32_t q_addr = smem_u32(sQ);
+                // descriptors: one base per operand tile, then the start-address field
+                // (address >> 4, in the low bits) advanced by a constant per K step
                 auto issue_s = [&](int i, int j) {          // S_i = Q_i K_j^T
-                    const uint32_t k_addr = smem_u32(sKV + (j % NS) * C::STAGE);
+                    const uint64_t qd = tc::smem_desc(smem_u32(sQ + i * C::Q_BYTES), 16, 1024, tc::LAYOUT_SW128);
+                    const uint64_t kd = tc::smem_desc(smem_u32(sKV + (j % NS) * C::STAGE), 16, 1024, tc::LAYOUT_SW128);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk & 3) * 32;   // 16 bf16 along K inside the 128-B row
-                        const uint64_t ad = tc::smem_desc(q_addr + i * C::Q_BYTES + (kk >> 2) * (BM * 128) + off, 16, 1024,
-                                                          tc::LAYOUT_SW128);
-                        const uint64_t bd = tc::smem_desc(k_addr + (kk >> 2) * C::HALF_T + off, 16, 1024, tc::LAYOUT_SW128);
+                        // 16 bf16 along K inside the 128-B row, then the next 64-column half
+                        const uint32_t off = (kk & 3) * 32;
+                        const uint64_t ad = qd + (((kk >> 2) * (BM * 128) + off) >> 4);
+                        const uint64_t bd = kd + (((kk >> 2) * C::HALF_T + off) >> 4);
                         tc::mma_ss(tS(i), ad, bd, idS, kk > 0 ? 1u : 0u);
                     }
                     tc::commit(&sy.s_full[i]);
@@ -451,12 +453,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 auto issue_pv = [&](int i, int j) {         // O_i += P_i V_j, P_i read from TMEM
                     wait_cta(sy, &sy.p_full[i], j & 1, a.wait_limit, a.err);
                     tc::fence_after();
-                    const uint32_t v_addr = smem_u32(sKV + (j % NS) * C::STAGE + C::TILE);
+                    const uint64_t vd =
+                        tc::smem_desc(smem_u32(sKV + (j % NS) * C::STAGE + C::TILE), C::HALF_T, 1024, tc::LAYOUT_SW128);
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        const uint64_t bd = tc::smem_desc(v_addr + kk * 16 * 128, C::HALF_T, 1024, tc::LAYOUT_SW128);
-                        tc::mma_ts(tO(i), tS(i) + kk * 8, bd, idO, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        tc::mma_ts(tO(i), tS(i) + kk * 8, vd + ((kk * 16 * 128) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
                 };
                 auto wait_kv = [&](int j) {
                     wait_cta(sy, MIX ? &sy.kv_ready[j % NS] : &sy.kv_full[j % NS], (j / NS) & 1, a.wait_limit, a.err);

@@ -11,9 +11,8 @@
 //   score[t]    = x / (1 + x),  x = (T_b * sum_j mass[j][t]) / Hq     (fp32, in this order)
 // Tokens past the sequence get mass 0 and score 0. Per head, each block reduces its
 // entropy terms p (lse2 - s) ln 2 and its largest p in shared memory and stores one
-// partial; the last block of the sequence to finish (an arrival counter) adds the
-// partials in a fixed order (per lane over blocks, then the warps in order), so
-// entropy and peak are deterministic.
+// partial; a second small kernel (one block per sequence and head) adds the partials
+// in a fixed order, so entropy and peak are deterministic.
 #include "kvs_device.cuh"
 
 namespace kvs {
@@ -126,55 +125,52 @@ __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
             a.score[static_cast<size_t>(b) * a.T + t] = __fdiv_rn(x, __fadd_rn(1.f, x));
         }
     }
-    if (!want_red) return;
-    // the last block of the sequence to arrive adds the per-block partials
-    __threadfence();
-    __shared__ unsigned last;
-    __syncthreads();
-    if (threadIdx.x == 0) last = atomicAdd(a.counters + b, 1u) == gridDim.x - 1 ? 1u : 0u;
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    // lane = head (32 at a time), warp w adds blocks w, w + 8, ... in order (coalesced
-    // rows of the partials); then the warps' sums in order: a fixed order throughout
-    for (int h0 = 0; h0 < a.Hq; h0 += 32) {
-        const int h = h0 + lane;
-        float e = 0.f, p = 0.f;
-        if (h < a.Hq) {
-#pragma unroll 8
-            for (unsigned blk = warp; blk < gridDim.x; blk += NT / 32) {
-                const float2 v = __ldcg(reinterpret_cast<const float2*>(
-                    a.part + ((static_cast<size_t>(b) * gridDim.x + blk) * a.Hq + h) * 2));
-                e += v.x;
-                p = fmaxf(p, v.y);
-            }
-        }
-        red_e[warp][lane] = e;
-        red_p[warp][lane] = p;
-        __syncthreads();
-        if (threadIdx.x < 32 && h0 + threadIdx.x < a.Hq) {
-            float se = 0.f, sp = 0.f;
-            for (int w = 0; w < NT / 32; ++w) {
-                se += red_e[w][threadIdx.x];
-                sp = fmaxf(sp, red_p[w][threadIdx.x]);
-            }
-            const size_t o = static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x;
-            if (a.entropy != nullptr) a.entropy[o] = se * LN2_F;
-            if (a.peak != nullptr) a.peak[o] = sp;
-        }
-        __syncthreads();
+}
+
+// Entropy and peak of every (sequence, head) from the per-block partials: thread i adds
+// blocks i, i + 256, ... in order, then a fixed tree (shuffles, the warps in order).
+constexpr int NF = 256;
+__global__ void __launch_bounds__(NF) router_stats_final_kernel(const StatsArgs a, int blocks) {
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float e = 0.f, p = 0.f;
+#pragma unroll 4
+    for (int blk = threadIdx.x; blk < blocks; blk += NF) {
+        const float2 v = *reinterpret_cast<const float2*>(a.part + ((static_cast<size_t>(b) * blocks + blk) * a.Hq + h) * 2);
+        e += v.x;
+        p = fmaxf(p, v.y);
     }
-    if (threadIdx.x == 0) a.counters[b] = 0u;
+    e = warp_sum(e);
+    p = warp_max(p);
+    __shared__ float we[NF / 32], wp[NF / 32];
+    if (lane == 0) {
+        we[warp] = e;
+        wp[warp] = p;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float se = 0.f, sp = 0.f;
+        for (int w = 0; w < NF / 32; ++w) {
+            se += we[w];
+            sp = fmaxf(sp, wp[w]);
+        }
+        const size_t o = static_cast<size_t>(b) * a.Hq + h;
+        if (a.entropy != nullptr) a.entropy[o] = se * LN2_F;
+        if (a.peak != nullptr) a.peak[o] = sp;
+    }
 }
 
 }  // namespace
 
 int router_stats_blocks(int T) { return (T + NT * TPT - 1) / (NT * TPT); }
 
-cudaError_t launch_router_stats(const StatsArgs& a, cudaStream_t st) {
-    dim3 grid(router_stats_blocks(a.T), a.B);
-    router_stats_kernel<<<grid, NT, 0, st>>>(a);
-    return cudaGetLastError();
+int launch_router_stats(const StatsArgs& a, cudaStream_t st) {
+    const int blocks = router_stats_blocks(a.T);
+    router_stats_kernel<<<dim3(blocks, a.B), NT, 0, st>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    if (a.entropy == nullptr && a.peak == nullptr) return 1;
+    router_stats_final_kernel<<<dim3(a.Hq, a.B), NF, 0, st>>>(a, blocks);
+    return cudaGetLastError() == cudaSuccess ? 2 : -1;
 }
 
 }  // namespace kvs

@@ -175,7 +175,8 @@ kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const v
  * Any of the four may be NULL; lse is required. The first call with an output
  * allocates a score buffer of max_batch x Hq x max_context floats and a small
  * reduction buffer in the context (KVS_ENOMEM if that fails); each layer adds one
- * statistics kernel after its decode kernel. Results are the same bits run to run. */
+ * statistics kernel after its decode kernel, and a second small one when entropy or
+ * peak is asked for. Results are the same bits run to run. */
 kvshare_status kvshare_decode_stats(kvshare_t ctx, const kvshare_cache* cache, const void* q, float* out,
                                     float* lse, float* mass, float* score, float* entropy, float* peak,
                                     int l0, int l1, void* stream);
