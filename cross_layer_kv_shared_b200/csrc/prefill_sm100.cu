@@ -17,7 +17,7 @@
 //                 that the tensor core computes one tile's product while the other
 //                 tile's softmax runs:  S = Q K^T  (A, B from shared memory)
 //                                       O += P V  (A = P straight from TMEM, B = V from shared)
-//   warpgroups 2, 3 (two-source layers only) mixers: K~ = w K1 + (1-w) K2 and the
+//   warpgroup 2 (two-source layers only) mixers: K~ = w K1 + (1-w) K2 and the
 //                 same for V, in fp32, rounded once to bf16, written in place over
 //                 the first source's tile, so the MMA reads the mixed operand and
 //                 the mixed K/V never reach HBM ("DepthGraft: Structural
@@ -36,6 +36,9 @@ namespace {
 constexpr int BM = 128;   // rows per query tile
 constexpr int NQ = 2;     // query tiles per CTA
 constexpr int NS_MAX = 3;   // K/V stages of the first-source ring, at most
+#ifndef KVS_PF_MIXERS
+#define KVS_PF_MIXERS 128
+#endif
 
 template <int D, bool MIX>
 struct PfCfg {
@@ -55,15 +58,17 @@ struct PfCfg {
     static_assert(NS <= NS_MAX, "ring A depth");
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static constexpr uint32_t TMEM_COLS = 512;     // S0 | S1 | O0 | O1
-    // warpgroups: 0, 1 softmax; MIX: 2, 3 mixers, 4 TMA + MMA (+2 idle); single: 2 TMA + MMA (+2 idle)
-    static constexpr int MIXERS = 256;                      // mixer threads (two warpgroups)
-    static constexpr int THREADS = MIX ? 640 : 384;
+    // warpgroups: 0, 1 softmax; MIX: 2 mixers, 3 TMA + MMA (+2 idle); single: 2 TMA + MMA (+2 idle)
+    // (one mixer warpgroup measured faster than two: mix layers 619 -> 629 TFLOP/s, the
+    // mixers still run ahead, and the softmax threads get 184 registers instead of 152)
+    static constexpr int MIXERS = KVS_PF_MIXERS;            // mixer threads (whole warpgroups)
+    static constexpr int THREADS = MIX ? 384 + MIXERS : 384;
     static constexpr int W_MIX = 8;
-    static constexpr int W_TMA = MIX ? 16 : 8, W_MMA = W_TMA + 1;
+    static constexpr int W_TMA = MIX ? 8 + MIXERS / 32 : 8, W_MMA = W_TMA + 1;
     // per-thread registers after the split (setmaxnreg): the softmax threads hold a whole
     // S row; the sum over the block must not exceed what the block was launched with
-    static constexpr int LAUNCH_REGS = MIX ? 96 : 168;
-    static constexpr int REG_SOFTMAX = MIX ? 152 : 216;
+    static constexpr int LAUNCH_REGS = MIX ? (MIXERS == 128 ? 128 : 96) : 168;
+    static constexpr int REG_SOFTMAX = MIX ? (MIXERS == 128 ? 184 : 152) : 216;
     static constexpr int REG_MIXER = 56;
     static constexpr int REG_CTRL = 64;
     static constexpr int REG_SUM = 2 * 128 * REG_SOFTMAX + (MIX ? MIXERS * REG_MIXER : 0) + 128 * REG_CTRL;
