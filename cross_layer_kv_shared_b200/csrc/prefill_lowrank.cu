@@ -16,7 +16,7 @@
 // two-source prefill: one CTA = two 128-row query tiles of one head; warpgroups 0, 1
 // run the softmax of one query tile each (one thread per row, P written back into
 // TMEM as bf16 and read from there by the PV product) and the epilogue
-// o = O' W / l; warpgroups 2, 3 convert each raw tile (coefficients by TMA, int8
+// o = O' W / l; warpgroup 2 converts each raw tile (coefficients by TMA, int8
 // codes by TMA, per-token scales and ranks by plain loads) into the K', V' operands;
 // the last warpgroup has the TMA producer and the MMA issuer. Every wait is bounded.
 #include <type_traits>
@@ -57,13 +57,16 @@ struct LrPfCfg {
                   "TMA destinations 128-byte aligned, swizzled tiles 1024-byte aligned");
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static constexpr uint32_t TMEM_COLS = 256;         // S0 | S1 | O'0 | O'1
-    static constexpr int CONV = 256;                   // converter threads (two warpgroups)
-    static constexpr int THREADS = 640;
+    // converter threads: one warpgroup, each thread a whole token row of K' or V' (two
+    // warpgroups that split each row measured 8% slower over the layer: more threads
+    // contending for the shared-memory pipes and fewer registers for softmax)
+    static constexpr int CONV = 128;
+    static constexpr int THREADS = 384 + CONV;
     static constexpr int W_CONV = 8;
-    static constexpr int W_TMA = 16, W_MMA = 17;
-    static constexpr int LAUNCH_REGS = 96;
-    static constexpr int REG_SOFTMAX = 152;
-    static constexpr int REG_CONV = 56;
+    static constexpr int W_TMA = 8 + CONV / 32, W_MMA = W_TMA + 1;
+    static constexpr int LAUNCH_REGS = 128;
+    static constexpr int REG_SOFTMAX = 184;
+    static constexpr int REG_CONV = 72;
     static constexpr int REG_CTRL = 64;
     static constexpr int REG_SUM = 2 * 128 * REG_SOFTMAX + CONV * REG_CONV + 128 * REG_CTRL;
     static_assert(REG_SUM <= THREADS * LAUNCH_REGS, "register split exceeds the launch allocation");
@@ -308,11 +311,10 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     } else if (wg >= C::W_CONV / 4 && wg < C::W_CONV / 4 + C::CONV / 128) {
         tc::reg_dec<C::REG_CONV>();
         // ------------------------------------------------------------ converters: raw tiles -> K', V'
-        // thread t: operand m (0: K', 1: V'), token row r of the tile, half hf of the 128-byte row
+        // thread t: operand m (0: K', 1: V') and token row r of the tile (the whole 128-byte row)
         const int t = threadIdx.x - 32 * C::W_CONV;
-        const int m = t >> 7;
-        const int r = (t & 127) >> 1;
-        const int hf = t & 1;
+        const int m = t >> 6;
+        const int r = t & 63;
         const size_t tok_row = (static_cast<size_t>(b) * a.Hkv + jkv) * a.T;
         const uint16_t* s_src = m == 0 ? a.s_k : a.s_v;
         // the token's scale bits and rank, loaded PF tiles ahead of their use (plain loads;
@@ -323,7 +325,7 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             const int tok = jj * BN + r;
             sb = 0u;
             rb = 0u;
-            if (hf == 1 && jj < n_kv && tok < a.S) {     // rows past the sequence stay zero
+            if (jj < n_kv && tok < a.S) {                // rows past the sequence stay zero
                 sb = s_src[tok_row + tok];
                 rb = a.rank[static_cast<size_t>(b) * a.T + tok];
             }
@@ -342,21 +344,21 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             meta(j + PF, pf_s[q], pf_r[q]);
             // where the token's codes start in its 32-token code group: after the codes of
             // the group's earlier tokens (the converters exchange the tile's code lengths)
-            if (hf == 1 && m == 0) conv_len[j & 1][r] = code_len(static_cast<unsigned>(rk));
+            if (m == 0) conv_len[j & 1][r] = code_len(static_cast<unsigned>(rk));
             named_sync(3, C::CONV);
             int o = 0;
-            if (hf == 1)
-                for (int i = r & ~31; i < r; ++i) o += conv_len[j & 1][i];
+            for (int i = r & ~31; i < r; ++i) o += conv_len[j & 1][i];
             wait_lr(sy, &sy.raw_full[sb], (j / NSB) & 1, a.wait_limit, a.err);
             if (j >= NS) wait_lr(sy, &sy.op_empty[s], ((j / NS) - 1) & 1, a.wait_limit, a.err);
             const uint8_t* raw = sB + sb * C::STAGE_B;
             uint8_t* op = sA + s * C::STAGE_A + m * C::OP_TILE;
-            if (hf == 0) {
+            {
                 // chunks 0-3: the 32 coefficients, copied into the swizzled row
                 const uint4* src = reinterpret_cast<const uint4*>(raw + m * C::C_BYTES + r * (RB * 2));
 #pragma unroll
                 for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(op + swz128(r, c)) = src[c];
-            } else {
+            }
+            {
                 // chunks 4-5: s * u for the first r_t codes (exact product, one bf16 rounding); 6-7: zero
                 const uint4 w = codes_at(raw + 2 * C::C_BYTES + m * C::U_BYTES + (r & ~31) * RM + o);
                 const uint32_t words[4] = {w.x, w.y, w.z, w.w};
