@@ -23,7 +23,31 @@ constexpr int TPT = 1;                        // tokens per thread
 constexpr int HC = 32;                        // heads per pass: all their scores loaded at once
 constexpr float LOG2E_F = 1.4426950408889634f;
 
-__global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
+// Reduces 32 per-lane values across the warp in 31 shuffles (16 + 8 + 4 + 2 + 1):
+// at the step of width w every lane keeps the half of its values whose index has bit
+// w equal to its own lane bit, adds the partner's copy of that half and sends the
+// other half. Lane i ends with the total of index i in v[0]. Sum (MAX false) or max.
+template <bool MAX>
+__device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane) {
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+        const bool upper = (lane & w) != 0;
+#pragma unroll
+        for (int k = 0; k < w; ++k) {
+            const float keep = upper ? v[k + w] : v[k];
+            const float send = upper ? v[k] : v[k + w];
+            const float got = __shfl_xor_sync(0xffffffffu, send, w);
+            v[k] = MAX ? fmaxf(keep, got) : keep + got;
+        }
+    }
+    return v[0];
+}
+
+__global__ void __launch_bounds__(NT, 4) router_stats_kernel(const StatsArgs a) {
+    // dependent launch: the decode's scores and lse are read only after it completes;
+    // the next kernel may then be scheduled while this one runs
+    grid_dep_wait();
+    if (threadIdx.x == 0) grid_dep_launch();
     const int b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int n = a.T;
@@ -35,6 +59,7 @@ __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
         }
     }
     const bool want_red = a.entropy != nullptr || a.peak != nullptr;
+    static_assert(HC == 32, "one head per lane in the block reduction");
     __shared__ float red_e[NT / 32][HC], red_p[NT / 32][HC];
     __shared__ float lse2_s[HC];
     float macc[TPT], total[TPT];
@@ -89,18 +114,9 @@ __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
             }
         }
         if (want_red) {
-#pragma unroll
-            for (int q = 0; q < HC; ++q) {
-                es[q] = warp_sum(es[q]);
-                pm[q] = warp_max(pm[q]);
-            }
-            if (lane == 0) {
-#pragma unroll
-                for (int q = 0; q < HC; ++q) {
-                    red_e[warp][q] = es[q];
-                    red_p[warp][q] = pm[q];
-                }
-            }
+            // lane q ends with head q's warp total and largest weight
+            red_e[warp][lane] = warp_transpose_reduce<false>(es, lane);
+            red_p[warp][lane] = warp_transpose_reduce<true>(pm, lane);
         }
         __syncthreads();
         if (want_red && threadIdx.x < hn) {
@@ -131,6 +147,8 @@ __global__ void __launch_bounds__(NT) router_stats_kernel(const StatsArgs a) {
 // blocks i, i + 256, ... in order, then a fixed tree (shuffles, the warps in order).
 constexpr int NF = 256;
 __global__ void __launch_bounds__(NF) router_stats_final_kernel(const StatsArgs a, int blocks) {
+    grid_dep_wait();
+    if (threadIdx.x == 0) grid_dep_launch();
     const int h = blockIdx.x, b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float e = 0.f, p = 0.f;
@@ -166,11 +184,13 @@ int router_stats_blocks(int T) { return (T + NT * TPT - 1) / (NT * TPT); }
 
 int launch_router_stats(const StatsArgs& a, cudaStream_t st) {
     const int blocks = router_stats_blocks(a.T);
-    router_stats_kernel<<<dim3(blocks, a.B), NT, 0, st>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return -1;
+    // both launches are dependent launches: their start overlaps the tail of the kernel
+    // ahead, and they wait for it before touching memory
+    if (launch_kernel(router_stats_kernel, dim3(blocks, a.B), dim3(NT), 0, st, true, a) != cudaSuccess) return -1;
     if (a.entropy == nullptr && a.peak == nullptr) return 1;
-    router_stats_final_kernel<<<dim3(a.Hq, a.B), NF, 0, st>>>(a, blocks);
-    return cudaGetLastError() == cudaSuccess ? 2 : -1;
+    if (launch_kernel(router_stats_final_kernel, dim3(a.Hq, a.B), dim3(NF), 0, st, true, a, blocks) != cudaSuccess)
+        return -1;
+    return 2;
 }
 
 }  // namespace kvs
