@@ -6,7 +6,7 @@
 // second component; Key Concepts, Token-Conditional Depth Routing). The decode
 // kernels keep every valid token's log2-domain scaled score s_{h,t} for the layer;
 // with the layer's lse (exact weight sums) each weight is p_{h,t} = 2^(s - lse/ln 2).
-// Each thread takes TPT tokens of one sequence (all of a pass's head scores loaded at once) and writes
+// Each thread takes one token of one sequence (all of a pass's head scores loaded at once) and writes
 //   mass[j][t]  = sum over the g heads of kv head j of p_{h,t}
 //   score[t]    = x / (1 + x),  x = (T_b * sum_j mass[j][t]) / Hq     (fp32, in this order)
 // Tokens past the sequence get mass 0 and score 0. Per head, each block reduces its
@@ -19,7 +19,6 @@ namespace kvs {
 namespace {
 
 constexpr int NT = 128;
-constexpr int TPT = 1;                        // tokens per thread
 constexpr int HC = 32;                        // heads per pass: all their scores loaded at once
 constexpr float LOG2E_F = 1.4426950408889634f;
 
@@ -43,7 +42,11 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane)
     return v[0];
 }
 
+// G: query heads per kv head when it divides HC (the groups then never straddle a
+// pass and their bookkeeping is static), 0: any g, read at run time.
+template <int G>
 __global__ void __launch_bounds__(NT, 4) router_stats_kernel(const StatsArgs a) {
+    static_assert(G == 0 || HC % G == 0, "groups inside one pass");
     // dependent launch: the decode's scores and lse are read only after it completes;
     // the next kernel may then be scheduled while this one runs
     grid_dep_wait();
@@ -62,55 +65,50 @@ __global__ void __launch_bounds__(NT, 4) router_stats_kernel(const StatsArgs a) 
     static_assert(HC == 32, "one head per lane in the block reduction");
     __shared__ float red_e[NT / 32][HC], red_p[NT / 32][HC];
     __shared__ float lse2_s[HC];
-    float macc[TPT], total[TPT];
-#pragma unroll
-    for (int k = 0; k < TPT; ++k) macc[k] = total[k] = 0.f;
-    const int t0 = blockIdx.x * NT * TPT + threadIdx.x;   // this thread's tokens: t0 + k * NT
-    const float* srow0 = a.sscore + static_cast<size_t>(b) * a.Hq * a.T;
-    int hg = 0, j = 0;                                   // head h = j g + hg, heads in order
+    const int t = blockIdx.x * NT + threadIdx.x;         // this thread's token
+    const bool live = t < n;
+    const float* srow = a.sscore + static_cast<size_t>(b) * a.Hq * a.T + t;
+    float* mrow = a.mass != nullptr ? a.mass + static_cast<size_t>(b) * a.Hkv * a.T + t : nullptr;
+    float macc = 0.f, total = 0.f;
+    int hg = 0, j = 0;                                   // run-time grouping (G == 0): head j g + hg
     for (int h0 = 0; h0 < a.Hq; h0 += HC) {
         const int hn = min(HC, a.Hq - h0);
         if (threadIdx.x < hn) lse2_s[threadIdx.x] = a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] * LOG2E_F;
         __syncthreads();
         // every score of the pass first, all loads in flight together
-        float sv[HC][TPT];
+        float sv[HC];
 #pragma unroll
-        for (int q = 0; q < HC; ++q)
-#pragma unroll
-            for (int k = 0; k < TPT; ++k) {
-                const int t = t0 + k * NT;
-                sv[q][k] = (q < hn && t < n) ? __ldcs(srow0 + static_cast<size_t>(h0 + q) * a.T + t) : 0.f;
-            }
-        // this thread's entropy terms and largest weight per head; reduced over the block
-        // after the pass, so the reductions of different heads overlap
+        for (int q = 0; q < HC; ++q) sv[q] = (q < hn && live) ? __ldcs(srow + static_cast<size_t>(h0 + q) * a.T) : 0.f;
+        // per head: the weight p (this thread's largest weight, one token) and the entropy
+        // term p (lse2 - s); reduced over the block after the pass
         float es[HC], pm[HC];
 #pragma unroll
         for (int q = 0; q < HC; ++q) {
-            es[q] = pm[q] = 0.f;
-            if (q >= hn) continue;
-            const float l2 = lse2_s[q];
-#pragma unroll
-            for (int k = 0; k < TPT; ++k) {
-                const int t = t0 + k * NT;
-                float p = 0.f;
-                if (t < n) {
-                    p = exp2f(sv[q][k] - l2);
-                    es[q] += p * (l2 - sv[q][k]);
-                    pm[q] = fmaxf(pm[q], p);
-                }
-                macc[k] = hg == 0 ? p : macc[k] + p;
+            float p = 0.f, e = 0.f;
+            if (q < hn && live) {
+                const float x = sv[q] - lse2_s[q];
+                p = ex2_approx(x);
+                e = -p * x;
             }
-            if (hg == a.g - 1) {                         // group complete: its mass, then the total
-#pragma unroll
-                for (int k = 0; k < TPT; ++k) {
-                    const int t = t0 + k * NT;
-                    if (a.mass != nullptr && t < a.T) a.mass[(static_cast<size_t>(b) * a.Hkv + j) * a.T + t] = macc[k];
-                    total[k] = j == 0 ? macc[k] : __fadd_rn(total[k], macc[k]);
+            es[q] = e;
+            pm[q] = p;
+            if (G > 0) {
+                macc = q % G == 0 ? p : macc + p;
+                if (q % G == G - 1 && q < hn) {          // group complete: its mass, then the total
+                    const int jj = (h0 + q) / G;
+                    if (mrow != nullptr && t < a.T) mrow[static_cast<size_t>(jj) * a.T] = macc;
+                    total = jj == 0 ? macc : __fadd_rn(total, macc);
                 }
-                hg = 0;
-                ++j;
-            } else {
-                ++hg;
+            } else if (q < hn) {
+                macc = hg == 0 ? p : macc + p;
+                if (hg == a.g - 1) {
+                    if (mrow != nullptr && t < a.T) mrow[static_cast<size_t>(j) * a.T] = macc;
+                    total = j == 0 ? macc : __fadd_rn(total, macc);
+                    hg = 0;
+                    ++j;
+                } else {
+                    ++hg;
+                }
             }
         }
         if (want_red) {
@@ -131,15 +129,10 @@ __global__ void __launch_bounds__(NT, 4) router_stats_kernel(const StatsArgs a) 
         }
         __syncthreads();
     }
-    if (a.score != nullptr) {
-#pragma unroll
-        for (int k = 0; k < TPT; ++k) {
-            const int t = t0 + k * NT;
-            if (t >= a.T) continue;
-            float x = __fmul_rn(static_cast<float>(n), total[k]);
-            x = __fdiv_rn(x, static_cast<float>(a.Hq));
-            a.score[static_cast<size_t>(b) * a.T + t] = __fdiv_rn(x, __fadd_rn(1.f, x));
-        }
+    if (a.score != nullptr && t < a.T) {
+        float x = __fmul_rn(static_cast<float>(n), total);
+        x = __fdiv_rn(x, static_cast<float>(a.Hq));
+        a.score[static_cast<size_t>(b) * a.T + t] = __fdiv_rn(x, __fadd_rn(1.f, x));
     }
 }
 
@@ -180,13 +173,15 @@ __global__ void __launch_bounds__(NF) router_stats_final_kernel(const StatsArgs 
 
 }  // namespace
 
-int router_stats_blocks(int T) { return (T + NT * TPT - 1) / (NT * TPT); }
+int router_stats_blocks(int T) { return (T + NT - 1) / NT; }
 
 int launch_router_stats(const StatsArgs& a, cudaStream_t st) {
     const int blocks = router_stats_blocks(a.T);
     // both launches are dependent launches: their start overlaps the tail of the kernel
     // ahead, and they wait for it before touching memory
-    if (launch_kernel(router_stats_kernel, dim3(blocks, a.B), dim3(NT), 0, st, true, a) != cudaSuccess) return -1;
+    auto kern = a.g == 4 ? router_stats_kernel<4> : a.g == 8 ? router_stats_kernel<8>
+              : a.g == 2 ? router_stats_kernel<2> : a.g == 16 ? router_stats_kernel<16> : router_stats_kernel<0>;
+    if (launch_kernel(kern, dim3(blocks, a.B), dim3(NT), 0, st, true, a) != cudaSuccess) return -1;
     if (a.entropy == nullptr && a.peak == nullptr) return 1;
     if (launch_kernel(router_stats_final_kernel, dim3(a.Hq, a.B), dim3(NF), 0, st, true, a, blocks) != cudaSuccess)
         return -1;
