@@ -661,7 +661,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--only", choices=["prefill"], default=None,
-                    help="profiling aid: run only the causal prefill workload and print its numbers")
+                    help="profiling aid: run only a causal prefill workload (the two-source one, or the "
+                         "prefill workload --config names) and print its numbers")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling aid: keep only the first N layers of the --config decode workload "
+                         "(its layer pattern, fewer layers: a smaller case of the same kernels)")
     ap.add_argument("--batch", type=int, default=0,
                     help="profiling aid: batch of the prefill workload (with --only prefill) or of the "
                          "--config decode workload (a smaller case of the same kernels)")
@@ -671,10 +675,12 @@ def main():
     if args.only == "prefill":
         import torch
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        name = "depthgraft_prefill"
+        # the two-source prefill unless --config names another prefill workload
+        base = args.config if BY_NAME[args.config].mode == "prefill" else "depthgraft_prefill"
+        name = base
         if args.batch > 0:
-            name = f"depthgraft_prefill_b{args.batch}"
-            BY_NAME[name] = BY_NAME["depthgraft_prefill"].replace(name=name, batch=args.batch)
+            name = f"{base}_b{args.batch}"
+            BY_NAME[name] = BY_NAME[base].replace(name=name, batch=args.batch)
         pr = prefill_arm(args, name)
         print(json.dumps({"workload": name, "tflops": pr["tflops"], "ms_per_step": pr["step_ms"],
                           "single_source_layer_tflops": pr["single_layer_tflops"],
@@ -699,6 +705,15 @@ def main():
     if args.batch > 0:
         name = f"{args.config}_b{args.batch}"
         BY_NAME[name] = BY_NAME[args.config].replace(name=name, batch=args.batch)
+        args.config = name
+    if args.layers > 0:
+        c = BY_NAME[args.config]
+        n_l = min(args.layers, c.layers)
+        name = f"{args.config}_l{n_l}"
+        kw = dict(name=name, layers=n_l, layer_map=c.layer_map[:n_l])
+        if c.lowrank:
+            kw["pairs"] = (n_l + 1) // 2
+        BY_NAME[name] = c.replace(**kw)
         args.config = name
     main_res = gpu_arm(args, args.config)
     cfg = main_res["cfg"]

@@ -99,8 +99,6 @@ struct kvshare_ctx {
     float* sscore = nullptr;
     // projected queries of one low-rank prefill layer [max_batch][Hq][max_context][64] bf16
     uint16_t* qp = nullptr;
-    // statistics kernel: per-block entropy/peak partials
-    float* stats_part = nullptr;
     // staging for kvshare_decode_host
     void* q_stage = nullptr;
     float* out_stage = nullptr;
@@ -253,7 +251,13 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
         a.T = T;
         a.g = g;
         a.lens = k->lengths;
-        a.sscore = stats != nullptr ? c->sscore : nullptr;
+        // the kept scores feed the per-token statistics (mass, router score); entropy and
+        // peak come out of the decode's own merge
+        const bool per_token = stats != nullptr && (stats->mass != nullptr || stats->score != nullptr);
+        a.sscore = per_token ? c->sscore : nullptr;
+        const size_t lbh = static_cast<size_t>(l) * B * Hq;
+        a.entropy = stats != nullptr && stats->entropy != nullptr ? stats->entropy + lbh : nullptr;
+        a.peak = stats != nullptr && stats->peak != nullptr ? stats->peak + lbh : nullptr;
         a.scale_log2 = c->scale * 1.4426950408889634f;
         a.ws = c->ws;
         a.counters = c->counters;
@@ -271,6 +275,7 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
             const int tt = decode_f32_tile();
             const int tiles = (T + tt - 1) / tt;
             int s = choose_splits(c, B * Hkv, tiles, 4, g, D);
+            if (s > F32_MAX_SPLITS) s = F32_MAX_SPLITS;
             a.tiles_per_split = (tiles + s - 1) / s;
             a.splits = (tiles + a.tiles_per_split - 1) / a.tiles_per_split;
             err = launch_decode_f32(e.kind == KVS_SRC_MIX, D, a, st);
@@ -354,7 +359,7 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
         }
         if (err != cudaSuccess) return KVS_ECUDA;
         ++c->launches;
-        if (stats != nullptr) {
+        if (per_token) {
             StatsArgs sa;
             std::memset(&sa, 0, sizeof(sa));
             sa.sscore = c->sscore;
@@ -363,9 +368,6 @@ kvshare_status decode_layers(kvshare_ctx* c, const kvshare_cache* k, const void*
             const size_t lbt = static_cast<size_t>(l) * B;
             sa.mass = stats->mass ? stats->mass + lbt * Hkv * T : nullptr;
             sa.score = stats->score ? stats->score + lbt * T : nullptr;
-            sa.entropy = stats->entropy ? stats->entropy + lbt * Hq : nullptr;
-            sa.peak = stats->peak ? stats->peak + lbt * Hq : nullptr;
-            sa.part = c->stats_part;
             sa.err = c->err;
             sa.B = B;
             sa.Hq = Hq;
@@ -541,7 +543,6 @@ kvshare_status kvshare_destroy(kvshare_t ctx) {
     cudaFree(ctx->w_dev);
     cudaFree(ctx->sscore);
     cudaFree(ctx->qp);
-    cudaFree(ctx->stats_part);
     cudaFree(ctx->q_stage);
     cudaFree(ctx->out_stage);
     cudaFree(ctx->lse_stage);
@@ -619,17 +620,12 @@ kvshare_status kvshare_decode_stats(kvshare_t ctx, const kvshare_cache* cache, c
         return decode_layers(ctx, cache, q, out, lse, ls.data(), static_cast<int>(ls.size()),
                              static_cast<cudaStream_t>(stream));
     if (cudaSetDevice(ctx->device) != cudaSuccess) return KVS_ECUDA;
-    if (ctx->sscore == nullptr) {
+    if (ctx->sscore == nullptr && (mass != nullptr || score != nullptr)) {
         const kvshare_config& cf = ctx->cfg;
         const size_t n = static_cast<size_t>(cf.max_batch) * cf.num_q_heads * cf.max_context;
-        const size_t np = static_cast<size_t>(cf.max_batch) * router_stats_blocks(cf.max_context) * cf.num_q_heads * 2;
-        if (cudaMalloc(&ctx->sscore, n * sizeof(float)) != cudaSuccess ||
-            cudaMalloc(&ctx->stats_part, np * sizeof(float)) != cudaSuccess) {
+        if (cudaMalloc(&ctx->sscore, n * sizeof(float)) != cudaSuccess) {
             cudaGetLastError();
-            cudaFree(ctx->sscore);
-            cudaFree(ctx->stats_part);
             ctx->sscore = nullptr;
-            ctx->stats_part = nullptr;
             return KVS_ENOMEM;
         }
     }

@@ -32,18 +32,20 @@ struct DecodeCfg {
     static constexpr int NSRC = MIX ? 2 : 1;
     static constexpr int STAGE_BYTES = 2 * NSRC * TILE_BYTES;
     static constexpr int RING_BYTES = NW * NSW * STAGE_BYTES;
-    static constexpr int COMBINE_FLOATS = NW * 16 * D + 3 * NW * 16 + 48 + 16 * D + 3 * MAX_GROUP * MAX_SPLITS + 64;
+    static constexpr int COMBINE_FLOATS = NW * 16 * D + 4 * NW * 16 + 64 + 16 * D + 4 * MAX_GROUP * MAX_SPLITS + 64;
     static constexpr int MERGE_STAGE_OFF = ((COMBINE_FLOATS * 4 + 1023) / 1024) * 1024;   // free smem for the merge
     static constexpr int BODY = RING_BYTES > COMBINE_FLOATS * 4 ? RING_BYTES : COMBINE_FLOATS * 4;
     // per-warp state of the first unit when a warp's tiles cross into the second one
-    static constexpr int SAVE_FLOATS = NW * (16 * D + 48);
+    static constexpr int SAVE_FLOATS = NW * (16 * D + 64);
     static constexpr int SMEM = BODY + SAVE_FLOATS * 4 + 1024;  // + slack to align the ring to 1024 B
     static constexpr int SMEM_ALIGNED = BODY + 1024;             // grids whose ranges never straddle
     static_assert(TT % 16 == 0, "token tile must hold whole m16 tiles");
     static_assert(HALF_BYTES % 1024 == 0, "swizzled halves must stay 1024-B aligned");
 };
 
-template <int D, bool MIX, int TT, int NSW, int NW, int NH, bool STRADDLE>
+// ENT: the launch asks for the entropy; only then does the softmax carry z (a separate
+// instantiation, so the plain decode loop carries nothing for it)
+template <int D, bool MIX, int TT, int NSW, int NW, int NH, bool STRADDLE, bool ENT>
 __global__ void __launch_bounds__(NW * 32, 1)
 decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const DecodeArgs a) {
@@ -52,7 +54,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     constexpr int NB = NH / 8;       // n8 head blocks
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    float* save = reinterpret_cast<float*>(smem + C::BODY);    // [NW][16][D] O, then [NW][48]: m, l, lx
+    float* save = reinterpret_cast<float*>(smem + C::BODY);    // [NW][16][D] O, then [NW][64]: m, l, lx, z
     __shared__ __align__(8) uint64_t bars[NW * NSW + 1];
     __shared__ int fin_unit[NW], sav_unit[NW];
 
@@ -161,6 +163,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     float o[D / 16][NB][4];          // O^T: rows = channels, columns = heads nb*8 + 2(lane%4) (+1)
     float mrow[NB][2], lrow[NB][2];  // softmax statistics of those two heads
     float lxrow[NB][2];              // sums of the unrounded weights (for the lse)
+    float zrow[NB][2];               // sums of 2^(s - m) (m - s) (for the entropy, when asked for)
+    constexpr bool want_z = ENT;
     float w = 1.f, w1 = 0.f;
     int tlen = a.T;                  // tokens of the current unit's sequence
     float* srow = nullptr;           // the current unit's kept scores [g][T], if requested
@@ -181,6 +185,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             mrow[nb][0] = mrow[nb][1] = NEG_INF;
             lrow[nb][0] = lrow[nb][1] = 0.f;
             lxrow[nb][0] = lxrow[nb][1] = 0.f;
+            zrow[nb][0] = zrow[nb][1] = 0.f;
 #pragma unroll
             for (int i = 0; i < D / 16; ++i) o[i][nb][0] = o[i][nb][1] = o[i][nb][2] = o[i][nb][3] = 0.f;
         }
@@ -190,8 +195,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         srow = a.sscore != nullptr ? a.sscore + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * g) * a.T
                                    : nullptr;
     };
-    // write this warp's statistics and O^T for heads < g: O to dst_o [16][D], m, l, lx to
-    // dst_ml [48]
+    // write this warp's statistics and O^T for heads < g: O to dst_o [16][D], m, l, lx, z
+    // to dst_ml [64]
     auto store_state = [&](float* dst_o, float* dst_ml) {
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
@@ -201,6 +206,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                 lrow[nb][1] += __shfl_xor_sync(0xffffffffu, lrow[nb][1], off);
                 lxrow[nb][0] += __shfl_xor_sync(0xffffffffu, lxrow[nb][0], off);
                 lxrow[nb][1] += __shfl_xor_sync(0xffffffffu, lxrow[nb][1], off);
+                zrow[nb][0] += __shfl_xor_sync(0xffffffffu, zrow[nb][0], off);
+                zrow[nb][1] += __shfl_xor_sync(0xffffffffu, zrow[nb][1], off);
             }
         const int e0 = lane >> 2;
 #pragma unroll
@@ -224,6 +231,8 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
                 dst_ml[16 + h0 + 1] = lrow[nb][1];
                 dst_ml[32 + h0] = lxrow[nb][0];
                 dst_ml[32 + h0 + 1] = lxrow[nb][1];
+                dst_ml[48 + h0] = zrow[nb][0];
+                dst_ml[48 + h0 + 1] = zrow[nb][1];
             }
         }
     };
@@ -241,7 +250,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     for (int k = 0; k < my_n; ++k, advance(u, t)) {
         if (STRADDLE && u != cur_u) {
             if (cur_u >= 0) {
-                store_state(save + warp * 16 * D, save + NW * 16 * D + warp * 48);
+                store_state(save + warp * 16 * D, save + NW * 16 * D + warp * 64);
                 saved_u = cur_u;
             }
             begin_unit(u);
@@ -353,6 +362,11 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
             const float cr0 = ex2_approx(mrow[nb][0] - ref0);
             const float cr1 = ex2_approx(mrow[nb][1] - ref1);
+            if (want_z) {
+                // z moves to the new reference with the unscaled lx (see kvs_device.cuh)
+                zrow[nb][0] = cr0 * fmaf(lxrow[nb][0], mrow[nb][0] == NEG_INF ? 0.f : ref0 - mrow[nb][0], zrow[nb][0]);
+                zrow[nb][1] = cr1 * fmaf(lxrow[nb][1], mrow[nb][1] == NEG_INF ? 0.f : ref1 - mrow[nb][1], zrow[nb][1]);
+            }
             mrow[nb][0] = mn0;
             mrow[nb][1] = mn1;
             lrow[nb][0] *= cr0;
@@ -366,12 +380,21 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const float p0 = ex2_approx(fmaf(sc[mt][nb][0], a.scale_log2, -ref0));
-                const float p1 = ex2_approx(fmaf(sc[mt][nb][1], a.scale_log2, -ref1));
-                const float p2 = ex2_approx(fmaf(sc[mt][nb][2], a.scale_log2, -ref0));
-                const float p3 = ex2_approx(fmaf(sc[mt][nb][3], a.scale_log2, -ref1));
+                const float x0 = fmaf(sc[mt][nb][0], a.scale_log2, -ref0);
+                const float x1 = fmaf(sc[mt][nb][1], a.scale_log2, -ref1);
+                const float x2 = fmaf(sc[mt][nb][2], a.scale_log2, -ref0);
+                const float x3 = fmaf(sc[mt][nb][3], a.scale_log2, -ref1);
+                const float p0 = ex2_approx(x0);
+                const float p1 = ex2_approx(x1);
+                const float p2 = ex2_approx(x2);
+                const float p3 = ex2_approx(x3);
                 lxrow[nb][0] += p0 + p2;
                 lxrow[nb][1] += p1 + p3;
+                if (want_z) {
+                    // p (ref - s); a masked token (x = -inf, p = 0) adds 0
+                    zrow[nb][0] = fmaf(p0, -fmaxf(x0, -3.0e38f), fmaf(p2, -fmaxf(x2, -3.0e38f), zrow[nb][0]));
+                    zrow[nb][1] = fmaf(p1, -fmaxf(x1, -3.0e38f), fmaf(p3, -fmaxf(x3, -3.0e38f), zrow[nb][1]));
+                }
                 if (!MIX) {
                     const uint32_t lo = pack_bf16(p0, p1), hi = pack_bf16(p2, p3);
                     lrow[nb][0] += bf16_lo(lo) + bf16_lo(hi);
@@ -421,13 +444,14 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     __syncthreads();
     (void)t;
     float* comb_o = reinterpret_cast<float*>(smem);   // [NW][16][D]
-    float* comb_ml = comb_o + NW * 16 * D;            // [NW][48]: m[16], l[16], lx[16]
-    float* fin_m = comb_ml + NW * 48;                 // [16]
+    float* comb_ml = comb_o + NW * 16 * D;            // [NW][64]: m[16], l[16], lx[16], z[16]
+    float* fin_m = comb_ml + NW * 64;                 // [16]
     float* fin_l = fin_m + 16;                        // [16]
     float* fin_lx = fin_l + 16;                       // [16]
-    float* fin_o = fin_lx + 16;                       // [16][D]
+    float* fin_z = fin_lx + 16;                       // [16]
+    float* fin_o = fin_z + 16;                        // [16][D]
     float* scratch = fin_o + 16 * D;                  // merge scratch
-    if (cur_u >= 0) store_state(comb_o + warp * 16 * D, comb_ml + warp * 48);
+    if (cur_u >= 0) store_state(comb_o + warp * 16 * D, comb_ml + warp * 64);
     if (lane == 0) {
         fin_unit[warp] = cur_u;
         sav_unit[warp] = saved_u;
@@ -445,31 +469,35 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             const int h = threadIdx.x;
             float M = NEG_INF;
             for (int ww = 0; ww < NW; ++ww) {
-                if (fin_unit[ww] == u) M = fmaxf(M, comb_ml[ww * 48 + h]);
-                if (STRADDLE && sav_unit[ww] == u) M = fmaxf(M, save_ml[ww * 48 + h]);
+                if (fin_unit[ww] == u) M = fmaxf(M, comb_ml[ww * 64 + h]);
+                if (STRADDLE && sav_unit[ww] == u) M = fmaxf(M, save_ml[ww * 64 + h]);
             }
             // a warp without a state for u left its slots as they were (ring data, or an
             // earlier kernel's shared memory, NaN included): never read them, not even as 0 * x
-            float L = 0.f, LX = 0.f;
+            float L = 0.f, LX = 0.f, Z = 0.f;
             for (int ww = 0; ww < NW; ++ww) {
                 float ff = 0.f;
                 if (fin_unit[ww] == u) {
-                    const float mf = comb_ml[ww * 48 + h];
+                    const float* st = comb_ml + ww * 64;
+                    const float mf = st[h];
                     if (mf != NEG_INF) {
                         ff = ex2_approx(mf - M);
-                        L = fmaf(ff, comb_ml[ww * 48 + 16 + h], L);
-                        LX = fmaf(ff, comb_ml[ww * 48 + 32 + h], LX);
+                        L = fmaf(ff, st[16 + h], L);
+                        LX = fmaf(ff, st[32 + h], LX);
+                        Z += merged_z(ff, mf, M, st[32 + h], st[48 + h]);
                     }
                 }
                 fac_f[ww][h] = ff;
                 if (STRADDLE) {
                     float fs = 0.f;
                     if (sav_unit[ww] == u) {
-                        const float ms = save_ml[ww * 48 + h];
+                        const float* st = save_ml + ww * 64;
+                        const float ms = st[h];
                         if (ms != NEG_INF) {
                             fs = ex2_approx(ms - M);
-                            L = fmaf(fs, save_ml[ww * 48 + 16 + h], L);
-                            LX = fmaf(fs, save_ml[ww * 48 + 32 + h], LX);
+                            L = fmaf(fs, st[16 + h], L);
+                            LX = fmaf(fs, st[32 + h], LX);
+                            Z += merged_z(fs, ms, M, st[32 + h], st[48 + h]);
                         }
                     }
                     fac_s[ww][h] = fs;
@@ -478,6 +506,7 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
             fin_m[h] = M;
             fin_l[h] = L;
             fin_lx[h] = LX;
+            fin_z[h] = Z;
         }
         __syncthreads();
         for (int idx = threadIdx.x; idx < g * D; idx += blockDim.x) {
@@ -502,16 +531,16 @@ decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         const int c_last = static_cast<int>(((static_cast<long long>(u + 1) * a.n_t - 1) * G) / W);
         const EmitPlain emit{a, D, static_cast<size_t>(u / a.Hkv) * a.Hq + static_cast<size_t>(u % a.Hkv) * g};
         finish_unit(a, D, u, cta - c_first, c_last - c_first + 1, static_cast<long long>(u) + c_first, fin_m, fin_l,
-                    fin_lx, fin_o, scratch, smem + C::MERGE_STAGE_OFF,
+                    fin_lx, fin_z, fin_o, scratch, smem + C::MERGE_STAGE_OFF,
                     C::BODY > C::MERGE_STAGE_OFF ? C::BODY - C::MERGE_STAGE_OFF : 0, emit);
         __syncthreads();
     }
 }
 
-template <int D, bool MIX, int TT, int NSW, int NW, int NH, bool STRADDLE>
-cudaError_t launch_nh(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a, cudaStream_t st) {
+template <int D, bool MIX, int TT, int NSW, int NW, int NH, bool STRADDLE, bool ENT>
+cudaError_t launch_ent(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a, cudaStream_t st) {
     using C = DecodeCfg<D, MIX, TT, NSW, NW>;
-    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, NW, NH, STRADDLE>;
+    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, NW, NH, STRADDLE, ENT>;
     constexpr int smem = STRADDLE ? C::SMEM : C::SMEM_ALIGNED;
     static std::atomic<unsigned long long> attr_done{0};
     cudaError_t e = once_per_device(attr_done, [&] {
@@ -519,6 +548,12 @@ cudaError_t launch_nh(const CUtensorMap& tmK, const CUtensorMap& tmV, const Deco
     });
     if (e != cudaSuccess) return e;
     return launch_kernel(kern, dim3(a.splits), dim3(NW * 32), smem, st, a.pdl != 0, tmK, tmV, a);
+}
+
+template <int D, bool MIX, int TT, int NSW, int NW, int NH, bool STRADDLE>
+cudaError_t launch_nh(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a, cudaStream_t st) {
+    return a.entropy != nullptr ? launch_ent<D, MIX, TT, NSW, NW, NH, STRADDLE, true>(tmK, tmV, a, st)
+                                : launch_ent<D, MIX, TT, NSW, NW, NH, STRADDLE, false>(tmK, tmV, a, st);
 }
 
 template <int D, bool MIX, int TT, int NSW, int NW>
@@ -537,7 +572,7 @@ template <int D, bool MIX, int TT, int NSW, int NW>
 int occupancy() {
     using C = DecodeCfg<D, MIX, TT, NSW, NW>;
     // the default grid is unit-aligned, so its CTAs carry no straddle save area
-    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, NW, 8, false>;
+    auto kern = decode_bf16_kernel<D, MIX, TT, NSW, NW, 8, false, false>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALIGNED);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NW * 32, C::SMEM_ALIGNED) != cudaSuccess) return 1;

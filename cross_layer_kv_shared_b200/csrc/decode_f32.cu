@@ -19,12 +19,12 @@ template <int D, bool MIX>
 __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
     // the query rows and a chunk's scores during the stream; the split merge's scratch after it
     constexpr int STREAM_FLOATS = MAX_GROUP * D + MAX_GROUP * CH;
-    constexpr int MERGE_FLOATS = 3 * MAX_GROUP * MAX_SPLITS;
+    constexpr int MERGE_FLOATS = 4 * MAX_GROUP * F32_MAX_SPLITS;
     __shared__ float pool[STREAM_FLOATS > MERGE_FLOATS ? STREAM_FLOATS : MERGE_FLOATS];
     float (*sq)[D] = reinterpret_cast<float (*)[D]>(pool);
     float (*ss)[CH] = reinterpret_cast<float (*)[CH]>(pool + MAX_GROUP * D);
     float* scratch = pool;
-    __shared__ float sm_m[MAX_GROUP], sm_l[MAX_GROUP], scorr[MAX_GROUP];
+    __shared__ float sm_m[MAX_GROUP], sm_l[MAX_GROUP], sm_z[MAX_GROUP], scorr[MAX_GROUP];
     __shared__ float fin_o[MAX_GROUP * D];
     __shared__ __align__(8) uint64_t never_bar;
 
@@ -57,7 +57,9 @@ __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
     if (tid < g) {
         sm_m[tid] = NEG_INF;
         sm_l[tid] = 0.f;
+        sm_z[tid] = 0.f;
     }
+    const bool want_z = a.entropy != nullptr;   // sum of 2^(s - m) (m - s), for the entropy
     float acc[OPT];
 #pragma unroll
     for (int i = 0; i < OPT; ++i) acc[i] = 0.f;
@@ -96,12 +98,15 @@ __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
             for (int tt = 0; tt < n; ++tt) mx = fmaxf(mx, ss[h][tt]);
             const float mn = fmaxf(sm_m[h], mx);
             const float corr = exp2f(sm_m[h] - mn);
-            float sum = 0.f;
+            float sum = 0.f, zs = 0.f;
             for (int tt = 0; tt < n; ++tt) {
-                const float p = exp2f(ss[h][tt] - mn);
+                const float sv = ss[h][tt];
+                const float p = exp2f(sv - mn);
                 ss[h][tt] = p;
                 sum += p;
+                if (want_z) zs = fmaf(p, mn - sv, zs);
             }
+            if (want_z) sm_z[h] = fmaf(corr, sm_m[h] != NEG_INF ? fmaf(sm_l[h], mn - sm_m[h], sm_z[h]) : 0.f, zs);
             sm_l[h] = sm_l[h] * corr + sum;
             sm_m[h] = mn;
             scorr[h] = corr;
@@ -131,7 +136,7 @@ __global__ void __launch_bounds__(NT) decode_f32_kernel(const DecodeArgs a) {
     }
     __syncthreads();
     // the weights are fp32 throughout: the P.V sum and the exact sum are the same
-    finish_split(a, D, b, j, split, sm_m, sm_l, sm_l, fin_o, scratch, nullptr, 0);
+    finish_split(a, D, b, j, split, sm_m, sm_l, sm_l, sm_z, fin_o, scratch, nullptr, 0);
 }
 
 template <int D, bool MIX>

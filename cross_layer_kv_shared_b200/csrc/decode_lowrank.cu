@@ -64,7 +64,7 @@ struct LrCfg {
     // [K | V][TT][16] halves, rows of 32 B whose two 16-B halves swap on every 4th row
     static constexpr int CVT_BYTES = NW * 2 * TT * 32;
     static constexpr int PD = RB + RM;    // coefficient-space partial width
-    static constexpr int COMBINE_FLOATS = NW * 16 * PD + 3 * NW * 16 + 48 + 16 * PD + 16 * D + 3 * MAX_GROUP * MAX_SPLITS + 64;
+    static constexpr int COMBINE_FLOATS = NW * 16 * PD + 4 * NW * 16 + 64 + 16 * PD + 16 * D + 4 * MAX_GROUP * MAX_SPLITS + 64;
     static constexpr int QPROJ_FLOATS = 16 * PD;
     // staging: B_K [RB][D] + R_K [RM][D] (bf16), the query rows [<=16][D], then B_V + R_V
     static constexpr int STAGE_FACTORS = (RB + RM) * D * 2;
@@ -84,7 +84,7 @@ struct EmitProject {
     size_t head0;
     const uint16_t* Bv;     // [RB][D] bf16 in shared memory
     const uint16_t* Rv;     // [16][D] bf16 in shared memory
-    __device__ void operator()(const float* v, const float* l, const float* lx, const float* m) const {
+    __device__ void operator()(const float* v, const float* l, const float* lx, const float* m, const float* z) const {
         constexpr int PDV = RB + RM;
         for (int idx = threadIdx.x; idx < a.g * D; idx += blockDim.x) {
             const int h = idx / D;
@@ -97,6 +97,7 @@ struct EmitProject {
             a.out[(head0 + h) * D + e] = l[h] > 0.f ? acc / l[h] : 0.f;
         }
         if (a.lse != nullptr && threadIdx.x < a.g) a.lse[head0 + threadIdx.x] = lse_of(m[threadIdx.x], lx[threadIdx.x]);
+        emit_entropy_peak(a, head0, lx, z);
     }
 };
 
@@ -107,7 +108,9 @@ __device__ __forceinline__ uint32_t i8pair_bf16(uint32_t w16, bool keep0, bool k
     return pack_bf16(static_cast<float>(x0), static_cast<float>(x1));
 }
 
-template <int D, int RB, int TT, int NSW, int NW, int NH>
+// ENT: the launch asks for the entropy; only then does the softmax carry z (a separate
+// instantiation, so the plain decode loop carries nothing for it)
+template <int D, int RB, int TT, int NSW, int NW, int NH, bool ENT>
 __global__ void __launch_bounds__(NW * 32, 1)
 decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_constant__ CUtensorMap tmCV,
                       const DecodeArgs a) {
@@ -352,10 +355,13 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         ou[nb][0] = ou[nb][1] = ou[nb][2] = ou[nb][3] = 0.f;
     }
     float mrow[NB][2], lrow[NB][2], lxrow[NB][2];
+    float zrow[NB][2];                    // sums of 2^(s - m) (m - s), for the entropy when asked for
+    constexpr bool want_z = ENT;
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
         mrow[nb][0] = mrow[nb][1] = NEG_INF;
         lrow[nb][0] = lrow[nb][1] = lxrow[nb][0] = lxrow[nb][1] = 0.f;
+        zrow[nb][0] = zrow[nb][1] = 0.f;
     }
 
     float* tks = tok + warp * TT * 3;     // [3][TT]: s_K, s_V, rank
@@ -536,6 +542,11 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
             const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
             const float cr0 = ex2_approx(mrow[nb][0] - ref0), cr1 = ex2_approx(mrow[nb][1] - ref1);
+            if (want_z) {
+                // z moves to the new reference with the unscaled lx (see kvs_device.cuh)
+                zrow[nb][0] = cr0 * fmaf(lxrow[nb][0], mrow[nb][0] == NEG_INF ? 0.f : ref0 - mrow[nb][0], zrow[nb][0]);
+                zrow[nb][1] = cr1 * fmaf(lxrow[nb][1], mrow[nb][1] == NEG_INF ? 0.f : ref1 - mrow[nb][1], zrow[nb][1]);
+            }
             mrow[nb][0] = mn0;
             mrow[nb][1] = mn1;
             lrow[nb][0] *= cr0;
@@ -548,15 +559,24 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const int ta = mt * 16 + (lane >> 2);
-                const float p0 = ex2_approx(fmaf(sc[mt][nb][0], a.scale_log2, -ref0));
-                const float p1 = ex2_approx(fmaf(sc[mt][nb][1], a.scale_log2, -ref1));
-                const float p2 = ex2_approx(fmaf(sc[mt][nb][2], a.scale_log2, -ref0));
-                const float p3 = ex2_approx(fmaf(sc[mt][nb][3], a.scale_log2, -ref1));
+                const float x0 = fmaf(sc[mt][nb][0], a.scale_log2, -ref0);
+                const float x1 = fmaf(sc[mt][nb][1], a.scale_log2, -ref1);
+                const float x2 = fmaf(sc[mt][nb][2], a.scale_log2, -ref0);
+                const float x3 = fmaf(sc[mt][nb][3], a.scale_log2, -ref1);
+                const float p0 = ex2_approx(x0);
+                const float p1 = ex2_approx(x1);
+                const float p2 = ex2_approx(x2);
+                const float p3 = ex2_approx(x3);
                 const uint32_t lo = pack_bf16(p0, p1), hi = pack_bf16(p2, p3);
                 lrow[nb][0] += bf16_lo(lo) + bf16_lo(hi);
                 lrow[nb][1] += bf16_hi(lo) + bf16_hi(hi);
                 lxrow[nb][0] += p0 + p2;
                 lxrow[nb][1] += p1 + p3;
+                if (want_z) {
+                    // p (ref - s); a masked token (x = -inf, p = 0) adds 0
+                    zrow[nb][0] = fmaf(p0, -fmaxf(x0, -3.0e38f), fmaf(p2, -fmaxf(x2, -3.0e38f), zrow[nb][0]));
+                    zrow[nb][1] = fmaf(p1, -fmaxf(x1, -3.0e38f), fmaf(p3, -fmaxf(x3, -3.0e38f), zrow[nb][1]));
+                }
                 pb[mt][nb][0] = movmatrix_t(lo);
                 pb[mt][nb][1] = movmatrix_t(hi);
                 const float sva = tks[TT + ta], svb = tks[TT + ta + 8];
@@ -603,6 +623,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
             lrow[nb][1] += __shfl_xor_sync(0xffffffffu, lrow[nb][1], off);
             lxrow[nb][0] += __shfl_xor_sync(0xffffffffu, lxrow[nb][0], off);
             lxrow[nb][1] += __shfl_xor_sync(0xffffffffu, lxrow[nb][1], off);
+            zrow[nb][0] += __shfl_xor_sync(0xffffffffu, zrow[nb][0], off);
+            zrow[nb][1] += __shfl_xor_sync(0xffffffffu, zrow[nb][1], off);
         }
 
     // ---- merge warps in coefficient space, project once, finish the split
@@ -615,10 +637,12 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     float* comb_m = comb + NW * 16 * PD;
     float* comb_l = comb_m + NW * 16;
     float* comb_lx = comb_l + NW * 16;
-    float* fin_m = comb_lx + NW * 16;
+    float* comb_z = comb_lx + NW * 16;
+    float* fin_m = comb_z + NW * 16;
     float* fin_l = fin_m + 16;
     float* fin_lx = fin_l + 16;
-    float* fin_c = fin_lx + 16;                     // [16][PD]
+    float* fin_z = fin_lx + 16;
+    float* fin_c = fin_z + 16;                      // [16][PD]
     float* fin_o = fin_c + 16 * PD;                 // [16][D]
     float* scratch = fin_o + 16 * D;
     {
@@ -644,6 +668,8 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
                 comb_l[warp * 16 + h0 + 1] = lrow[nb][1];
                 comb_lx[warp * 16 + h0] = lxrow[nb][0];
                 comb_lx[warp * 16 + h0 + 1] = lxrow[nb][1];
+                comb_z[warp * 16 + h0] = zrow[nb][0];
+                comb_z[warp * 16 + h0 + 1] = zrow[nb][1];
             }
         }
     }
@@ -654,17 +680,19 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
         const int h = threadIdx.x;
         float M = NEG_INF;
         for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, comb_m[ww * 16 + h]);
-        float L = 0.f, LX = 0.f;
+        float L = 0.f, LX = 0.f, Z = 0.f;
         for (int ww = 0; ww < NW; ++ww) {
             const float m = comb_m[ww * 16 + h];
-            const float f = m != NEG_INF ? ex2_approx(m - M) : 0.f;
+            const float f = merge_factor(m, M);
             fac[ww][h] = f;
             L += f * comb_l[ww * 16 + h];
             LX += f * comb_lx[ww * 16 + h];
+            Z += merged_z(f, m, M, comb_lx[ww * 16 + h], comb_z[ww * 16 + h]);
         }
         fin_m[h] = M;
         fin_l[h] = L;
         fin_lx[h] = LX;
+        fin_z[h] = Z;
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < g * PD; idx += blockDim.x) {
@@ -685,14 +713,14 @@ decode_lowrank_kernel(const __grid_constant__ CUtensorMap tmCK, const __grid_con
     const int unit = b * a.Hkv + j;
     // the per-token and code-conversion buffers are free now: they stage the unit's partials
     finish_unit<(PD > D ? PD : D)>(a, PD, unit, split, a.splits, static_cast<long long>(unit) * a.splits, fin_m, fin_l,
-                                   fin_lx, fin_c, scratch,
+                                   fin_lx, fin_z, fin_c, scratch,
                 reinterpret_cast<uint8_t*>(tok), C::TOK_BYTES + C::CVT_BYTES, emit);
 }
 
-template <int D, int RB, int TT, int NSW, int NW, int NH>
-cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
+template <int D, int RB, int TT, int NSW, int NW, int NH, bool ENT>
+cudaError_t launch_ent(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
     using C = LrCfg<D, RB, TT, NSW, NW>;
-    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, NH>;
+    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, NH, ENT>;
     static std::atomic<unsigned long long> attr_done{0};
     cudaError_t e = once_per_device(attr_done, [&] {
         return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -700,6 +728,12 @@ cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t
     if (e != cudaSuccess) return e;
     dim3 grid(a.splits, a.Hkv, a.B);
     return launch_kernel(kern, grid, dim3(NW * 32), C::SMEM, st, a.pdl != 0, maps[0], maps[1], a);
+}
+
+template <int D, int RB, int TT, int NSW, int NW, int NH>
+cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_t st) {
+    return a.entropy != nullptr ? launch_ent<D, RB, TT, NSW, NW, NH, true>(a, maps, st)
+                                : launch_ent<D, RB, TT, NSW, NW, NH, false>(a, maps, st);
 }
 
 template <int D, int RB, int TT, int NSW, int NW>
@@ -710,7 +744,7 @@ cudaError_t launch_one(const DecodeArgs& a, const CUtensorMap* maps, cudaStream_
 template <int D, int RB, int TT, int NSW, int NW>
 int occupancy_of() {
     using C = LrCfg<D, RB, TT, NSW, NW>;
-    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, 8>;
+    auto kern = decode_lowrank_kernel<D, RB, TT, NSW, NW, 8, false>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, NW * 32, C::SMEM) != cudaSuccess) return 1;

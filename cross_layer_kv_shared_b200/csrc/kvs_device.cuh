@@ -240,10 +240,18 @@ __device__ __forceinline__ void zero_tile_rows(uint8_t* base, int row_bytes, int
 }
 
 // ------------------------------------------------------------------ split merge
-// Partial layout: [unit][split][head][D + 4] floats: o[0..D), m, l, lx, one pad word
-// (rows stay 16-byte aligned so whole partial blocks can move by bulk copy). l sums the
-// weights as the P.V products used them (rounded to the operand type), so o / l is a
-// convex combination of the values; lx sums the unrounded fp32 weights and gives the lse.
+// Partial layout: [unit][split][head][D + 4] floats: o[0..D), m, l, lx, z (rows stay
+// 16-byte aligned so whole partial blocks can move by bulk copy). l sums the weights as
+// the P.V products used them (rounded to the operand type), so o / l is a convex
+// combination of the values; lx sums the unrounded fp32 weights and gives the lse;
+// z = sum 2^(s - m) (m - s), kept when the entropy is asked for (0 otherwise).
+//
+// Entropy and peak of the attention weights p_t = 2^(s_t - lse2), lse2 = M + log2 lx,
+// from the merged statistics of a head (M the largest score, every term of lx and z
+// taken against it): H = -sum p ln p = ln 2 (log2 lx + z / lx), every term of z being
+// non-negative (no cancellation, also for sharply peaked rows); max p = 2^(M - lse2) =
+// 1 / lx. When the running max rises from m to m' a partial sum moves to the new
+// reference as z' = 2^(m - m') (z + lx (m' - m)), lx' = 2^(m - m') lx.
 __host__ __device__ constexpr int partial_width(int D) { return D + 4; }
 
 // 2^x by the MUFU unit (ex2.approx, flush-to-zero): one instruction; -inf gives 0.
@@ -268,34 +276,52 @@ __device__ __forceinline__ float warp_sum(float v) {
 //   sm_m[h]  running max of the log2-domain scores,
 //   sm_l[h]  sum of 2^(s - m) weights as rounded for the P.V products,
 //   sm_lx[h] sum of the unrounded 2^(s - m) weights,
+//   sm_z[h]  sum of 2^(s - m) (m - s) (when the entropy is asked for),
 //   sm_v[h][e] un-normalised accumulated vector (e < DV): the output
 //            sum_t 2^(s_t - m) V_t, or the low-rank form's coefficient-space sums.
 // With one partial per unit the CTA emits it at once. Otherwise it stores its
 // partial and the last CTA of the unit to arrive merges all partials:
-// M = max m_s, l = sum 2^(m_s - M) l_s (lx likewise), v = sum 2^(m_s - M) v_s, then emits
+// M = max m_s, l = sum 2^(m_s - M) l_s (lx likewise), z = sum 2^(m_s - M) (z_s + lx_s
+// (M - m_s)), v = sum 2^(m_s - M) v_s, then emits
 // (and resets the unit's arrival counter to zero). Arrival is one acq_rel
 // atomic per CTA. The last CTA bulk-copies the unit's partials (contiguous) into
 // `stage` (free shared memory of `stage_bytes`, 16-B aligned) in one copy when
 // they fit, in chunks otherwise (0 bytes: read them directly); one warp per head
 // reduces (m, l), then every thread combines its share of the vector.
-// `emit(v, l, lx, m)` writes the unit's outputs from v [g][DV] (shared memory),
-// l[g], lx[g] and m[g]; it is called by all threads of the CTA. A unit with no tokens
-// has l = 0: its outputs are 0 and its lse is -inf.
-// sm_scratch holds at least 3 * g * count floats; sm_v is reused for the merge.
+// `emit(v, l, lx, m, z)` writes the unit's outputs from v [g][DV] (shared memory),
+// l[g], lx[g], m[g] and z[g]; it is called by all threads of the CTA. A unit with no
+// tokens has l = 0: its outputs are 0, its lse is -inf, its entropy and peak 0.
+// sm_scratch holds at least 4 * g * count floats; sm_v is reused for the merge.
 __device__ __forceinline__ float lse_of(float m, float lx) {
     return lx > 0.f ? (m + log2f(lx)) * LN2_F : NEG_INF;
+}
+
+// Writes the entropy and peak of heads head0 .. head0 + g - 1 (threads 0 .. g - 1).
+__device__ __forceinline__ void emit_entropy_peak(const DecodeArgs& a, size_t head0, const float* lx, const float* z) {
+    if (threadIdx.x >= a.g) return;
+    const float x = lx[threadIdx.x];
+    if (a.entropy != nullptr) a.entropy[head0 + threadIdx.x] = x > 0.f ? (log2f(x) + z[threadIdx.x] / x) * LN2_F : 0.f;
+    if (a.peak != nullptr) a.peak[head0 + threadIdx.x] = x > 0.f ? 1.f / x : 0.f;
+}
+
+// The weight a split or warp statistic (m, lx, z) carries in a merge against the common
+// max M, and its z moved to that reference. A statistic with m = -inf has no tokens.
+__device__ __forceinline__ float merge_factor(float m, float M) { return m != NEG_INF ? ex2_approx(m - M) : 0.f; }
+__device__ __forceinline__ float merged_z(float f, float m, float M, float lx, float z) {
+    return f != 0.f ? f * fmaf(lx, M - m, z) : 0.f;
 }
 
 struct EmitPlain {
     const DecodeArgs& a;
     int D;
     size_t head0;
-    __device__ void operator()(const float* v, const float* l, const float* lx, const float* m) const {
+    __device__ void operator()(const float* v, const float* l, const float* lx, const float* m, const float* z) const {
         for (int idx = threadIdx.x; idx < a.g * D; idx += blockDim.x) {
             const float lh = l[idx / D];
             a.out[(head0 + idx / D) * D + (idx % D)] = lh > 0.f ? v[idx] / lh : 0.f;
         }
         if (a.lse != nullptr && threadIdx.x < a.g) a.lse[head0 + threadIdx.x] = lse_of(m[threadIdx.x], lx[threadIdx.x]);
+        emit_entropy_peak(a, head0, lx, z);
     }
 };
 
@@ -303,13 +329,13 @@ struct EmitPlain {
 // MAX_GROUP * MAXDV / 128 merged values, as every caller runs at least 128 threads.
 template <int MAXDV = 128, typename Emit>
 __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int index, int count, long long slot0,
-                                   const float* sm_m, const float* sm_l, const float* sm_lx, float* sm_v,
-                                   float* sm_scratch, uint8_t* stage, int stage_bytes, const Emit& emit) {
+                                   const float* sm_m, const float* sm_l, const float* sm_lx, const float* sm_z,
+                                   float* sm_v, float* sm_scratch, uint8_t* stage, int stage_bytes, const Emit& emit) {
     const int g = a.g;
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;
     if (count == 1) {
-        emit(sm_v, sm_l, sm_lx, sm_m);
+        emit(sm_v, sm_l, sm_lx, sm_m, sm_z);
         return;
     }
     const int PD = partial_width(DV);
@@ -321,6 +347,7 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         part[tid * PD + DV] = sm_m[tid];
         part[tid * PD + DV + 1] = sm_l[tid];
         part[tid * PD + DV + 2] = sm_lx[tid];
+        part[tid * PD + DV + 3] = sm_z[tid];
     }
     // the last CTA reads the partials with a bulk copy (the async proxy): every writer
     // orders its own generic stores before that proxy before the arrival releases them
@@ -344,7 +371,8 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
     float* fm = sm_scratch;            // [n][g]: m, then the factors 2^(m - M)
     float* fl = sm_scratch + n * g;    // [n][g]: l
     float* flx = fl + n * g;           // [n][g]: lx
-    __shared__ float hm[MAX_GROUP], hl[MAX_GROUP], hlx[MAX_GROUP];
+    float* fz = flx + n * g;           // [n][g]: z
+    __shared__ float hm[MAX_GROUP], hl[MAX_GROUP], hlx[MAX_GROUP], hz[MAX_GROUP];
     __shared__ __align__(8) uint64_t mbar;
     const int chunk = stage_bytes / (per * 4);
     float* sp_buf = reinterpret_cast<float*>(stage);
@@ -373,6 +401,7 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
             fm[idx] = own ? sm_m[h] : sp_buf[sp * per + h * PD + DV];
             fl[idx] = own ? sm_l[h] : sp_buf[sp * per + h * PD + DV + 1];
             flx[idx] = own ? sm_lx[h] : sp_buf[sp * per + h * PD + DV + 2];
+            fz[idx] = own ? sm_z[h] : sp_buf[sp * per + h * PD + DV + 3];
         }
     } else {
         for (int idx = tid; idx < n * g; idx += nthr) {
@@ -382,6 +411,7 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
             fm[idx] = own ? sm_m[h] : __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV);
             fl[idx] = own ? sm_l[h] : __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 1);
             flx[idx] = own ? sm_lx[h] : __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 2);
+            fz[idx] = own ? sm_z[h] : __ldcg(base + static_cast<size_t>(sp) * per + h * PD + DV + 3);
         }
     }
     __syncthreads();
@@ -390,21 +420,24 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         float M = NEG_INF;
         for (int sp = lane; sp < n; sp += 32) M = fmaxf(M, fm[sp * g + h]);
         M = warp_max(M);
-        float L = 0.f, LX = 0.f;
+        float L = 0.f, LX = 0.f, Z = 0.f;
         for (int sp = lane; sp < n; sp += 32) {
             // a split without tokens has m = -inf and weighs nothing (also when all do)
             const float ms = fm[sp * g + h];
-            const float f = ms != NEG_INF ? ex2_approx(ms - M) : 0.f;
+            const float f = merge_factor(ms, M);
             fm[sp * g + h] = f;
             L += f * fl[sp * g + h];
             LX += f * flx[sp * g + h];
+            Z += merged_z(f, ms, M, flx[sp * g + h], fz[sp * g + h]);
         }
         L = warp_sum(L);
         LX = warp_sum(LX);
+        Z = warp_sum(Z);
         if (lane == 0) {
             hm[h] = M;
             hl[h] = L;
             hlx[h] = LX;
+            hz[h] = Z;
         }
     }
     __syncthreads();
@@ -471,17 +504,17 @@ __device__ inline void finish_unit(const DecodeArgs& a, int DV, int unit_i, int 
         if (idx < g * DV) sm_v[idx] = acc[k];
     }
     __syncthreads();
-    emit(sm_v, hl, hlx, hm);
+    emit(sm_v, hl, hlx, hm, hz);
     if (tid == 0) a.counters[unit] = 0u;
 }
 
 // Split-grid kernels: CTA (split, j, b) holds partial `split` of `a.splits` for its unit.
 __device__ inline void finish_split(const DecodeArgs& a, int D, int b, int j, int split, const float* sm_m,
-                                    const float* sm_l, const float* sm_lx, float* sm_o, float* sm_scratch,
-                                    uint8_t* stage, int stage_bytes) {
+                                    const float* sm_l, const float* sm_lx, const float* sm_z, float* sm_o,
+                                    float* sm_scratch, uint8_t* stage, int stage_bytes) {
     const int unit = b * a.Hkv + j;
     const EmitPlain emit{a, D, static_cast<size_t>(b) * a.Hq + static_cast<size_t>(j) * a.g};
-    finish_unit(a, D, unit, split, a.splits, static_cast<long long>(unit) * a.splits, sm_m, sm_l, sm_lx, sm_o,
+    finish_unit(a, D, unit, split, a.splits, static_cast<long long>(unit) * a.splits, sm_m, sm_l, sm_lx, sm_z, sm_o,
                 sm_scratch, stage, stage_bytes, emit);
 }
 

@@ -15,6 +15,7 @@ constexpr unsigned ERR_RANGE = 2u;     // a per-sequence length outside [0, cont
 
 // one split partial: o[d] (un-normalised, relative to m), m (log2 domain), l
 constexpr int MAX_SPLITS = 160;
+constexpr int F32_MAX_SPLITS = 128;   // the fp32 kernel merges from static shared memory
 constexpr int MAX_GROUP = 16;
 
 // Arguments of one decode launch (one layer). Pointers are already offset to the layer.
@@ -29,12 +30,14 @@ struct DecodeArgs {
     int B, Hq, Hkv, T, g;   // T: tokens each store holds (row stride of the cache)
     const int* lens;        // [B] tokens of each sequence (device), or nullptr: all T
     float* sscore;          // [B][Hq][T] log2-domain scaled scores for the statistics, or nullptr
+    float* entropy;         // [B][Hq] attention entropy (nats) of every head, or nullptr
+    float* peak;            // [B][Hq] largest attention weight of every head, or nullptr
     int splits;             // splits per (b, kv head)            (split-grid kernels)
     int tiles_per_split;    // token tiles per split               (split-grid kernels)
     int units;              // B * Hkv                             (balanced-grid kernels)
     int n_t;                // token tiles per unit                (balanced-grid kernels)
     float scale_log2;       // softmax scale * log2(e)
-    float* ws;              // split partials: [g][d + 4] each (o, m, l, lx, pad)
+    float* ws;              // split partials: [g][d + 4] each (o, m, l, lx, z)
     unsigned* counters;     // [B*Hkv] arrival counters, zero between launches
     unsigned* err;          // device status word
     long long wait_limit;   // clock cycles a bounded wait may spin
@@ -97,15 +100,11 @@ struct StatsArgs {
     const int* lens;        // [B] or nullptr
     float* mass;            // [B][Hkv][T] or nullptr
     float* score;           // [B][T] or nullptr
-    float* entropy;         // [B][Hq] or nullptr
-    float* peak;            // [B][Hq] or nullptr
-    float* part;            // [B][blocks][Hq][2] per-block entropy and peak partials
     unsigned* err;
     int B, Hq, Hkv, T, g;
 };
-int router_stats_blocks(int T);
-// launches the statistics kernel and, when entropy or peak is asked for, the kernel that
-// finishes them; returns the number of launches, or -1 on a launch error
+// launches the per-token statistics kernel (mass and router score); returns the number
+// of launches, or -1 on a launch error
 int launch_router_stats(const StatsArgs& a, cudaStream_t st);
 
 // Append of one new token to a low-rank cache (every basis pair, sequence and kv head).

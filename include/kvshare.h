@@ -172,11 +172,12 @@ kvshare_status kvshare_decode(kvshare_t ctx, const kvshare_cache* cache, const v
  *           rank: 8 from 7/3 times the uniform share, 16 from 9 times.
  *   entropy [L][batch][Hq] fp32: -sum_t p ln p (nats) per query head
  *   peak    [L][batch][Hq] fp32: max_t p per query head
- * Any of the four may be NULL; lse is required. The first call with an output
- * allocates a score buffer of max_batch x Hq x max_context floats and a small
- * reduction buffer in the context (KVS_ENOMEM if that fails); each layer adds one
- * statistics kernel after its decode kernel, and a second small one when entropy or
- * peak is asked for. Results are the same bits run to run. */
+ * Any of the four may be NULL; lse is required. Entropy and peak come out of the
+ * decode kernel's own online softmax and split merge (no extra pass). Mass and
+ * score need the layer's final lse: the first call asking for either allocates a
+ * score buffer of max_batch x Hq x max_context floats in the context (KVS_ENOMEM if
+ * that fails), the decode keeps every valid token's score there, and one statistics
+ * kernel per layer follows its decode kernel. Results are the same bits run to run. */
 kvshare_status kvshare_decode_stats(kvshare_t ctx, const kvshare_cache* cache, const void* q, float* out,
                                     float* lse, float* mass, float* score, float* entropy, float* peak,
                                     int l0, int l1, void* stream);

@@ -95,8 +95,8 @@ def test_stats_match_the_oracle(K, cfg, lengths):
         n0 = K.kvshare_launch_count(h)
         K.kvshare_decode_stats(h, cache, d["q"], out, lse, *st)
         assert K.kvshare_sync_status(h) == K.KVS_OK
-        # per layer: decode, statistics, and the kernel finishing entropy and peak
-        assert K.kvshare_launch_count(h) - n0 == 3 * cfg.layers
+        # per layer: the decode (entropy and peak from its merge) and the per-token statistics
+        assert K.kvshare_launch_count(h) - n0 == 2 * cfg.layers
         out2 = torch.empty_like(out)
         lse2 = torch.empty_like(lse)
         K.kvshare_decode(h, cache, d["q"], out2, lse2)
@@ -107,6 +107,46 @@ def test_stats_match_the_oracle(K, cfg, lengths):
     get = lambda name, index: ref.to_f64(inp[name][index], cfg.dtype)  # noqa: E731
     want = rr.decode_stats(cfg.layer_map, ref.to_f64(inp["q"], cfg.dtype), get, w=inp["w"], lengths=lens)
     check_stats(cfg, st, want, lens)
+
+
+@pytest.mark.parametrize("grid", [None, 7, 13], ids=["default", "grid7", "grid13"])
+@pytest.mark.parametrize("cfg", KV_CASES, ids=lambda c: c.name)
+def test_entropy_and_peak_alone_from_the_decode_merge(K, cfg, grid):
+    """Entropy and peak without mass or score: no score buffer and no statistics kernel,
+    the values come out of the decode's online softmax and its merge of warps, saved
+    unit states (straddling debug grids) and split partials (forced splits on the fp32
+    path); the same bits on a second call, and against the oracle."""
+    import torch
+    inp = cfg.make_all()
+    d = {n: to_dev(a, cfg.dtype) for n, a in inp.items()}
+    lens = np.array([1, cfg.context - 31, 77][:cfg.batch] + [5] * max(0, cfg.batch - 3), np.int32)
+    h = make_ctx(K, cfg)
+    try:
+        K.kvshare_set_map(h, cfg.layer_map, inp["w"])
+        if grid is not None:
+            if cfg.dtype == "f32":
+                K.kvshare_set_splits(h, grid)
+            else:
+                K.kvshare_debug_set_grid(h, grid)
+        cache = K.Cache(batch=cfg.batch, context=cfg.context, k=d["k"], v=d["v"], slots=cfg.slots,
+                        lengths=torch.from_numpy(lens).cuda())
+        out = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim, device="cuda")
+        lse = torch.empty(cfg.layers, cfg.batch, cfg.q_heads, device="cuda")
+        ent, peak = stats_outputs(torch, cfg)[2:]
+        n0 = K.kvshare_launch_count(h)
+        K.kvshare_decode_stats(h, cache, d["q"], out, lse, None, None, ent, peak)
+        assert K.kvshare_sync_status(h) == K.KVS_OK
+        assert K.kvshare_launch_count(h) - n0 == cfg.layers      # the decode kernels only
+        ent2, peak2 = torch.empty_like(ent), torch.empty_like(peak)
+        K.kvshare_decode_stats(h, cache, d["q"], out, lse, None, None, ent2, peak2)
+        assert K.kvshare_sync_status(h) == K.KVS_OK
+        assert torch.equal(ent, ent2) and torch.equal(peak, peak2)
+    finally:
+        K.kvshare_destroy(h)
+    get = lambda name, index: ref.to_f64(inp[name][index], cfg.dtype)  # noqa: E731
+    _, went, wpeak = rr.decode_stats(cfg.layer_map, ref.to_f64(inp["q"], cfg.dtype), get, w=inp["w"], lengths=lens)
+    assert_rel(ent.cpu().numpy(), went, "entropy", floor=1e-5)
+    assert_rel(peak.cpu().numpy(), wpeak, "peak")
 
 
 def test_stats_feed_the_packer_bit_for_bit(K):
