@@ -451,17 +451,18 @@ kvshare_status prefill_lowrank_layer(kvshare_ctx* ctx, const kvshare_cache* cach
     void* o = static_cast<uint16_t*>(out) + static_cast<size_t>(l) * per_layer * D;
     const int crows = cache->pairs * B * Hkv;
     CUtensorMap maps[6];
+    const int bn = prefill_lowrank_tile();
     if (!get_map(ctx, ctx->qp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, LR_QW, seqlen, B * Hq, 64, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B, &maps[0]) ||
         !get_map(ctx, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, seqlen, B * Hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B,
                  &maps[1]) ||
-        !get_map(ctx, cache->coef_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, seqlen, crows, 32, 64,
+        !get_map(ctx, cache->coef_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, seqlen, crows, 32, bn,
                  CU_TENSOR_MAP_SWIZZLE_NONE, &maps[2], T) ||
-        !get_map(ctx, cache->coef_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, seqlen, crows, 32, 64,
+        !get_map(ctx, cache->coef_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 32, seqlen, crows, 32, bn,
                  CU_TENSOR_MAP_SWIZZLE_NONE, &maps[3], T) ||
-        !get_map(ctx, uk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, seqlen, B * Hkv, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE,
+        !get_map(ctx, uk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, seqlen, B * Hkv, 16, bn, CU_TENSOR_MAP_SWIZZLE_NONE,
                  &maps[4], T) ||
-        !get_map(ctx, uv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, seqlen, B * Hkv, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE,
+        !get_map(ctx, uv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 16, seqlen, B * Hkv, 16, bn, CU_TENSOR_MAP_SWIZZLE_NONE,
                  &maps[5], T))
         return KVS_ECUDA;
     if (launch_lr_qproj(a, st) != cudaSuccess) return KVS_ECUDA;

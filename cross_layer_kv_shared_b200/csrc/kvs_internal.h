@@ -166,6 +166,9 @@ struct PrefillLrArgs {
 cudaError_t launch_lr_qproj(const PrefillLrArgs& a, cudaStream_t st);
 // maps: Q' [B*Hq][S][64], O [B*Hq][S][d], C_K, C_V [P*B*Hkv][T][32], U_K, U_V [B*Hkv][T][16] (the layer's)
 cudaError_t launch_prefill_lowrank(int d, const CUtensorMap* maps, const PrefillLrArgs& a, cudaStream_t st);
+// tokens per K/V tile of the low-rank prefill: the row count of its coefficient and
+// code tensor-map boxes
+int prefill_lowrank_tile();
 
 // kernel launchers (return cudaGetLastError() of the launch)
 struct TileShape { int tt; int nsw; int smem; };

@@ -29,7 +29,13 @@ namespace {
 
 constexpr int BM = 128;     // rows per query tile
 constexpr int NQ = 2;       // query tiles per CTA
-constexpr int BN = 64;      // tokens per K/V tile
+// tokens per K/V tile: 128 measured 4 % faster than 64 on the 4K-token DepthWeave
+// prefill (half as many S/P handoffs per token; ring depth and registers rebalanced)
+#ifndef KVS_LR_PF_BN
+#define KVS_LR_PF_BN 128
+#endif
+constexpr int BN = KVS_LR_PF_BN;
+static_assert(BN == 64 || BN == 128, "K/V tile of 64 or 128 tokens");
 constexpr int RB = 32;      // basis rank
 constexpr int RM = 16;      // residual slots
 constexpr int QW = LR_QW;   // operand width: RB + RM padded to one 128-byte swizzle row
@@ -37,13 +43,13 @@ constexpr int QW = LR_QW;   // operand width: RB + RM padded to one 128-byte swi
 template <int D>
 struct LrPfCfg {
     static constexpr int Q_BYTES = BM * QW * 2;        // one projected query tile [128][64] bf16
-    static constexpr int OP_TILE = BN * QW * 2;        // one K' or V' tile [64][64] bf16
-    static constexpr int NS = 3;                       // ring A: [K' | V'] stages (built by the converters)
+    static constexpr int OP_TILE = BN * QW * 2;        // one K' or V' tile [BN][64] bf16
+    static constexpr int NS = BN == 128 ? 2 : 3;       // ring A: [K' | V'] stages (built by the converters)
     static constexpr int STAGE_A = 2 * OP_TILE;
     // ring B: raw tiles [C_K | C_V | U_K | U_V], filled by TMA, freed by the converters
-    static constexpr int NSB = 4;
-    static constexpr int C_BYTES = BN * RB * 2;        // [64][32] bf16, unswizzled 64-byte rows
-    static constexpr int U_BYTES = BN * RM;            // [64][16] int8
+    static constexpr int NSB = BN == 128 ? 2 : 4;
+    static constexpr int C_BYTES = BN * RB * 2;        // [BN][32] bf16, unswizzled 64-byte rows
+    static constexpr int U_BYTES = BN * RM;            // [BN][16] int8
     static constexpr int STAGE_B = 2 * C_BYTES + 2 * U_BYTES;
     static constexpr int W_BYTES = (RB + RM) * D * 2;  // [B_V; R_V] bf16
     static constexpr int OUT_TILE = BM * D * 2;        // one output tile, 64-column swizzled halves
@@ -56,7 +62,7 @@ struct LrPfCfg {
                       C_BYTES % 128 == 0 && OFF_W % 16 == 0,
                   "TMA destinations 128-byte aligned, swizzled tiles 1024-byte aligned");
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static constexpr uint32_t TMEM_COLS = 256;         // S0 | S1 | O'0 | O'1
+    static constexpr uint32_t TMEM_COLS = BN == 128 ? 512 : 256;   // S0 | S1 | O'0 | O'1
     // converter threads: one warpgroup, each thread a whole token row of K' or V' (two
     // warpgroups that split each row measured 8% slower over the layer: more threads
     // contending for the shared-memory pipes and fewer registers for softmax)
@@ -65,8 +71,10 @@ struct LrPfCfg {
     static constexpr int W_CONV = 8;
     static constexpr int W_TMA = 8 + CONV / 32, W_MMA = W_TMA + 1;
     static constexpr int LAUNCH_REGS = 128;
-    static constexpr int REG_SOFTMAX = 184;
-    static constexpr int REG_CONV = 72;
+    // with 128-token tiles each converter thread builds two rows: registers move from
+    // the softmax (which then holds at most 64 scores of a row at a time) to the converters
+    static constexpr int REG_SOFTMAX = BN == 128 ? 168 : 184;
+    static constexpr int REG_CONV = BN == 128 ? 112 : 72;
     static constexpr int REG_CTRL = 64;
     static constexpr int REG_SUM = 2 * 128 * REG_SOFTMAX + CONV * REG_CONV + 128 * REG_CTRL;
     static_assert(REG_SUM <= THREADS * LAUNCH_REGS, "register split exceeds the launch allocation");
@@ -115,7 +123,7 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;                          // [NQ][128][64] swizzled
-    uint8_t* sA = smem + C::OFF_A;               // ring A [NS][K' | V'], each [64][64] swizzled
+    uint8_t* sA = smem + C::OFF_A;               // ring A [NS][K' | V'], each [BN][64] swizzled
     uint8_t* sB = smem + C::OFF_B;               // ring B [NSB][C_K | C_V | U_K | U_V]
     uint8_t* sW = smem + C::OFF_W;               // [B_V; R_V] [48][D] bf16
     uint8_t* sOut = smem + C::OFF_OUT;           // [NQ][D / 64][128][64] swizzled
@@ -186,26 +194,36 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const int diag0 = (q0 + qi * BM) / BN;
         float m_used = NEG_INF;
         float l = 0.f;
-        auto step = [&](auto mask_tag, int j) {
+        // one tile of S in groups of 64 columns (two 32-column TMEM loads each): with BN =
+        // 128 the row max is taken over both groups first and each group is loaded again
+        // for its weights, so a row never holds more than 64 scores in registers
+        constexpr int G64 = BN / 64;
+        auto load_group = [&](auto mask_tag, int gi, int lim, uint32_t (&r)[2][32]) {
             constexpr bool MASKED = decltype(mask_tag)::value;
-            const int lim = qpos - j * BN;               // column c is visible iff c <= lim
-            uint32_t r[BN / 32][32];
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) tc::ld32(sS + c * 32, r[c]);
+            for (int c = 0; c < 2; ++c) tc::ld32(sS + gi * 64 + c * 32, r[c]);
             tc::wait_ld();
             if (MASKED) {
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c)
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        if (c * 32 + i > lim) r[c][i] = __float_as_uint(NEG_INF);
+                        if (gi * 64 + c * 32 + i > lim) r[c][i] = __float_as_uint(NEG_INF);
             }
+        };
+        auto step = [&](auto mask_tag, int j) {
+            const int lim = qpos - j * BN;               // column c is visible iff c <= lim
+            uint32_t r[2][32];
             float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c)
+            for (int gi = 0; gi < G64; ++gi) {
+                load_group(mask_tag, gi, lim, r);
 #pragma unroll
-                for (int i = 0; i < 32; i += 2)
-                    mx[(i >> 1) & 3] = fmaxf(mx[(i >> 1) & 3], fmaxf(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])));
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2)
+                        mx[(i >> 1) & 3] = fmaxf(mx[(i >> 1) & 3], fmaxf(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])));
+            }
             const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.scale_log2;
             // lazy max: rescale O' only when the row max grew by more than 2^8
             float corr = 1.f;
@@ -230,16 +248,20 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             const float nm = -m_used;
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t pk[16];
+            for (int gi = 0; gi < G64; ++gi) {
+                if (G64 > 1) load_group(mask_tag, gi, lim, r);   // P of group 0 lands over its own S
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = tc::ex2(fmaf(__uint_as_float(r[c][2 * i]), a.scale_log2, nm));
-                    const float p1 = tc::ex2(fmaf(__uint_as_float(r[c][2 * i + 1]), a.scale_log2, nm));
-                    ls[i & 3] += p0 + p1;
-                    pk[i] = pack_bf16(p0, p1);
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = tc::ex2(fmaf(__uint_as_float(r[c][2 * i]), a.scale_log2, nm));
+                        const float p1 = tc::ex2(fmaf(__uint_as_float(r[c][2 * i + 1]), a.scale_log2, nm));
+                        ls[i & 3] += p0 + p1;
+                        pk[i] = pack_bf16(p0, p1);
+                    }
+                    tc::st16(sS + (gi * 2 + c) * 16, pk);
                 }
-                tc::st16(sS + c * 16, pk);
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         };
@@ -311,23 +333,28 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     } else if (wg >= C::W_CONV / 4 && wg < C::W_CONV / 4 + C::CONV / 128) {
         tc::reg_dec<C::REG_CONV>();
         // ------------------------------------------------------------ converters: raw tiles -> K', V'
-        // thread t: operand m (0: K', 1: V') and token row r of the tile (the whole 128-byte row)
+        // thread t: operand m (0: K', 1: V') and token rows r0 + 64 k of the tile (whole
+        // 128-byte rows)
+        constexpr int RPT = BN / 64;                     // rows per thread
         const int t = threadIdx.x - 32 * C::W_CONV;
         const int m = t >> 6;
-        const int r = t & 63;
+        const int r0 = t & 63;
         const size_t tok_row = (static_cast<size_t>(b) * a.Hkv + jkv) * a.T;
         const uint16_t* s_src = m == 0 ? a.s_k : a.s_v;
-        // the token's scale bits and rank, loaded PF tiles ahead of their use (plain loads;
+        // the tokens' scale bits and ranks, loaded PF tiles ahead of their use (plain loads;
         // the loop below is unrolled by PF so that no register with a load in flight moves)
-        constexpr int PF = 3;
-        uint32_t pf_s[PF], pf_r[PF];
-        auto meta = [&](int jj, uint32_t& sb, uint32_t& rb) {
-            const int tok = jj * BN + r;
-            sb = 0u;
-            rb = 0u;
-            if (jj < n_kv && tok < a.S) {                // rows past the sequence stay zero
-                sb = s_src[tok_row + tok];
-                rb = a.rank[static_cast<size_t>(b) * a.T + tok];
+        constexpr int PF = BN == 128 ? 2 : 3;     // 256 or 192 tokens ahead
+        uint32_t pf_s[PF][RPT], pf_r[PF][RPT];
+        auto meta = [&](int jj, uint32_t (&sb)[RPT], uint32_t (&rb)[RPT]) {
+#pragma unroll
+            for (int k = 0; k < RPT; ++k) {
+                const int tok = jj * BN + r0 + 64 * k;
+                sb[k] = 0u;
+                rb[k] = 0u;
+                if (jj < n_kv && tok < a.S) {            // rows past the sequence stay zero
+                    sb[k] = s_src[tok_row + tok];
+                    rb[k] = a.rank[static_cast<size_t>(b) * a.T + tok];
+                }
             }
         };
 #pragma unroll
@@ -339,42 +366,61 @@ prefill_lowrank_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             if (j >= n_kv) break;
             const int s = j % NS;
             const int sb = j % NSB;
-            const float scale = __half2float(__ushort_as_half(static_cast<unsigned short>(pf_s[q])));
-            const int rk = static_cast<int>(pf_r[q]);
+            float scale[RPT];
+            int rkv[RPT];
+#pragma unroll
+            for (int k = 0; k < RPT; ++k) {
+                scale[k] = __half2float(__ushort_as_half(static_cast<unsigned short>(pf_s[q][k])));
+                rkv[k] = static_cast<int>(pf_r[q][k]);
+            }
             meta(j + PF, pf_s[q], pf_r[q]);
-            // where the token's codes start in its 32-token code group: after the codes of
+            // where a token's codes start in its 32-token code group: after the codes of
             // the group's earlier tokens (the converters exchange the tile's code lengths)
-            if (m == 0) conv_len[j & 1][r] = code_len(static_cast<unsigned>(rk));
+            if (m == 0) {
+#pragma unroll
+                for (int k = 0; k < RPT; ++k) conv_len[j & 1][r0 + 64 * k] = code_len(static_cast<unsigned>(rkv[k]));
+            }
             named_sync(3, C::CONV);
-            int o = 0;
-            for (int i = r & ~31; i < r; ++i) o += conv_len[j & 1][i];
+            int ov[RPT];
+#pragma unroll
+            for (int k = 0; k < RPT; ++k) {
+                const int r = r0 + 64 * k;
+                ov[k] = 0;
+                for (int i = r & ~31; i < r; ++i) ov[k] += conv_len[j & 1][i];
+            }
             wait_lr(sy, &sy.raw_full[sb], (j / NSB) & 1, a.wait_limit, a.err);
             if (j >= NS) wait_lr(sy, &sy.op_empty[s], ((j / NS) - 1) & 1, a.wait_limit, a.err);
             const uint8_t* raw = sB + sb * C::STAGE_B;
             uint8_t* op = sA + s * C::STAGE_A + m * C::OP_TILE;
-            {
-                // chunks 0-3: the 32 coefficients, copied into the swizzled row
-                const uint4* src = reinterpret_cast<const uint4*>(raw + m * C::C_BYTES + r * (RB * 2));
 #pragma unroll
-                for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(op + swz128(r, c)) = src[c];
-            }
-            {
-                // chunks 4-5: s * u for the first r_t codes (exact product, one bf16 rounding); 6-7: zero
-                const uint4 w = codes_at(raw + 2 * C::C_BYTES + m * C::U_BYTES + (r & ~31) * RM + o);
-                const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-                uint32_t pk[8];
+            for (int k = 0; k < RPT; ++k) {
+                const int r = r0 + 64 * k;
+                const int rk = rkv[k];
+                const int o = ov[k];
+                {
+                    // chunks 0-3: the 32 coefficients, copied into the swizzled row
+                    const uint4* src = reinterpret_cast<const uint4*>(raw + m * C::C_BYTES + r * (RB * 2));
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int c0 = 2 * i, c1 = 2 * i + 1;
-                    const int x0 = static_cast<int8_t>((words[c0 >> 2] >> (8 * (c0 & 3))) & 0xffu);
-                    const int x1 = static_cast<int8_t>((words[c1 >> 2] >> (8 * (c1 & 3))) & 0xffu);
-                    pk[i] = pack_bf16(c0 < rk ? static_cast<float>(x0) * scale : 0.f,
-                                      c1 < rk ? static_cast<float>(x1) * scale : 0.f);
+                    for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(op + swz128(r, c)) = src[c];
                 }
-                *reinterpret_cast<uint4*>(op + swz128(r, 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(op + swz128(r, 5)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                *reinterpret_cast<uint4*>(op + swz128(r, 6)) = make_uint4(0u, 0u, 0u, 0u);
-                *reinterpret_cast<uint4*>(op + swz128(r, 7)) = make_uint4(0u, 0u, 0u, 0u);
+                {
+                    // chunks 4-5: s * u for the first r_t codes (exact product, one bf16 rounding); 6-7: zero
+                    const uint4 w = codes_at(raw + 2 * C::C_BYTES + m * C::U_BYTES + (r & ~31) * RM + o);
+                    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int c0 = 2 * i, c1 = 2 * i + 1;
+                        const int x0 = static_cast<int8_t>((words[c0 >> 2] >> (8 * (c0 & 3))) & 0xffu);
+                        const int x1 = static_cast<int8_t>((words[c1 >> 2] >> (8 * (c1 & 3))) & 0xffu);
+                        pk[i] = pack_bf16(c0 < rk ? static_cast<float>(x0) * scale[k] : 0.f,
+                                          c1 < rk ? static_cast<float>(x1) * scale[k] : 0.f);
+                    }
+                    *reinterpret_cast<uint4*>(op + swz128(r, 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4*>(op + swz128(r, 5)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    *reinterpret_cast<uint4*>(op + swz128(r, 6)) = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(op + swz128(r, 7)) = make_uint4(0u, 0u, 0u, 0u);
+                }
             }
             fence_proxy_async();
             mbar_arrive(&sy.op_ready[s]);
@@ -570,6 +616,8 @@ cudaError_t launch_lr_one(const CUtensorMap* maps, const PrefillLrArgs& a, cudaS
 }
 
 }  // namespace
+
+int prefill_lowrank_tile() { return BN; }
 
 cudaError_t launch_lr_qproj(const PrefillLrArgs& a, cudaStream_t st) {
     dim3 grid(a.Hq, a.B, (a.S + QP_ROWS - 1) / QP_ROWS);
