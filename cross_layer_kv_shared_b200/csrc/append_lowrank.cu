@@ -13,9 +13,10 @@
 //   codes, scale of u_a at the rank the router gives the token in layer a
 // Every dot product runs in fp32 from index 0 up, each product and each sum
 // correctly rounded (no fused multiply-add), so the bf16 coefficients and the
-// integer codes are reproducible bit for bit. One CTA per (pair, sequence, kv head);
-// it first copies the pair's basis and both layers' residual factors into shared
-// memory (one coalesced pass), then walks them there.
+// integer codes are reproducible bit for bit. One CTA per (pair, sequence, kv head,
+// K or V): the two sides' dependent chains run side by side on different SMs. A CTA
+// first copies the pair's basis and both layers' residual factors into shared memory
+// (one coalesced pass), then walks them there.
 #include "kvs_quant.cuh"
 
 namespace kvs {
@@ -30,7 +31,8 @@ __device__ __forceinline__ float bf(uint16_t v) { return __uint_as_float(static_
 __global__ void __launch_bounds__(NT) append_lowrank_kernel(const AppendArgs a) {
     const int p = blockIdx.x;
     const int b = blockIdx.y;
-    const int j = blockIdx.z;
+    const int j = blockIdx.z >> 1;
+    const int side = blockIdx.z & 1;                      // 0: K, 1: V
     const int tid = threadIdx.x;
     const int la = a.pair_layers[2 * p], lb = a.pair_layers[2 * p + 1];
     if (la < 0) return;                                   // a pair no layer reads
@@ -46,7 +48,7 @@ __global__ void __launch_bounds__(NT) append_lowrank_kernel(const AppendArgs a) 
     const size_t BHkv = static_cast<size_t>(a.B) * a.Hkv;
     const size_t bj = static_cast<size_t>(b) * a.Hkv + j;
     const int rows = RB + nl * QUANT_RM;
-    for (int side = 0; side < 2; ++side) {                 // K, then V
+    {
         const uint16_t* nw = side == 0 ? a.k_new : a.v_new;
         const uint16_t* basis = (side == 0 ? a.basis_k : a.basis_v) + (static_cast<size_t>(p) * a.Hkv + j) * RB * D;
         const uint16_t* Rf = side == 0 ? a.r_k : a.r_v;
@@ -131,14 +133,13 @@ __global__ void __launch_bounds__(NT) append_lowrank_kernel(const AppendArgs a) 
             (side == 0 ? a.s_k : a.s_v)[row] = sc;
             if (side == 0 && j == 0) a.rank[(static_cast<size_t>(l) * a.B + b) * a.T + t] = r;
         }
-        __syncthreads();
     }
 }
 
 }  // namespace
 
 cudaError_t launch_append_lowrank(const AppendArgs& a, cudaStream_t st) {
-    dim3 grid(a.P, a.B, a.Hkv);
+    dim3 grid(a.P, a.B, 2 * a.Hkv);
     // at most (128 + 32) rows of LDB bf16 (41.6 KB), with the static arrays under 48 KB
     const size_t smem = static_cast<size_t>(a.Rb + 2 * QUANT_RM) * LDB * sizeof(uint16_t);
     append_lowrank_kernel<<<grid, NT, smem, st>>>(a);
