@@ -1,10 +1,13 @@
 // Split-KV GQA decode over a shared cache, bf16 storage, forms SINGLE and MIX.
 //
 // Balanced split scheduling: the (batch, kv head) units' token tiles form one
-// flat list of units * n_t tiles that is cut into G equal ranges, one per CTA
-// (G = the CTAs resident at once, one per SM), so every SM streams the same
-// number of bytes whatever the batch. A range covers at most two units; each
-// unit's partial results merge in the last CTA to finish it.
+// flat list of units * n_t tiles that is cut into G equal ranges, one per CTA.
+// By default G is a whole number of CTAs per unit, as many as are resident at
+// once, so no range crosses a unit (the STRADDLE = false instance); any other G
+// is handled too, a range then covering at most two units. Each unit's partial
+// results merge in the last CTA to finish it. When the entropy is asked for, the
+// online softmax also carries z = sum 2^(s - m) (m - s) through every merge (the
+// ENT instance), so entropy and peak need no pass over the scores.
 // Inside a CTA, NW warps each own a private ring of NSW shared-memory stages
 // and stream every NW-th tile of the range into it with TMA (128-byte swizzle),
 // re-issuing a stage as soon as it is consumed. Per tile and warp, with the

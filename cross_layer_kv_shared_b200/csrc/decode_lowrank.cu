@@ -12,7 +12,8 @@
 //   c^ = sum_t p_t C_V[t],   u^ = sum_t p_t s_V[t] U_V[t],   o = (c^ B_V + u^ R_V) / sum_t p_t
 // This is the "basis lookup, residual dequantisation and attention projection in
 // a single pass" the DepthWeave pages describe, restated for sm_100a:
-//   - TMA streams coefficient tiles (64/128-B swizzle) and int8 code tiles per warp;
+//   - TMA streams coefficient tiles (64/128-B swizzle) per warp, and bulk copies
+//     bring each 32-token group's used code bytes (group-packed codes);
 //   - q~ = B_K q and q^ = R_K q are split into bf16 hi + lo halves so the score
 //     MMAs (mma.sync m16n8k16) keep ~16 bits of the fp32 projection;
 //   - tokens are the MMA's M rows and the g heads its N columns (S^T = C q~^T),
@@ -20,7 +21,10 @@
 //     PV MMAs through an in-register transpose (movmatrix);
 //   - int8 codes convert exactly to f16 operands, masked by the token's rank;
 //   - c^ and u^ accumulate in fp32 MMA accumulators; split partials stay in this
-//     coefficient space and the CTA that merges a unit projects it once.
+//     coefficient space and the CTA that merges a unit projects it once;
+//   - when the entropy is asked for, the online softmax also carries
+//     z = sum 2^(s - m) (m - s) through the warp and split merges (a separate
+//     compiled instance), so entropy and peak need no pass over the scores.
 #include "kvs_quant.cuh"
 
 namespace kvs {
