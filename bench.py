@@ -48,8 +48,8 @@ METRIC = "decode tok/s and KV GB/s (% of HBM peak); prefill TFLOP/s, 1×B200"
 # (ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
 #  --cache-control none --clock-control none -k regex:decode_bf16 -s 88 -c 22
 #  python bench.py --steps 1 --warmup 3 --no-secondary --no-cpu-baseline):
-# 67,255,273 B read + 1,422,068 B written
-NCU_TRAFFIC_BYTES = {"cla2_1p1b": 68677341}
+# 67,244,079 B read + 953,519 B written
+NCU_TRAFFIC_BYTES = {"cla2_1p1b": 68197597}
 
 
 def load_peaks():
