@@ -49,12 +49,13 @@ __global__ void __launch_bounds__(NT, 4) router_stats_kernel(const StatsArgs a) 
     int hg = 0, j = 0;                                   // run-time grouping (G == 0): head j g + hg
     for (int h0 = 0; h0 < a.Hq; h0 += HC) {
         const int hn = min(HC, a.Hq - h0);
-        if (threadIdx.x < hn) lse2_s[threadIdx.x] = a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] * LOG2E_F;
-        __syncthreads();
-        // every score of the pass first, all loads in flight together
+        // every score of the pass first, all loads in flight together (and in flight
+        // while the heads' lse values are fetched and shared)
         float sv[HC];
 #pragma unroll
         for (int q = 0; q < HC; ++q) sv[q] = (q < hn && live) ? __ldcs(srow + static_cast<size_t>(h0 + q) * a.T) : 0.f;
+        if (threadIdx.x < hn) lse2_s[threadIdx.x] = a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] * LOG2E_F;
+        __syncthreads();
         // the weights, summed per kv head in head order
 #pragma unroll
         for (int q = 0; q < HC; ++q) {
